@@ -1,0 +1,369 @@
+"""Python binding of libhga.so, the sm_100a library for HGA routed
+exact-token attention (the C ABI is include/hga.h).
+
+This module only marshals torch tensors into the C calls: it checks device,
+dtype, shape and contiguity, passes data pointers, sizes and the current
+CUDA stream, and raises on a non-OK status.  Every step of the computation
+runs in the library's CUDA kernels; there is no CPU fallback, and every call
+fails loudly if the library is missing or no CUDA device is present.
+
+Function names follow the C ABI: hga_build_summaries, hga_route, hga_attend,
+hga_forward (prefill and decode), hga_workspace_size.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "hga_route",
+           "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
+           "hga_workspace_size", "HGAError", "PREFILL", "DECODE"]
+
+PREFILL, DECODE = 0, 1
+_F32, _BF16 = 0, 1
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libhga.so")
+_lib = None
+_lock = threading.Lock()
+
+
+class HGAError(RuntimeError):
+    pass
+
+
+# ------------------------------------------------------------ C structs --
+
+class _Params(ctypes.Structure):
+    _fields_ = [("C", ctypes.c_int32), ("g_s", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("K_c", ctypes.c_int32), ("K_g", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double), ("hf_wavelength", ctypes.c_double)]
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("capacity", ctypes.c_int32), ("k_rot", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p), ("k_open", ctypes.c_void_p),
+                ("s_chunk", ctypes.c_void_p), ("s_group", ctypes.c_void_p),
+                ("lens", ctypes.c_void_p)]
+
+
+class _IO(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p), ("q_new", ctypes.c_void_p), ("k_new", ctypes.c_void_p),
+                ("v_new", ctypes.c_void_p), ("pos_new", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("lse", ctypes.c_void_p), ("sel_chunk", ctypes.c_void_p),
+                ("sel_group", ctypes.c_void_p), ("cache", _Cache)]
+
+
+@dataclasses.dataclass(frozen=True)
+class HGAParams:
+    """Method parameters (page section 3; setup table of section 6)."""
+    C: int = 64
+    g_s: int = 16
+    F: int = 2
+    L: int = 8
+    K_c: int = 16
+    K_g: int = 32
+    rope_theta: float = 1e6
+    hf_wavelength: float = 0.0   # <= 0: the chunk length C
+
+    def c(self) -> _Params:
+        return _Params(self.C, self.g_s, self.F, self.L, self.K_c, self.K_g,
+                       float(self.rope_theta), float(self.hf_wavelength))
+
+
+# ------------------------------------------------------------- loading --
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libhga.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise HGAError(f"{_LIB_PATH} is missing: build it with "
+                           "hierarchical_kv_routing_b200._build.build()")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        lib.hga_build_summaries.argtypes = [P, P, P, P, P, P, P, P]
+        lib.hga_route.argtypes = [P, P, P, P, P, P, P, P, P]
+        lib.hga_attend.argtypes = [P, P, P, P, P, P, P, P, P, P]
+        lib.hga_workspace_size.argtypes = [ctypes.c_int, P, P]
+        lib.hga_workspace_size.restype = ctypes.c_size_t
+        lib.hga_forward.argtypes = [ctypes.c_int, P, P, P, P, ctypes.c_size_t, P]
+        lib.hga_status_string.argtypes = [ctypes.c_int]
+        lib.hga_status_string.restype = ctypes.c_char_p
+        lib.hga_last_cuda_error.restype = ctypes.c_int
+        for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        lib = load()
+        msg = lib.hga_status_string(status).decode()
+        extra = ""
+        if status == 3:
+            extra = f" (cuda error {lib.hga_last_cuda_error()})"
+        raise HGAError(f"{what}: {msg}{extra}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return _F32
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    raise HGAError(f"unsupported dtype {t.dtype}: float32 or bfloat16")
+
+
+def _need(t: torch.Tensor, name: str, shape=None, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise HGAError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise HGAError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise HGAError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise HGAError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise HGAError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _dims(B, T, Hq, Hkv, D, dtype_code) -> _Dims:
+    return _Dims(B, T, Hq, Hkv, D, dtype_code)
+
+
+# --------------------------------------------------------------- calls --
+
+def hga_build_summaries(k_raw: torch.Tensor, pos: torch.Tensor, params: HGAParams, *,
+                        k_rot: Optional[torch.Tensor] = None, s_chunk=None, s_group=None,
+                        want_k_rot: bool = True, stream=None):
+    """Stage 1.  k_raw [B,T,Hkv,D] -> (k_rot [B,T,Hkv,D] or None,
+    s_chunk [B,Hkv,T/C,D] f32, s_group [B,Hkv,(T/C)*(C/g_s),D] f32)."""
+    lib = load()
+    _need(k_raw, "k_raw")
+    B, T, Hkv, D = k_raw.shape
+    _need(pos, "pos", (B, T), torch.int32)
+    NC = T // params.C
+    dev = k_raw.device
+    if k_rot is None and want_k_rot:
+        k_rot = torch.empty_like(k_raw)
+    if s_chunk is None:
+        s_chunk = torch.empty(B, Hkv, NC, D, device=dev, dtype=torch.float32)
+    if s_group is None:
+        s_group = torch.empty(B, Hkv, NC * (params.C // params.g_s), D, device=dev,
+                              dtype=torch.float32)
+    dims = _dims(B, T, Hkv, Hkv, D, _dtype_code(k_raw))
+    pc = params.c()
+    st = lib.hga_build_summaries(ctypes.byref(dims), ctypes.byref(pc), _ptr(k_raw), _ptr(pos),
+                                 _ptr(k_rot), _ptr(s_chunk), _ptr(s_group), _stream(stream))
+    _check(st, "hga_build_summaries")
+    return k_rot, s_chunk, s_group
+
+
+def hga_route(q: torch.Tensor, pos: torch.Tensor, s_chunk: torch.Tensor, s_group: torch.Tensor,
+              params: HGAParams, *, sel_chunk=None, sel_group=None, stream=None):
+    """Stage 2.  q [B,T,Hq,D] -> sel_chunk [B,NB,Hkv,K_c], sel_group [B,NB,Hkv,K_g]."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    Hkv = s_chunk.shape[1]
+    _need(pos, "pos", (B, T), torch.int32)
+    _need(s_chunk, "s_chunk", dtype=torch.float32)
+    _need(s_group, "s_group", dtype=torch.float32)
+    NB = (T + params.C - 1) // params.C
+    if sel_chunk is None:
+        sel_chunk = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
+    if sel_group is None:
+        sel_group = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    st = lib.hga_route(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(s_chunk),
+                       _ptr(s_group), _ptr(sel_chunk), _ptr(sel_group), _stream(stream))
+    _check(st, "hga_route")
+    return sel_chunk, sel_group
+
+
+def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch.Tensor,
+               sel_group: torch.Tensor, params: HGAParams, *, out=None, want_lse: bool = False,
+               lse=None, stream=None):
+    """Stage 3.  -> out [B,T,Hq,D] (and lse [B,Hq,T] f32 when asked)."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    Hkv = k_rot.shape[2]
+    _need(k_rot, "k_rot", (B, T, Hkv, D), q.dtype)
+    _need(v, "v", (B, T, Hkv, D), q.dtype)
+    _need(pos, "pos", (B, T), torch.int32)
+    _need(sel_group, "sel_group", dtype=torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    st = lib.hga_attend(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(k_rot),
+                        _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "hga_attend")
+    return (out, lse) if want_lse or lse is not None else out
+
+
+def hga_workspace_size(mode: int, B: int, T: int, Hq: int, Hkv: int, D: int, dtype,
+                       params: HGAParams) -> int:
+    lib = load()
+    code = _F32 if dtype in (torch.float32, "f32") else _BF16
+    dims = _dims(B, T, Hq, Hkv, D, code)
+    pc = params.c()
+    return int(lib.hga_workspace_size(mode, ctypes.byref(dims), ctypes.byref(pc)))
+
+
+class KVCache:
+    """Decode state for `capacity` tokens per sequence (caller-owned device
+    memory, laid out as hga_kv_cache in include/hga.h)."""
+
+    def __init__(self, B: int, capacity: int, Hkv: int, D: int, dtype, params: HGAParams,
+                 device="cuda"):
+        if capacity % params.C:
+            raise HGAError("capacity must be a multiple of C")
+        self.B, self.capacity, self.Hkv, self.D, self.dtype = B, capacity, Hkv, D, dtype
+        self.params = params
+        z = dict(device=device)
+        self.k_rot = torch.zeros(B, capacity, Hkv, D, dtype=dtype, **z)
+        self.v = torch.zeros(B, capacity, Hkv, D, dtype=dtype, **z)
+        self.pos = torch.zeros(B, capacity, dtype=torch.int32, **z)
+        self.k_open = torch.zeros(B, Hkv, params.C, D, dtype=dtype, **z)
+        self.s_chunk = torch.zeros(B, Hkv, capacity // params.C, D, dtype=torch.float32, **z)
+        self.s_group = torch.zeros(B, Hkv, capacity // params.g_s, D, dtype=torch.float32, **z)
+        self.lens = torch.zeros(B, dtype=torch.int32, **z)
+
+    def c(self) -> _Cache:
+        return _Cache(self.capacity, self.k_rot.data_ptr(), self.v.data_ptr(), self.pos.data_ptr(),
+                      self.k_open.data_ptr(), self.s_chunk.data_ptr(), self.s_group.data_ptr(),
+                      self.lens.data_ptr())
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor], zero: bool):
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise HGAError(f"workspace too small: need {nbytes} bytes")
+        return workspace
+    w = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+    if zero:
+        w.zero_()
+    return w
+
+
+def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCache] = None,
+                        out=None, want_lse=False, want_sel=False, workspace=None, stream=None):
+    """Stages 1-3 in one call.  Returns dict(out, lse?, sel_chunk?, sel_group?)."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _need(k, "k", (B, T, Hkv, D), q.dtype)
+    _need(v, "v", (B, T, Hkv, D), q.dtype)
+    _need(pos, "pos", (B, T), torch.int32)
+    NB = (T + params.C - 1) // params.C
+    res = {"out": torch.empty_like(q) if out is None else out}
+    io = _IO()
+    io.q, io.k, io.v, io.pos = q.data_ptr(), k.data_ptr(), v.data_ptr(), pos.data_ptr()
+    io.out = res["out"].data_ptr()
+    if want_lse:
+        res["lse"] = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+        io.lse = res["lse"].data_ptr()
+    if want_sel:
+        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+        io.sel_chunk = res["sel_chunk"].data_ptr()
+        io.sel_group = res["sel_group"].data_ptr()
+    if cache is not None:
+        io.cache = cache.c()
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    nbytes = int(lib.hga_workspace_size(PREFILL, ctypes.byref(dims), ctypes.byref(pc)))
+    ws = _workspace(nbytes, q.device, workspace, zero=False)
+    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
+    st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    _check(st, "hga_forward(prefill)")
+    return res
+
+
+def hga_forward_decode(q_new, k_new, v_new, pos_new, cache: KVCache, params: HGAParams, *,
+                       out=None, want_lse=False, want_sel=False, workspace=None, stream=None):
+    """One decode step per sequence.  q_new [B,Hq,D], k_new/v_new [B,Hkv,D],
+    pos_new [B] int32.  `workspace` must come from decode_workspace() (zeroed
+    once) when given.  Returns dict(out, lse?, sel_chunk?, sel_group?)."""
+    lib = load()
+    _need(q_new, "q_new")
+    B, Hq, D = q_new.shape
+    Hkv = k_new.shape[1]
+    _need(k_new, "k_new", (B, Hkv, D), q_new.dtype)
+    _need(v_new, "v_new", (B, Hkv, D), q_new.dtype)
+    _need(pos_new, "pos_new", (B,), torch.int32)
+    res = {"out": torch.empty_like(q_new) if out is None else out}
+    io = _IO()
+    io.q_new, io.k_new, io.v_new = q_new.data_ptr(), k_new.data_ptr(), v_new.data_ptr()
+    io.pos_new = pos_new.data_ptr()
+    io.out = res["out"].data_ptr()
+    if want_lse:
+        res["lse"] = torch.empty(B, Hq, device=q_new.device, dtype=torch.float32)
+        io.lse = res["lse"].data_ptr()
+    if want_sel:
+        res["sel_chunk"] = torch.empty(B, Hkv, params.K_c, device=q_new.device, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, Hkv, params.K_g, device=q_new.device, dtype=torch.int32)
+        io.sel_chunk = res["sel_chunk"].data_ptr()
+        io.sel_group = res["sel_group"].data_ptr()
+    io.cache = cache.c()
+    dims = _dims(B, cache.capacity, Hq, Hkv, D, _dtype_code(q_new))
+    pc = params.c()
+    nbytes = int(lib.hga_workspace_size(DECODE, ctypes.byref(dims), ctypes.byref(pc)))
+    ws = _workspace(nbytes, q_new.device, workspace, zero=True)
+    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
+    st = lib.hga_forward(DECODE, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    _check(st, "hga_forward(decode)")
+    return res
+
+
+def decode_workspace(B, capacity, Hq, Hkv, D, dtype, params: HGAParams, device="cuda"):
+    """A zero-filled decode workspace (reusable across steps)."""
+    n = hga_workspace_size(DECODE, B, capacity, Hq, Hkv, D, dtype, params)
+    return torch.zeros(max(n, 1) + 256, dtype=torch.uint8, device=device)
+
+
+def hga_forward(mode: int, *args, **kw):
+    """hga_forward(PREFILL, q, k, v, pos, params, ...) or
+    hga_forward(DECODE, q_new, k_new, v_new, pos_new, cache, params, ...)."""
+    if mode == PREFILL:
+        return hga_forward_prefill(*args, **kw)
+    if mode == DECODE:
+        return hga_forward_decode(*args, **kw)
+    raise HGAError(f"unknown mode {mode}")

@@ -1,0 +1,196 @@
+/*
+ * hga.h — C ABI of the B200 (sm_100a) library for Hierarchical Global
+ * Attention (HGA): routed exact-token causal attention.
+ *
+ * Sources.  The operations follow the HGA paper-review page ("HGA:
+ * Hierarchical Global Attention — Drop-In Exact-Token Routing for Pretrained
+ * Long-Context Transformers", xllm-io), section 3 (技术架构): the mixed-RoPE
+ * summary formula, the routing policy (deterministic visibility, middle
+ * routing, the selection equation M_sel = topK_c, G_sel = topK_g), exact
+ * token output attention (eq. (1) restricted to the routed set) and the
+ * store's four operations (append closed chunk, read chunk summaries, fetch
+ * group summaries, gather token K/V, section "三层 K/V 存储").  The
+ * gist.science page "Hierarchical Global Attention (HGA)", technical summary,
+ * "Core Mechanism", restates the same mechanism.
+ *
+ * Conventions for every call.
+ *  - Pointers are DEVICE pointers (cudaMalloc / PyTorch CUDA memory) unless a
+ *    comment says host.  The caller owns every buffer; the library allocates
+ *    nothing and keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued asynchronously; no call synchronises the host
+ *    except where stated.
+ *  - Layouts are dense row-major with the last index fastest:
+ *      Q, O      [B, T, Hq,  D]      query head hq uses KV head hq / (Hq/Hkv)
+ *      K, V, K_rot [B, T, Hkv, D]    K is the RAW (pre-RoPE) key projection
+ *      pos       [B, T] int32        RoPE positions (any values; causality
+ *                                    follows the token index, not pos)
+ *      s_chunk   [B, Hkv, NC, D] f32 NC = T / C closed chunks (a partial last
+ *                                    chunk is open and has no summary)
+ *      s_group   [B, Hkv, NC*C/g_s, D] f32, group j of chunk m at m*C/g_s + j
+ *      sel_chunk [B, NB, Hkv, K_c] int32, NB = ceil(T / C) query blocks
+ *      sel_group [B, NB, Hkv, K_g] int32 global group ids
+ *      lse       [B, Hq, T] f32      natural-log softmax denominators
+ *    Selected ids are ascending and padded with -1.
+ *  - dtype (hga_dims.dtype) is the element type of Q, K, V, K_rot and O:
+ *    HGA_F32 or HGA_BF16.  Summaries, scores and accumulation are fp32 or
+ *    wider.
+ *  - Errors: arguments are checked on the host first; a failing check
+ *    returns HGA_ERR_INVALID_ARG or HGA_ERR_UNSUPPORTED and launches nothing.
+ *    A launch failure returns HGA_ERR_CUDA (the CUDA error is not cleared by
+ *    the library; hga_last_cuda_error() gives its code).
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hga_status {
+    HGA_OK = 0,
+    HGA_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size or a bad layout */
+    HGA_ERR_UNSUPPORTED = 2,   /* valid, but not a shape this build handles  */
+    HGA_ERR_CUDA = 3,          /* a CUDA launch or copy failed               */
+    HGA_ERR_TIMEOUT = 4,       /* a bounded device wait gave up              */
+    HGA_ERR_BOUNDS = 5,        /* a device-side index check failed           */
+    HGA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} hga_status;
+
+typedef enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
+
+typedef enum hga_mode { HGA_PREFILL = 0, HGA_DECODE = 1 } hga_mode;
+
+/* Method parameters (page section 3 and its setup table in section 6). */
+typedef struct hga_params {
+    int32_t C;            /* chunk length in tokens; this build needs C == 64,
+                             which is also the prefill query block            */
+    int32_t g_s;          /* group length; divides C                          */
+    int32_t F;            /* sink chunks 0..F-1, always visible               */
+    int32_t L;            /* recent closed chunks, always visible; with L == 0
+                             the previous chunk is still forced visible       */
+    int32_t K_c;          /* middle chunks routed per block and KV head (>=0) */
+    int32_t K_g;          /* groups opened inside those chunks (>= 0)         */
+    double rope_theta;    /* RoPE base: omega_i = theta^(-2i/D), pair (i, i+D/2) */
+    double hf_wavelength; /* pair i is high-frequency iff 2*pi/omega_i is below
+                             this; <= 0 selects C; +inf makes every pair high */
+} hga_params;
+
+/* Problem shape. */
+typedef struct hga_dims {
+    int32_t B;      /* sequences                                              */
+    int32_t T;      /* prefill: tokens per sequence; decode: cache capacity   */
+    int32_t Hq;     /* query heads, a multiple of Hkv                         */
+    int32_t Hkv;    /* key/value heads                                        */
+    int32_t D;      /* head dimension: 64 or 128                              */
+    int32_t dtype;  /* hga_dtype                                              */
+} hga_dims;
+
+/* Decode state, all device memory owned by the caller, for `capacity` tokens
+ * per sequence (Tc below; a multiple of C).  hga_forward(HGA_PREFILL) fills
+ * it when io.cache.k_rot is non-NULL; every hga_forward(HGA_DECODE) appends
+ * one token per sequence and increments lens. */
+typedef struct hga_kv_cache {
+    int32_t capacity;  /* Tc                                                  */
+    void *k_rot;       /* [B, Tc, Hkv, D] rotated keys                        */
+    void *v;           /* [B, Tc, Hkv, D] values                              */
+    int32_t *pos;      /* [B, Tc] positions of the cached tokens              */
+    void *k_open;      /* [B, Hkv, C, D] raw keys of each sequence's open chunk
+                          (needed for the low-frequency pairs when it closes) */
+    float *s_chunk;    /* [B, Hkv, Tc/C, D]                                   */
+    float *s_group;    /* [B, Hkv, Tc/g_s, D]                                 */
+    int32_t *lens;     /* [B] tokens already cached                           */
+} hga_kv_cache;
+
+/* Inputs and outputs of hga_forward.  Unused members must be NULL. */
+typedef struct hga_io {
+    /* HGA_PREFILL */
+    const void *q;             /* [B, T, Hq, D]                                */
+    const void *k;             /* [B, T, Hkv, D] raw keys                      */
+    const void *v;             /* [B, T, Hkv, D]                               */
+    const int32_t *pos;        /* [B, T]                                       */
+    /* HGA_DECODE: one new token per sequence, at index lens[b]               */
+    const void *q_new;         /* [B, Hq, D]                                   */
+    const void *k_new;         /* [B, Hkv, D] raw key                          */
+    const void *v_new;         /* [B, Hkv, D]                                  */
+    const int32_t *pos_new;    /* [B]                                          */
+    /* outputs */
+    void *out;                 /* prefill [B, T, Hq, D]; decode [B, Hq, D]     */
+    float *lse;                /* optional: prefill [B, Hq, T]; decode [B, Hq] */
+    int32_t *sel_chunk;        /* optional: prefill [B, NB, Hkv, K_c];
+                                  decode [B, Hkv, K_c]                         */
+    int32_t *sel_group;        /* optional: prefill [B, NB, Hkv, K_g];
+                                  decode [B, Hkv, K_g]                         */
+    hga_kv_cache cache;        /* decode: required; prefill: optional output   */
+} hga_io;
+
+/* Stage 1 — rotate keys and build mixed-RoPE summaries ("append closed
+ * chunk").  Page section 3, "Mixed-RoPE Routing Summaries": for each closed
+ * chunk and each g_s-token group, high-frequency pairs are the mean of the
+ * per-token rotated keys; low-frequency pairs are the mean raw key rotated at
+ * the set's mean position.  Also writes K_rot = RoPE(K) for attention.
+ * k_rot may be NULL (summaries only).  Shapes as in the header comment. */
+hga_status hga_build_summaries(const hga_dims *dims, const hga_params *prm,
+                               const void *k_raw, const int32_t *pos,
+                               void *k_rot, float *s_chunk, float *s_group,
+                               void *stream);
+
+/* Stage 2 — two-level routing per 64-token query block and KV head.  Page
+ * section 3, "路由策略" (routing policy) and the selection equation: the
+ * routing query is the block's RoPE-rotated queries summed over its tokens and
+ * over the KV head's query heads; middle chunks F..b-L-1 (minus the forced
+ * previous chunk when L == 0) are scored by q.c_m, the top K_c kept, their
+ * groups scored by q.g_{m,g} and the top K_g kept.  Ties in score go to the
+ * lower index.  Outputs sel_chunk / sel_group as in the header comment. */
+hga_status hga_route(const hga_dims *dims, const hga_params *prm,
+                     const void *q, const int32_t *pos,
+                     const float *s_chunk, const float *s_group,
+                     int32_t *sel_chunk, int32_t *sel_group, void *stream);
+
+/* Stage 3 — exact softmax attention over the routed token set.  Page section
+ * 3, "精确 Token 输出注意力" (exact token output attention) with eq. (1): each
+ * query token i of block b attends, with scale 1/sqrt(D), to the union of
+ * sink chunks 0..F-1, recent chunks b-L..b-1, chunk b-1, the tokens of
+ * sel_group, and tokens b*C..i of its own chunk.  q is raw (pre-RoPE) and is
+ * rotated inside; k_rot comes from hga_build_summaries.  lse may be NULL. */
+hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
+                      const void *q, const int32_t *pos,
+                      const void *k_rot, const void *v,
+                      const int32_t *sel_group, void *out, float *lse,
+                      void *stream);
+
+/* Bytes of device workspace hga_forward needs for `mode` (0 if none). */
+size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm);
+
+/* The whole path in one call.
+ * HGA_PREFILL: stages 1-3 over the T prompt tokens (K_rot, summaries and
+ *   selections live in the workspace unless io.cache / io.sel_* are given).
+ *   With io.cache.k_rot set (capacity >= T), the cache is filled for decoding:
+ *   K_rot, V, pos, summaries, the open chunk's raw keys, and lens = T.
+ * HGA_DECODE: dims.T must equal io.cache.capacity.  For each sequence b, appends the new token at t = lens[b]
+ *   (rotated key, value, position, raw key of the open chunk), builds the
+ *   summaries of chunk t/C if t closes it (page section 3, store operation
+ *   "append closed chunk"), routes with the token's own query (summed over the
+ *   KV head's query heads), attends over the visible set of token t and
+ *   increments lens[b].  Requires lens[b] < dims.T.
+ * workspace: hga_workspace_size(mode) bytes of device memory, 256-byte
+ * aligned.  For HGA_DECODE it must be zero-filled before its first use; the
+ * library leaves it zeroed between calls.  Calls that share a workspace must
+ * not overlap on the GPU. */
+hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
+                       const hga_io *io, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/* Static description of a status code. */
+const char *hga_status_string(hga_status s);
+
+/* The last CUDA error code seen by a failing call on this thread (0 = none). */
+int hga_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HGA_H */

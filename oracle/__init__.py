@@ -89,7 +89,7 @@ def _load():
             lib.or_visible_mark.argtypes = [i32, i32, i32, P, P, P]
             lib.or_attend_row.argtypes = [P, P, P, i64, P, i32, i32, P, P]
             lib.or_hga.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, i32, P, i32, i32,
-                                   P, P, P, P, P, P]
+                                   P, P, P, P, P, P, P, i32]
             lib.or_hga.restype = i32
             lib.or_dense.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, dbl, P, P]
             lib.or_dense.restype = i32
@@ -216,12 +216,15 @@ def visible_mark(c: int, i: int, T: int, sel_g, params: Params) -> np.ndarray:
 
 
 def hga(Q, K, V, pos, params: Params, route_block: int | None = None, units=None,
-        nthreads: int | None = None, want_scores: bool = False):
+        nthreads: int | None = None, want_scores: bool = False, sel_g_force=None,
+        attend: bool = True):
     """Full HGA over query sets.  route_block = C (prefill blocks, default) or
     1 (per-token routing, as in decode).  units: list of (b, s) pairs; default
     every query set of every batch row.  Returns dict with O [B,T,Hq,D] (rows
     of the computed units; NaN elsewhere), LSE [B,Hq,T], units, sel_c
-    [n_units,Hkv,K_c], sel_g [n_units,Hkv,K_g] and optionally cscore/gscore."""
+    [n_units,Hkv,K_c], sel_g [n_units,Hkv,K_g] and optionally cscore/gscore.
+    sel_g_force [n_units,Hkv,K_g]: attend over these routed groups instead of
+    the oracle's own choice.  attend=False: routing only."""
     Q = _f64(Q)
     K = _f64(K)
     V = _f64(V)
@@ -244,10 +247,14 @@ def hga(Q, K, V, pos, params: Params, route_block: int | None = None, units=None
     gs = np.full((nu, Hkv, max(NG, 1)), np.nan) if want_scores else None
     if nthreads is None:
         nthreads = len(os.sched_getaffinity(0))
+    force = None
+    if sel_g_force is not None:
+        force = np.ascontiguousarray(_i32(sel_g_force).reshape(nu, Hkv, params.K_g))
     pc = params.c()
     rc = _load().or_hga(_p(Q), _p(K), _p(V), _p(pos), B, T, Hq, Hkv, D, ctypes.byref(pc), rb,
                         _p(u), nu, int(nthreads), _p(O), _p(LSE), _p(sel_c), _p(sel_g),
-                        _p(cs) if want_scores else None, _p(gs) if want_scores else None)
+                        _p(cs) if want_scores else None, _p(gs) if want_scores else None,
+                        _p(force) if force is not None else None, 1 if attend else 0)
     if rc != 0:
         raise ValueError("oracle: malformed arguments")
     out = {"O": O, "LSE": LSE, "units": u, "sel_c": sel_c[:, :, :params.K_c],

@@ -352,6 +352,8 @@ typedef struct {
     double *O, *LSE;
     int32_t *sel_c, *sel_g;
     double *cscore, *gscore;
+    const int32_t *sel_g_force; /* nullable: routed groups given, not chosen */
+    int do_attend;
     /* shared precomputation */
     const double *Krot, *S_c, *S_g, *omega;
     int NC, NG;
@@ -374,6 +376,10 @@ static void run_item(const or_job *J, int item, uint8_t *mark, double *q_r, doub
              J->S_g + ((int64_t)b * J->Hkv + h) * J->NG * D, J->NC, c, D, p, sel_c, sel_g,
              J->cscore ? J->cscore + ((int64_t)u * J->Hkv + h) * J->NC : NULL,
              J->gscore ? J->gscore + ((int64_t)u * J->Hkv + h) * J->NG : NULL);
+    if (J->sel_g_force)
+        memcpy(sel_g, J->sel_g_force + ((int64_t)u * J->Hkv + h) * p->K_g,
+               sizeof(int32_t) * (size_t)p->K_g);
+    if (!J->do_attend) return;
     const double *Kb = J->Krot + ((int64_t)b * J->T * J->Hkv + h) * D;
     const double *Vb = J->V + ((int64_t)b * J->T * J->Hkv + h) * D;
     for (int i = i0; i < i1; ++i) {
@@ -409,12 +415,15 @@ static void *worker(void *arg)
  * O rows [B,T,Hq,D] and LSE [B,Hq,T] (rows of the unit only; LSE nullable),
  * sel_c [n_units,Hkv,K_c], sel_g [n_units,Hkv,K_g], and if non-NULL the
  * candidate scores cscore [n_units,Hkv,NC], gscore [n_units,Hkv,NG].
- * Summaries are rebuilt here from K (a "full recompute").  Returns 0, or -1
- * on a malformed argument. */
+ * Summaries are rebuilt here from K (a "full recompute").  If sel_g_force
+ * is non-NULL ([n_units,Hkv,K_g]) the attention uses those routed groups
+ * instead of its own choice (sel_g still reports the oracle's choice's
+ * replacement: the forced ids).  With do_attend == 0 only routing runs.
+ * Returns 0, or -1 on a malformed argument. */
 int or_hga(const double *Q, const double *K, const double *V, const int32_t *pos, int B, int T,
            int Hq, int Hkv, int D, const or_params *p, int route_block, const int32_t *units,
            int n_units, int nthreads, double *O, double *LSE, int32_t *sel_c, int32_t *sel_g,
-           double *cscore, double *gscore)
+           double *cscore, double *gscore, const int32_t *sel_g_force, int do_attend)
 {
     if (Hq % Hkv || D % 2 || p->C % p->g_s || route_block < 1 || p->C % route_block) return -1;
     int NC = T / p->C, NG = NC * (p->C / p->g_s);
@@ -432,7 +441,8 @@ int or_hga(const double *Q, const double *K, const double *V, const int32_t *pos
     pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
     for (int t = 0; t < nthreads; ++t) {
         or_job J = {Q, K, V, pos, B, T, Hq, Hkv, D, p, route_block, units, n_units, O, LSE,
-                    sel_c, sel_g, cscore, gscore, Krot, S_c, S_g, omega, NC, NG, nthreads, t};
+                    sel_c, sel_g, cscore, gscore, sel_g_force, do_attend, Krot, S_c, S_g,
+                    omega, NC, NG, nthreads, t};
         jobs[t] = J;
     }
     for (int t = 1; t < nthreads; ++t)

@@ -1,0 +1,132 @@
+"""GPU parity of the prefill path (summaries, routing, attention) against the
+CPU oracle, through the C ABI (via the thin Python binding).
+
+Sizes: small enough for the oracle to finish in seconds, spanning several
+tiles and ragged tails; plus the 32K Qwen3-shaped workload at full size in
+the launch configuration the bench times, with every routed index set
+compared and outputs on sampled blocks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import TOL, RouteRef, check_unit_selection, row_rel_err
+from workloads import WORKLOADS, make_prefill_inputs
+
+pytestmark = pytest.mark.gpu
+
+TINY = WORKLOADS["tiny_f32_prefill_1k"]
+SMALLLM = WORKLOADS["smalllm40m_bf16_prefill_4k"]
+QWEN = WORKLOADS["qwen3_30b_a3b_bf16_prefill_32k"]
+
+CASES = {
+    "tiny_f32_1k": TINY,
+    "f32_ragged_1000": TINY.replace(T=1000),
+    "f32_F0_L0_gqa": TINY.replace(T=700, F=0, L=0, Hq=4, Hkv=2, K_c=3, K_g=5),
+    "f32_gs8_D128": TINY.replace(T=832, g_s=8, D=128, Hq=8, Hkv=2, theta=1e6),
+    "f32_gs64": TINY.replace(T=900, g_s=64, K_g=3),
+    "f32_gs1": TINY.replace(T=512, g_s=1, K_g=40),
+    "f32_T1": TINY.replace(T=1),
+    "f32_T63": TINY.replace(T=63),
+    "f32_T65": TINY.replace(T=65),
+    "f32_full_budget": TINY.replace(T=640, K_c=64, K_g=256),
+    "bf16_smalllm_2x1024": SMALLLM.replace(B=2, T=1024),
+    "bf16_qwen_2048": QWEN.replace(T=2048),
+    "bf16_qwen_ragged": QWEN.replace(T=64 * 20 + 33),
+    "bf16_qwen_L0_F0": QWEN.replace(T=1280, F=0, L=0, K_c=5, K_g=9),
+}
+
+
+def _hp(w):
+    import hierarchical_kv_routing_b200 as hga
+    return hga.HGAParams(C=w.C, g_s=w.g_s, F=w.F, L=w.L, K_c=w.K_c, K_g=w.K_g,
+                         rope_theta=w.theta)
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def run_and_check(hga, w, seed, units=None, sample_rows=None):
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=seed)
+    dev = torch.device("cuda")
+    qd, kd, vd, pd = (x.to(dev) for x in (q, k, v, pos))
+    hp = _hp(w)
+    p = oracle.Params.of(w)
+    tol = TOL[w.dtype]
+
+    k_rot, s_c, s_g = hga.hga_build_summaries(kd, pd, hp)
+    sel_c, sel_g = hga.hga_route(qd, pd, s_c, s_g, hp)
+    out, lse = hga.hga_attend(qd, pd, k_rot, vd, sel_g, hp, want_lse=True)
+    res = hga.hga_forward_prefill(qd, kd, vd, pd, hp, want_lse=True, want_sel=True)
+    torch.cuda.synchronize()
+    # the one-call path runs the same kernels: identical results
+    assert torch.equal(res["sel_chunk"], sel_c) and torch.equal(res["sel_group"], sel_g)
+    assert torch.equal(res["out"].view(torch.int16 if w.dtype == "bf16" else torch.int32),
+                       out.view(torch.int16 if w.dtype == "bf16" else torch.int32))
+
+    # stage 1: K_rot and summaries
+    ref = RouteRef(q, k, pos, p, w.Hkv)
+    krot_ref = oracle.rope_rows(k, np.broadcast_to(_np(pd)[:, :, None], k.shape[:3]), w.theta)
+    kr = _np(k_rot)
+    ulp = 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -22
+    assert np.all(np.abs(kr - krot_ref) <= ulp * np.abs(krot_ref) + 1e-6), "K_rot"
+    for gpu, orc in ((s_c, ref.S_c), (s_g, ref.S_g)):
+        if orc.size:
+            assert row_rel_err(_np(gpu), orc) < 2e-6, "summaries"
+
+    # stage 2: every routed set (all units), with the tie rule
+    B, T = w.B, pos.shape[1]
+    NB = (T + 63) // 64
+    sc, sg = sel_c.cpu().numpy(), sel_g.cpu().numpy()
+    all_units = [(b, u) for b in range(B) for u in range(NB)]
+    rr = oracle.hga(q, k, v, pos, p, units=all_units, attend=False)
+    tie_units = []
+    for i, (b, u) in enumerate(all_units):
+        for h in range(w.Hkv):
+            ok, tie = check_unit_selection(ref, b, h, 64 * u, min(T, 64 * u + 64), u,
+                                           sc[b, u, h], sg[b, u, h], rr["sel_c"][i, h],
+                                           rr["sel_g"][i, h])
+            assert ok, f"routing mismatch at b={b} block={u} h={h}"
+            if tie:
+                tie_units.append((b, u))
+
+    # stage 3: outputs on the checked units
+    units = all_units if units is None else units
+    force = np.stack([sg[b, u] for (b, u) in units])
+    orc = oracle.hga(q, k, v, pos, p, units=units, sel_g_force=force)
+    O = _np(out)
+    L = _np(lse)
+    for (b, u) in units:
+        sl = slice(64 * u, min(T, 64 * u + 64))
+        e = row_rel_err(O[b, sl], orc["O"][b, sl])
+        assert e <= tol, f"output rel err {e} at b={b} block={u}"
+        le = np.abs(L[b, :, sl] - orc["LSE"][b, :, sl]).max()
+        assert le <= (1e-5 if w.dtype == "f32" else 2e-2) * max(1.0, np.abs(orc["LSE"][b, :, sl]).max()), "lse"
+    return {"tie_units": tie_units}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_parity(gpu_lib, name):
+    run_and_check(gpu_lib, CASES[name], seed=7)
+
+
+def test_full_budget_is_dense(gpu_lib):
+    w = TINY.replace(T=640, K_c=64, K_g=256, Hq=4, Hkv=2)
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=3)
+    dev = torch.device("cuda")
+    res = gpu_lib.hga_forward_prefill(*(x.to(dev) for x in (q, k, v, pos)), _hp(w))
+    O, _ = oracle.dense(q, k, v, pos, w.theta)
+    assert row_rel_err(_np(res["out"]), O) <= 1e-5
+
+
+@pytest.mark.slow
+def test_qwen_32k_full_size(gpu_lib):
+    """The 32K Qwen3-shaped prefill exactly as the bench runs it: every
+    routed set checked; outputs on sampled blocks (first F+L+2, a spread
+    through the middle and the last)."""
+    w = QWEN
+    NB = w.T // 64
+    blocks = list(range(0, w.F + w.L + 2)) + list(range(40, NB, 61)) + [NB - 1]
+    run_and_check(gpu_lib, w, seed=11, units=[(0, u) for u in blocks])
