@@ -94,6 +94,8 @@ PrefillWs prefill_ws(const Geo &g, int dtype) {
 hga_status attend_dispatch(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                            const void *k_rot, int k_T, const void *v, int v_T,
                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st) {
+    if (attend_tc_supported(g, dtype))
+        return launch_attend_tc(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
     return launch_attend_simt(g, r, dtype, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
 }
 

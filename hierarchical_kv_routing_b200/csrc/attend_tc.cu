@@ -1,0 +1,519 @@
+// Stage 3 on the 5th-generation tensor cores (sm_100a, bf16): exact softmax
+// attention over the routed token set of each 64-token query block.
+//
+// Method: HGA paper-review page, section 3, exact token output attention with
+// eq. (1): the block's queries attend, with scale 1/sqrt(D), to the sink
+// chunks, the recent chunks, the previous chunk, the routed groups and the
+// causal part of their own chunk, and nothing else.
+//
+// Design.  One CTA owns up to 256 query rows of one (block, KV head) unit
+// (rows ordered token-major, head-minor, so the G query heads of a KV head
+// share every key tile) as two 128-row M-tiles.  The unit's visible set is a
+// list of 8-token segments; 16 segments make one 128-key tile.
+//   warp 0      TMA producer: both Q tiles once, then per key tile one
+//               8x64-element box per segment and D-half for K and for V, into
+//               128-byte-swizzled shared memory (a 2- or 4-stage ring).
+//   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into TMEM
+//               (SS form), then O += P V with P read from TMEM (TS form).
+//   warps 2-3   build the segment list at start.
+//   warps 4-11  two softmax warpgroups, one per M-tile; thread = TMEM lane =
+//               query row.  They rotate their Q rows in shared memory (RoPE),
+//               read S from TMEM, keep a running max in base 2 and rescale O
+//               in TMEM only when the max grows by more than 2^8 (exact: the
+//               final normalisation uses the same reference), write P (bf16)
+//               over the S columns, and finally normalise O and store it.
+// The two M-tiles ping-pong so the tensor core computes one tile's S and PV
+// while the other's softmax runs.  Every mbarrier wait is bounded; a timeout
+// records an error word and the CTA winds down.
+#include <cudaTypedefs.h>
+
+#include "hga_internal.cuh"
+#include "sm100.cuh"
+
+namespace hga {
+
+__device__ int g_attend_tc_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kMaxSeg = 2048;
+constexpr int kSegPerTile = 16;          // 16 x 8 tokens = 128 keys
+constexpr int kDummy = 0x7fffffff;       // padding segment
+
+template <int D>
+struct Cfg {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr uint32_t kHalfBytes = 128 * 128;          // 128 rows x 128 B
+    static constexpr uint32_t kTileBytes = kHalves * kHalfBytes;
+    static constexpr uint32_t oQ = 0;
+    static constexpr uint32_t oK = oQ + 2 * kTileBytes;
+    static constexpr uint32_t oV = oK + kStages * kTileBytes;
+    static constexpr uint32_t oEnd = oV + kStages * kTileBytes;
+};
+
+struct Ctl {
+    uint64_t q_full[2], q_ready[2], s_full[2], p_full[2], o_full[2];
+    uint64_t k_full[4], v_full[4], kv_empty[4];
+    uint64_t fin;
+    uint32_t tmem_base;
+    int nseg, first_cur;
+    volatile int abort;
+    int seg_tok[kMaxSeg];
+};
+
+struct TcArgs {
+    int T, Hq, Hkv, G, NB, F, L, K_g, g_s, k_T, v_T;
+    int rows_per_unit, ctas_per_unit, tokM;
+    const int32_t *sel_group;
+    const int32_t *pos;
+    __nv_bfloat16 *out;
+    float *lse;
+    float scale_log2;
+    Rope rope;
+};
+
+__device__ __forceinline__ void fail(Ctl &ctl) {
+    ctl.abort = 1;
+    atomicExch(&g_attend_tc_error, (int)HGA_ERR_TIMEOUT);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+            const __grid_constant__ CUtensorMap tmV, const TcArgs A) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ Ctl ctl;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x / A.ctas_per_unit, cu = blockIdx.x % A.ctas_per_unit;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c * kChunk;
+    const int row0 = cu * 256;
+    const int rows = min(256, A.rows_per_unit - row0);
+    const int NT = (rows + 127) >> 7;
+    const int max_tok = min(t0 + (row0 + rows - 1) / A.G, A.T - 1);
+
+    // ---------------------------------------------------------- set-up --
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl.q_full[i], 1);
+            mbar_init(&ctl.q_ready[i], 128);
+            mbar_init(&ctl.s_full[i], 1);
+            mbar_init(&ctl.p_full[i], 128);
+            mbar_init(&ctl.o_full[i], 1);
+        }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&ctl.k_full[i], 1);
+            mbar_init(&ctl.v_full[i], 1);
+            mbar_init(&ctl.kv_empty[i], 1);
+        }
+        mbar_init(&ctl.fin, 1);
+        ctl.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl.tmem_base, 512);
+        tc_fence_before();
+    }
+    if (warp == 2) {
+        // the visible set as 8-token segments: sinks, recent, routed groups,
+        // then the current chunk up to this CTA's last query token
+        const int nsink = min(A.F, c);
+        const int rec_lo = max(c - max(A.L, 1), nsink);
+        const int n_fixed = 8 * (nsink + (c - rec_lo));
+        for (int s = lane; s < n_fixed; s += 32)
+            ctl.seg_tok[s] = s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8;
+        const int32_t *sel = A.sel_group + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_g;
+        const int gseg = A.g_s / 8;
+        int kg = 0;
+        for (int base = 0; base < A.K_g; base += 32) {
+            const int v = base + lane < A.K_g ? sel[base + lane] : -1;
+            kg += __popc(__ballot_sync(0xffffffffu, v >= 0));
+        }
+        for (int j = lane; j < kg; j += 32) {
+            const int g = sel[j];
+            for (int e = 0; e < gseg; ++e) ctl.seg_tok[n_fixed + j * gseg + e] = g * A.g_s + e * 8;
+        }
+        const int n_route = n_fixed + kg * gseg;
+        const int ncur = (max_tok - t0) / 8 + 1;
+        for (int e = lane; e < ncur; e += 32) ctl.seg_tok[n_route + e] = t0 + e * 8;
+        int nseg = n_route + ncur;
+        if (lane == 0) {
+            if (nseg & 1) ctl.seg_tok[nseg++] = kDummy;
+            ctl.nseg = nseg;
+            ctl.first_cur = n_route;
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+    const int nseg = ctl.nseg;
+    const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
+    const int first_cur = ctl.first_cur;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            for (int mt = 0; mt < NT; ++mt) {
+                const int tok_first = t0 + (row0 + mt * 128) / A.G;
+                mbar_arrive_expect_tx(&ctl.q_full[mt], (uint32_t)(A.G * A.tokM * D * 2));
+                for (int hf = 0; hf < C::kHalves; ++hf)
+                    tma_load_3d(smem + C::oQ + mt * C::kTileBytes + hf * C::kHalfBytes, &tmQ,
+                                &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first);
+            }
+            for (int j = 0; j < ntiles && !ctl.abort; ++j) {
+                const int s = j % C::kStages;
+                if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1)) {
+                    fail(ctl);
+                    break;
+                }
+                const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
+                const uint32_t bytes = (uint32_t)nsj * 8 * D * 2;
+                uint8_t *kt = smem + C::oK + s * C::kTileBytes;
+                uint8_t *vt = smem + C::oV + s * C::kTileBytes;
+                mbar_arrive_expect_tx(&ctl.k_full[s], bytes);
+                for (int e = 0; e < nsj; ++e) {
+                    const int st = ctl.seg_tok[j * kSegPerTile + e];
+                    const int z = b * A.k_T + (st == kDummy ? 0 : st);
+                    for (int hf = 0; hf < C::kHalves; ++hf)
+                        tma_load_3d(kt + hf * C::kHalfBytes + e * 1024, &tmK, &ctl.k_full[s],
+                                    hf * 64, h, z);
+                }
+                mbar_arrive_expect_tx(&ctl.v_full[s], bytes);
+                for (int e = 0; e < nsj; ++e) {
+                    const int st = ctl.seg_tok[j * kSegPerTile + e];
+                    const int z = b * A.v_T + (st == kDummy ? 0 : st);
+                    for (int hf = 0; hf < C::kHalves; ++hf)
+                        tma_load_3d(vt + hf * C::kHalfBytes + e * 1024, &tmV, &ctl.v_full[s],
+                                    hf * 64, h, z);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issuer --
+        if (lane == 0) {
+            const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            bool ok = true;
+            for (int mt = 0; mt < NT && ok; ++mt) ok = mbar_wait(&ctl.q_ready[mt], 0);
+            tc_fence_after();
+            auto issue_pv = [&](int mt, int jj) {
+                const int sp = jj % C::kStages;
+                const int nsj = min(kSegPerTile, nseg - jj * kSegPerTile);
+                const uint32_t vbase = smem_addr(smem + C::oV + sp * C::kTileBytes);
+                for (int ks = 0; ks < nsj / 2; ++ks) {
+                    const uint64_t bd = smem_desc_sw128(vbase + ks * 2048, C::kHalfBytes, 1024);
+                    mma_ts(tmem + mt * 256 + 128, tmem + mt * 256 + ks * 8, bd, idesc_pv,
+                           (jj > 0 || ks > 0) ? 1u : 0u);
+                }
+            };
+            auto issue_s = [&](int mt, int jj) {
+                const int s = jj % C::kStages;
+                const int nsj = min(kSegPerTile, nseg - jj * kSegPerTile);
+                const uint32_t idesc = idesc_bf16_f32(128, nsj * 8, false, false);
+                const uint32_t qb = smem_addr(smem + C::oQ + mt * C::kTileBytes);
+                const uint32_t kb = smem_addr(smem + C::oK + s * C::kTileBytes);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+                    mma_ss(tmem + mt * 256, smem_desc_sw128(qb + off, 16, 1024),
+                           smem_desc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                }
+            };
+            for (int j = 0; j <= ntiles && ok; ++j) {
+                const int s = j % C::kStages;
+                if (j < ntiles) {
+                    if (!(ok = mbar_wait(&ctl.k_full[s], (j / C::kStages) & 1))) break;
+                    tc_fence_after();
+                }
+                for (int mt = 0; mt < NT && ok; ++mt) {
+                    if (j > 0) {
+                        if (!(ok = mbar_wait(&ctl.p_full[mt], (j - 1) & 1))) break;
+                        tc_fence_after();
+                        const int sp = (j - 1) % C::kStages;
+                        if (mt == 0) {
+                            if (!(ok = mbar_wait(&ctl.v_full[sp], ((j - 1) / C::kStages) & 1))) break;
+                            tc_fence_after();
+                        }
+                        issue_pv(mt, j - 1);
+                        if (j == ntiles) mma_commit(&ctl.o_full[mt]);
+                        else if (mt == NT - 1) mma_commit(&ctl.kv_empty[sp]);
+                    }
+                    if (j < ntiles) {
+                        issue_s(mt, j);
+                        mma_commit(&ctl.s_full[mt]);
+                    }
+                }
+            }
+            if (!ok) fail(ctl);
+            // all issued tensor-core work retires before TMEM is released
+            mma_commit(&ctl.fin);
+            if (!mbar_wait(&ctl.fin, 0)) fail(ctl);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------- softmax --
+        const int mt = (warp - 4) >> 2;
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const int R = row0 + mt * 128 + r;
+        const int tok = t0 + R / A.G;
+        const int head = R % A.G;
+        const bool valid = mt < NT && (mt * 128 + r) < rows && tok < A.T;
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
+        if (mt < NT) {
+            // RoPE of this row's query, in place in the swizzled Q tile
+            bool ok = mbar_wait(&ctl.q_full[mt], 0);
+            if (!ok) fail(ctl);
+            if (ok && valid) {
+                uint8_t *qt = smem + C::oQ + mt * C::kTileBytes;
+                const double p = (double)A.pos[(int64_t)b * A.T + tok];
+                constexpr int kGroups = D / 16;       // 8 pairs per 16-byte chunk
+                for (int g = 0; g < kGroups; ++g) {
+                    const int lo_half = 0, hi_half = D == 128 ? 1 : 0;
+                    const int lo_chunk = g, hi_chunk = D == 128 ? g : g + 4;
+                    uint4 *lo = reinterpret_cast<uint4 *>(qt + lo_half * C::kHalfBytes + r * 128 +
+                                                          ((lo_chunk ^ (r & 7)) << 4));
+                    uint4 *hi = reinterpret_cast<uint4 *>(qt + hi_half * C::kHalfBytes + r * 128 +
+                                                          ((hi_chunk ^ (r & 7)) << 4));
+                    uint4 a = *lo, bb = *hi;
+                    __nv_bfloat162 *pa = reinterpret_cast<__nv_bfloat162 *>(&a);
+                    __nv_bfloat162 *pb = reinterpret_cast<__nv_bfloat162 *>(&bb);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __bfloat1622float2(pa[e]);
+                        const float2 y = __bfloat1622float2(pb[e]);
+                        const float2 c0 = rope_cs(A.rope, p, g * 8 + 2 * e);
+                        const float2 c1 = rope_cs(A.rope, p, g * 8 + 2 * e + 1);
+                        pa[e] = __floats2bfloat162_rn(x.x * c0.x - y.x * c0.y, x.y * c1.x - y.y * c1.y);
+                        pb[e] = __floats2bfloat162_rn(y.x * c0.x + x.x * c0.y, y.y * c1.x + x.y * c1.y);
+                    }
+                    *lo = a;
+                    *hi = bb;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&ctl.q_ready[mt]);
+
+            float m_ref = -INFINITY, l = 0.f;
+            const float sc = A.scale_log2;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                if (!(ok = mbar_wait(&ctl.s_full[mt], j & 1))) {
+                    fail(ctl);
+                    break;
+                }
+                tc_fence_after();
+                const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
+                const int nj = nsj * 8;
+                const bool need_mask = (j + 1) * kSegPerTile > first_cur;
+                const int *segs = ctl.seg_tok + j * kSegPerTile;
+                auto masked = [&](int col) -> bool {
+                    if (col >= nj) return true;
+                    const int st = segs[col >> 3];
+                    return st == kDummy || st + (col & 7) > tok;
+                };
+                // pass 1: row max
+                float mx = -INFINITY;
+                for (int cb = 0; cb < (nj + 31) / 32; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + cb * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float x = __uint_as_float(v[e]);
+                        if (!need_mask || !masked(cb * 32 + e)) mx = fmaxf(mx, x);
+                    }
+                }
+                if (!valid) mx = -INFINITY;
+                const float mt_new = mx * sc;
+                // The rescale decision is per row, but tcgen05.ld/st are
+                // warp-collective: the warp rescales together, rows that
+                // keep their reference use factor 1.
+                const bool grow = mt_new > m_ref + 8.0f;
+                const bool rescale = grow && m_ref != -INFINITY;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float f = rescale ? ex2(m_ref - mt_new) : 1.0f;
+                    l *= f;
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_base + 128 + cb * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                        tmem_st32(lane_base + 128 + cb * 32, v);
+                    }
+                }
+                if (grow) m_ref = mt_new;
+                // pass 2: P = 2^(s*scale - m_ref) as bf16 over the S columns
+                const bool live = m_ref != -INFINITY;
+                for (int cb = 0; cb < (nj + 31) / 32; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + cb * 32, v);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float p0 = 0.f, p1 = 0.f;
+                        if (live) {
+                            const int c0 = cb * 32 + 2 * e;
+                            if (!need_mask || !masked(c0))
+                                p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, -m_ref));
+                            if (!need_mask || !masked(c0 + 1))
+                                p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, -m_ref));
+                        }
+                        l += p0 + p1;
+                        pk[e] = pack_bf16(p0, p1);
+                    }
+                    asm volatile(
+                        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, "
+                        "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(lane_base + cb * 16),
+                        "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]),
+                        "r"(pk[6]), "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]),
+                        "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+                        : "memory");
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&ctl.p_full[mt]);
+            }
+            // epilogue: O / l -> out, LSE
+            if (ok) {
+                if (!mbar_wait(&ctl.o_full[mt], 0)) {
+                    fail(ctl);
+                    ok = false;
+                }
+            }
+            tc_fence_after();
+            if (ok) {
+                const float inv = valid && l > 0.f ? 1.f / l : 0.f;
+                __nv_bfloat16 *orow =
+                    A.out + (((int64_t)b * A.T + tok) * A.Hq + (int64_t)h * A.G + head) * D;
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + 128 + cb * 32, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        uint4 w[4];
+                        uint32_t *wp = reinterpret_cast<uint32_t *>(w);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            wp[e] = pack_bf16(__uint_as_float(v[2 * e]) * inv,
+                                              __uint_as_float(v[2 * e + 1]) * inv);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cb * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) dst[e] = w[e];
+                    }
+                }
+                if (valid && A.lse)
+                    A.lse[((int64_t)b * A.Hq + (int64_t)h * A.G + head) * A.T + tok] =
+                        (m_ref + __log2f(l)) * 0.6931471805599453f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 3-D bf16 map over rows of [n_rows][heads][D]: box (64, box_heads, box_rows),
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap *m, const void *base, int D, int heads, long long n_rows, int box_heads,
+              int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)n_rows};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D>
+hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, const void *k_rot,
+               int k_T, const void *v, int v_T, const int32_t *sel_group, void *out, float *lse,
+               cudaStream_t st) {
+    TcArgs a;
+    a.T = g.T;
+    a.Hq = g.Hq;
+    a.Hkv = g.Hkv;
+    a.G = g.G;
+    a.NB = g.NB;
+    a.F = g.F;
+    a.L = g.L;
+    a.K_g = g.K_g;
+    a.g_s = g.g_s;
+    a.k_T = k_T;
+    a.v_T = v_T;
+    a.rows_per_unit = kChunk * g.G;
+    a.ctas_per_unit = (a.rows_per_unit + 255) / 256;
+    a.tokM = min(128, kChunk * g.G) / g.G;
+    a.sel_group = sel_group;
+    a.pos = pos;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    a.rope = r;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, D, g.Hq, (long long)g.B * g.T, g.G, a.tokM) ||
+        !make_map(&mk, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 8) ||
+        !make_map(&mv, v, D, g.Hkv, (long long)g.B * v_T, 1, 8))
+        return HGA_ERR_CUDA;
+    const size_t smem = Cfg<D>::oEnd + 1024;
+    auto kern = k_attend_tc<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    dim3 grid(g.NB * a.ctas_per_unit, g.Hkv, g.B);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Geo &g, int dtype) {
+    if (dtype != HGA_BF16 || (g.D != 64 && g.D != 128)) return false;
+    if (g.G < 1 || g.G > 16 || (g.G & (g.G - 1))) return false;
+    if (g.g_s % 8) return false;
+    const long long segs = 8ll * (g.F + max(g.L, 1) + 1) + (long long)g.K_g * (g.g_s / 8) + 2;
+    return segs <= kMaxSeg;
+}
+
+hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
+                            const void *k_rot, int k_T, const void *v, int v_T,
+                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st) {
+    if (g.NB <= 0) return HGA_OK;
+    return g.D == 128 ? run<128>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st)
+                      : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
+}
+
+}  // namespace hga

@@ -114,6 +114,10 @@ hga_status launch_attend_simt(const Geo &g, const Rope &r, int dtype, const void
                               int v_T, const int32_t *sel_group, void *out, float *lse,
                               cudaStream_t st);
 size_t attend_simt_smem(const Geo &g);
+bool attend_tc_supported(const Geo &g, int dtype);
+hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
+                            const void *k_rot, int k_T, const void *v, int v_T,
+                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st);
 
 // Decode step (append, close-chunk summaries, route, split attention).
 size_t decode_workspace_bytes(const Geo &g);
