@@ -1,0 +1,385 @@
+"""Benchmark of the HGA routed-attention hot path on B200.
+
+One step = the whole prefill path (mixed-RoPE summaries + K_rot, two-level
+routing, tensor-core routed attention) over the Qwen3-30B-A3B-shaped 32K
+workload (B=1, T=32768, 32 query / 4 KV heads, D=128, C=64, g_s=16, F=2,
+L=8, K_c=16, K_g=32, planted-topic keys), seeded synthetic bf16 inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun, one process per GPU)
+every rank runs an independent replica of the workload (the path has no
+cross-sequence exchange); value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen3_30b_a3b_bf16_prefill_32k"
+METRIC = "HGA routed-attn prefill tokens/s & decode steps/s at 32K/64K; % HBM roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attend_tc_qwen32k_traffic.txt")
+ATTEND_SRC = os.path.join(ROOT, "hierarchical_kv_routing_b200", "csrc", "attend_tc.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override the prefill length (small profiling cases only)")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def params_of(w):
+    import hierarchical_kv_routing_b200 as hga
+    return hga.HGAParams(C=w.C, g_s=w.g_s, F=w.F, L=w.L, K_c=w.K_c, K_g=w.K_g,
+                         rope_theta=w.theta)
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "C": w.C, "g_s": w.g_s, "F": w.F, "L": w.L, "K_c": w.K_c, "K_g": w.K_g,
+            "rope_theta": w.theta, "recipe": "planted-topic keys (sigma 0.5), queries at "
+            "cosine 0.5 to one earlier middle chunk per block",
+            "l2": "inputs larger than L2: Q and O stream 537 MB per step",
+            "parallelism": "single GPU" if n == 1 else f"{n} independent replicas"}
+
+
+def attention_flops(w, sel_group):
+    """Algorithmic FLOPs of one attention launch: for every query row,
+    4 * D per visible key (2 for q.k, 2 for p.v), visible keys = fixed
+    windows + routed groups + causal part of the own chunk."""
+    import numpy as np
+    sg = sel_group.cpu().numpy()                   # [B, NB, Hkv, K_g]
+    B, NB = sg.shape[0], sg.shape[1]
+    routed = (sg >= 0).sum(-1) * w.g_s             # [B, NB, Hkv]
+    total = 0
+    for c in range(NB):
+        nsink = min(w.F, c)
+        rec_lo = max(c - max(w.L, 1), nsink)
+        fixed = (nsink + (c - rec_lo)) * w.C
+        ncur = min(w.C, w.T - c * w.C)
+        causal = ncur * (ncur + 1) // 2            # sum over tokens of (i - t0 + 1)
+        keys_rows = (fixed + routed[:, c, :]) * ncur + causal   # [B, Hkv]
+        total += int(keys_rows.sum()) * w.G
+    return 4.0 * w.D * total
+
+
+class ClockSampler:
+    """Samples SM clock, max clock and active clock-event reasons via NVML
+    while the timed region runs (reading only; nothing is changed)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            h = None
+            if bus is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0")
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.h, self.nv = h, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self.t.join()
+
+    def result(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def traffic_for_current_kernel():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, only if that summary was taken on the current kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    src_hash = hashlib.sha256(open(ATTEND_SRC, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(TRAFFIC_FILE):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != src_hash:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def _oracle_inputs(w, seed):
+    import oracle
+    from workloads import make_prefill_inputs
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=seed)
+    return tuple(oracle._f64(x) for x in (q, k, v)) + (pos,)
+
+
+def _oracle_sample(w, inputs, blocks, nthreads):
+    import oracle
+    q, k, v, pos = inputs
+    t = time.perf_counter()
+    oracle.hga(q, k, v, pos, oracle.Params.of(w), units=[(0, b) for b in blocks],
+               nthreads=nthreads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(w, seed, budget_s=20.0, per_call=16):
+    """The oracle (plain fp64 C; the full-sequence rotation and summary pass
+    on one thread, then threads over (block, KV head) units) on a bounded
+    sample of the workload, scaled to the whole workload's tokens/s."""
+    inputs = _oracle_inputs(w, seed)
+    nthreads = len(os.sched_getaffinity(0))
+    t_pre = _oracle_sample(w, inputs, [], nthreads)
+    NB = (w.T + w.C - 1) // w.C
+    done, spent, t_blocks, i = 0, 0.0, 0.0, 0
+    while spent < budget_s and done < NB:
+        blocks = [(NB // 3 + (i * per_call + j) * 97) % NB for j in range(per_call)]
+        i += 1
+        dt = _oracle_sample(w, inputs, blocks, nthreads)
+        spent += dt
+        t_blocks += max(dt - t_pre, 0.0)
+        done += len(blocks)
+    est = t_pre + t_blocks / done * NB * w.B
+    return {"value": w.B * w.T / est, "unit": "tokens/s",
+            "cores": min(nthreads, per_call * w.Hkv), "kind": "oracle",
+            "sample": f"{done} of {NB} query blocks (all {w.Hkv} KV heads each), {per_call} per "
+                      f"call, after a {t_pre:.2f} s full-sequence pass; whole-workload time = that "
+                      f"pass + mean block time x {NB}"}
+
+
+def run_reference(args, per_step=2):
+    """The CPU oracle on the same workload (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from workloads import WORKLOADS
+    w = WORKLOADS[WORKLOAD]
+    inputs = _oracle_inputs(w, args.seed)
+    nthreads = len(os.sched_getaffinity(0))
+    t_pre = _oracle_sample(w, inputs, [], nthreads)
+    NB = w.T // w.C
+    step_est = []
+    for s in range(args.warmup + args.steps):
+        blocks = [(s * 97 * per_step + j * 211 + 11) % NB for j in range(per_step)]
+        dt = _oracle_sample(w, inputs, blocks, nthreads)
+        if s >= args.warmup:
+            step_est.append(t_pre + max(dt - t_pre, 0.0) / per_step * NB)
+    est = statistics.median(step_est)
+    value = w.B * w.T / est
+    cores = min(nthreads, per_step * w.Hkv)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"each step: {per_step} of {NB} query blocks (all KV "
+                                       f"heads) after a {t_pre:.2f} s full-sequence pass; step "
+                                       f"value = that pass + mean block time x {NB}; median "
+                                       f"over steps"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_kv_routing_b200 as hga
+    from workloads import WORKLOADS, make_prefill_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    hga.load()
+    w = WORKLOADS[WORKLOAD]
+    if args.seq:
+        w = w.replace(T=args.seq, name=f"{w.name}_T{args.seq}")
+    hp = params_of(w)
+
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=args.seed + rank, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    k_rot, s_c, s_g = hga.hga_build_summaries(k, pos, hp)
+    sel_c, sel_g = hga.hga_route(q, pos, s_c, s_g, hp)
+    out = torch.empty_like(q)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c, s_group=s_g)
+        if ev:
+            ev[1].record(stream)
+        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)
+        if ev:
+            ev[2].record(stream)
+        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    flops = attention_flops(w, sel_g)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    stage_ms = [statistics.mean(e[a].elapsed_time(e[a + 1]) for e in evs) for a in range(3)]
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.B * w.T * world * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    # end to end through the public one-call API, host buffers, copies inside
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 20))
+    hq, hk, hv, hpos = (x.cpu().pin_memory() for x in (q, k, v, pos))
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    ws = torch.empty(hga.hga_workspace_size(hga.PREFILL, w.B, w.T, w.Hq, w.Hkv, w.D,
+                                            torch.bfloat16, hp) + 256,
+                     dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        dq, dk, dv, dp = (x.to(dev, non_blocking=True) for x in (hq, hk, hv, hpos))
+        r = hga.hga_forward_prefill(dq, dk, dv, dp, hp, workspace=ws)
+        hout.copy_(r["out"], non_blocking=True)
+
+    for _ in range(2 if e2e_steps else 0):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = (w.B * w.T * world * e2e_steps / (float(te.item()) / 1e3)) if e2e_steps else None
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hpos))
+    d2h = hout.numel() * hout.element_size()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, src = peaks()
+    attend_s = stage_ms[2] / 1e3
+    achieved = flops / attend_s / 1e12
+    peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic_for_current_kernel(),
+            "kernel": "k_attend_tc<128> (routed attention, tcgen05)",
+            "flops_per_launch": flops, "avg_launch_ms": stage_ms[2],
+            "peak_source": f"{src} bf16_tflops (burst; the kernel is timed alone per launch)"}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, world), "clocks": clk.result(),
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "api": "hga_forward(HGA_PREFILL) via the Python binding"},
+            "gpu_launches": 3 * args.steps,
+            "stage_ms": {"summaries": stage_ms[0], "route": stage_ms[1], "attend": stage_ms[2]},
+            "roofline": roof}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.seed)
+    if args.seq or args.no_e2e:
+        line["note"] = "profiling variant, not a bench line"
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
