@@ -22,7 +22,8 @@ import torch
 
 __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "hga_route",
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
-           "hga_workspace_size", "HGAError", "PREFILL", "DECODE"]
+           "hga_workspace_size", "hga_forward_prefill_noalloc", "HGAError", "PREFILL",
+           "DECODE"]
 
 PREFILL, DECODE = 0, 1
 _F32, _BF16 = 0, 1
@@ -104,6 +105,8 @@ def load():
         lib.hga_workspace_size.argtypes = [ctypes.c_int, P, P]
         lib.hga_workspace_size.restype = ctypes.c_size_t
         lib.hga_forward.argtypes = [ctypes.c_int, P, P, P, P, ctypes.c_size_t, P]
+        lib.hga_forward_prefill_noalloc.argtypes = [P, P, P, P, P, P, P, P, P]
+        lib.hga_forward_prefill_noalloc.restype = ctypes.c_int
         lib.hga_status_string.argtypes = [ctypes.c_int]
         lib.hga_status_string.restype = ctypes.c_char_p
         lib.hga_last_cuda_error.restype = ctypes.c_int
@@ -314,6 +317,32 @@ def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCa
                          None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
     _check(st, "hga_forward(prefill)")
     return res
+
+
+def hga_forward_prefill_noalloc(q, k, v, pos, params: HGAParams, out: torch.Tensor, *,
+                                lse: Optional[torch.Tensor] = None, stream=None):
+    """The prefill path on the library's fixed 16 MiB device scratch, for
+    callers that cannot allocate at call time (their device memory belongs to
+    another allocator or a fixed arena).  The caller passes every buffer,
+    including `out` ([B,T,Hq,D]) and optionally `lse` ([B,Hq,T] f32); this
+    wrapper allocates nothing.  Shapes needing more scratch are rejected."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _need(k, "k", (B, T, Hkv, D), q.dtype)
+    _need(v, "v", (B, T, Hkv, D), q.dtype)
+    _need(pos, "pos", (B, T), torch.int32)
+    _need(out, "out", (B, T, Hq, D), q.dtype)
+    if lse is not None:
+        _need(lse, "lse", (B, Hq, T), torch.float32)
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    st = lib.hga_forward_prefill_noalloc(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(k),
+                                         _ptr(v), _ptr(pos), _ptr(out), _ptr(lse),
+                                         _stream(stream))
+    _check(st, "hga_forward_prefill_noalloc")
+    return out
 
 
 def hga_forward_decode(q_new, k_new, v_new, pos_new, cache: KVCache, params: HGAParams, *,

@@ -184,6 +184,32 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
                        const hga_io *io, void *workspace, size_t workspace_bytes,
                        void *stream);
 
+/* hga_forward(HGA_PREFILL) for callers that cannot allocate device memory.
+ * The paper has no counterpart to this call: it is a convenience of this
+ * library.  It is meant for code that only holds its inputs and outputs at
+ * call time and may not call cudaMalloc then, for example a serving step
+ * whose device memory belongs to another allocator or to a fixed arena
+ * (a cudaMalloc there can fail, or stall the device mid-step), or a plug-in
+ * that a host runtime hands nothing but tensors.
+ *
+ * Arguments are those of hga_forward(HGA_PREFILL) without a workspace: q, k,
+ * v, pos and out as in the header comment, lse optional (NULL to skip).  The
+ * scratch (rotated keys, summaries, routed ids) lives in one fixed 16 MiB
+ * array inside the library's device image, which every GPU that loads the
+ * library keeps until the process exits.  A shape whose scratch
+ * (hga_workspace_size(HGA_PREFILL, ...)) exceeds 16 MiB is rejected with
+ * HGA_ERR_WORKSPACE before anything is launched; about 14K tokens fit at
+ * Hkv=4, D=128, bf16.  Nothing in the scratch needs to start at zero.
+ *
+ * The first call on a device, with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture.  All calls share the one array:
+ * calls that overlap on the GPU (other streams, other threads, without
+ * ordering between them) race on it and give wrong results. */
+hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hga_params *prm,
+                                       const void *q, const void *k, const void *v,
+                                       const int32_t *pos, void *out, float *lse, void *stream);
+
 /* Static description of a status code. */
 const char *hga_status_string(hga_status s);
 
