@@ -105,3 +105,35 @@ __device__ __forceinline__ int topk_select(unsigned long long *cand, int n, int 
 }
 
 }  // namespace hga
+
+namespace hga {
+
+// The K largest candidate keys (cand is consumed), written to out[0..K)
+// (global or shared), descending, padded with 0.  Returns min(K, n).
+__device__ __forceinline__ int topk_keys(unsigned long long *cand, int n, int K,
+                                         unsigned long long *out, RouteScratch &rs) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int k = min(K, n);
+    for (int round = 0; round < k; ++round) {
+        unsigned long long m = 0;
+        for (int r = threadIdx.x; r < n; r += blockDim.x) m = cand[r] > m ? cand[r] : m;
+        m = warp_max_u64(m);
+        if (lane == 0) rs.wmax[warp] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            unsigned long long b = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = rs.wmax[w] > b ? rs.wmax[w] : b;
+            rs.best = b;
+            out[round] = b;
+        }
+        __syncthreads();
+        const unsigned long long b = rs.best;
+        for (int r = threadIdx.x; r < n; r += blockDim.x)
+            if (cand[r] == b) cand[r] = 0;
+    }
+    for (int r = k + threadIdx.x; r < K; r += blockDim.x) out[r] = 0;
+    __syncthreads();
+    return k;
+}
+
+}  // namespace hga

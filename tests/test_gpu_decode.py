@@ -1,0 +1,117 @@
+"""GPU parity of the decode step against the oracle's full recompute.
+
+A prompt fills the cache through hga_forward(HGA_PREFILL); then every decode
+step appends one token per sequence, builds the summaries of a chunk when the
+token closes it, routes with the token's own query and attends.  Each step's
+output, LSE and routed sets are compared with the oracle run on the whole
+sequence with per-token routing (the pages' "decode vs full recompute" check,
+Table 7); the incrementally built summaries are compared with the oracle's
+summaries of the final cache.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import TOL, RouteRef, check_unit_selection, row_rel_err
+from workloads import WORKLOADS, make_decode_inputs
+
+pytestmark = pytest.mark.gpu
+
+QWEN = WORKLOADS["qwen3_30b_a3b_bf16_decode_64k"]
+TINY = WORKLOADS["tiny_f32_prefill_1k"]
+
+CASES = {
+    # history, steps, capacity: every case crosses a chunk boundary
+    "bf16_qwen_like": (QWEN.replace(B=2, Hq=8, Hkv=2), 640, 72, 768),
+    "bf16_qwen_heads": (QWEN.replace(B=2), 700, 60, 832),
+    "f32_ragged_prompt": (TINY.replace(B=2, Hq=4, Hkv=2), 200, 60, 320),
+    "f32_L0_F0": (TINY.replace(B=1, F=0, L=0, K_c=3, K_g=5), 300, 40, 384),
+    "bf16_D64_mha": (WORKLOADS["smalllm40m_bf16_prefill_4k"].replace(B=2, Hq=4, Hkv=4), 500, 30, 576),
+}
+
+
+def _hp(hga, w):
+    return hga.HGAParams(C=w.C, g_s=w.g_s, F=w.F, L=w.L, K_c=w.K_c, K_g=w.K_g,
+                         rope_theta=w.theta)
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy()
+
+
+def run_decode(hga, w, T_hist, steps, cap, seed):
+    d = make_decode_inputs(w, seed=seed, T=T_hist, steps=steps)
+    dev = torch.device("cuda")
+    dt = d["k_hist"].dtype
+    hp = _hp(hga, w)
+    cache = hga.KVCache(w.B, cap, w.Hkv, w.D, dt, hp, device=dev)
+    q_hist = torch.randn(w.B, T_hist, w.Hq, w.D, generator=torch.Generator().manual_seed(seed)).to(dt)
+    hga.hga_forward_prefill(q_hist.to(dev), d["k_hist"].to(dev), d["v_hist"].to(dev),
+                            d["pos_hist"].to(dev), hp, cache=cache)
+    ws = hga.decode_workspace(w.B, cap, w.Hq, w.Hkv, w.D, dt, hp, device=dev)
+    outs, lses, selc, selg = [], [], [], []
+    for s in range(steps):
+        r = hga.hga_forward_decode(d["q"][s].to(dev), d["k_new"][s].to(dev), d["v_new"][s].to(dev),
+                                   d["pos_new"][s].to(dev), cache, hp, want_lse=True,
+                                   want_sel=True, workspace=ws)
+        outs.append(r["out"])
+        lses.append(r["lse"])
+        selc.append(r["sel_chunk"])
+        selg.append(r["sel_group"])
+    torch.cuda.synchronize()
+    return d, cache, torch.stack(outs), torch.stack(lses), torch.stack(selc), torch.stack(selg)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_decode_parity(gpu_lib, name):
+    w, T_hist, steps, cap = CASES[name]
+    d, cache, out, lse, selc, selg = run_decode(gpu_lib, w, T_hist, steps, cap, seed=5)
+    Ttot = T_hist + steps
+    K = torch.cat([d["k_hist"], d["k_new"].transpose(0, 1)], 1)
+    V = torch.cat([d["v_hist"], d["v_new"].transpose(0, 1)], 1)
+    pos = torch.cat([d["pos_hist"], d["pos_new"].transpose(0, 1)], 1)
+    Q = torch.zeros(w.B, Ttot, w.Hq, w.D, dtype=torch.float64)
+    Q[:, T_hist:] = d["q"].transpose(0, 1).double()
+    p = oracle.Params.of(w)
+    units = [(b, T_hist + s) for b in range(w.B) for s in range(steps)]
+    sc, sg = selc.cpu().numpy(), selg.cpu().numpy()          # [S, B, Hkv, K]
+    rr = oracle.hga(Q, K, V, pos, p, route_block=1, units=units, attend=False)
+    ref = RouteRef(Q, K, pos, p, w.Hkv)
+    for i, (b, t) in enumerate(units):
+        s = t - T_hist
+        for h in range(w.Hkv):
+            ok, _ = check_unit_selection(ref, b, h, t, t + 1, t // 64, sc[s, b, h], sg[s, b, h],
+                                         rr["sel_c"][i, h], rr["sel_g"][i, h])
+            assert ok, f"routing mismatch b={b} t={t} h={h}"
+    force = np.stack([sg[t - T_hist, b] for (b, t) in units])
+    orc = oracle.hga(Q, K, V, pos, p, route_block=1, units=units, sel_g_force=force)
+    O, L = _np(out), _np(lse)
+    tol = TOL[w.dtype]
+    for (b, t) in units:
+        s = t - T_hist
+        e = row_rel_err(O[s, b], orc["O"][b, t])
+        assert e <= tol, f"decode output rel err {e} at b={b} t={t}"
+        le = np.abs(L[s, b] - orc["LSE"][b, :, t]).max()
+        assert le <= tol * max(1.0, np.abs(orc["LSE"][b, :, t]).max())
+    # the cache: lens, positions, rotated keys, and incrementally built summaries
+    assert (cache.lens.cpu() == Ttot).all()
+    assert torch.equal(cache.pos[:, :Ttot].cpu(), pos)
+    S_c, S_g = oracle.build_summaries(K, pos, p)
+    nc = Ttot // 64
+    assert row_rel_err(_np(cache.s_chunk[:, :, :nc]), S_c[:, :, :nc]) < 2e-6
+    assert row_rel_err(_np(cache.s_group[:, :, :nc * (64 // w.g_s)]),
+                       S_g[:, :, :nc * (64 // w.g_s)]) < 2e-6
+
+
+def test_decode_full_budget_is_dense(gpu_lib):
+    w = TINY.replace(B=1, Hq=4, Hkv=2, K_c=64, K_g=256)
+    d, cache, out, lse, _, _ = run_decode(gpu_lib, w, 300, 30, 384, seed=9)
+    Ttot = 330
+    K = torch.cat([d["k_hist"], d["k_new"].transpose(0, 1)], 1)
+    V = torch.cat([d["v_hist"], d["v_new"].transpose(0, 1)], 1)
+    pos = torch.cat([d["pos_hist"], d["pos_new"].transpose(0, 1)], 1)
+    Q = torch.zeros(1, Ttot, w.Hq, w.D, dtype=torch.float64)
+    Q[:, 300:] = d["q"].transpose(0, 1).double()
+    O, _ = oracle.dense(Q, K, V, pos, w.theta)
+    assert row_rel_err(_np(out)[:, 0], O[0, 300:]) <= 1e-5
