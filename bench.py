@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-replays", type=int, default=10)
     ap.add_argument("--seq", type=int, default=0,
                     help="override the prefill length (small profiling cases only)")
     return ap.parse_args()
@@ -250,6 +252,109 @@ def run_reference(args, per_step=2):
     print(json.dumps(line), flush=True)
 
 
+DECODE_WORKLOAD = "qwen3_30b_a3b_bf16_decode_64k"
+
+
+def decode_bytes_per_step(w, T0, steps):
+    """Algorithmic HBM bytes of one decode step (average over the run): per
+    (sequence, KV head) the middle-chunk summary rows scanned, the group rows
+    of the routed chunks, the visible keys' K and V rows, and the step's own
+    q / k / v / cache writes / output."""
+    e = 2  # bf16
+    total = 0
+    for s in range(steps):
+        t = T0 + s
+        c = t // w.C
+        n_mid = max(0, (c - w.L - 1 if w.L > 0 else c - 2) - w.F + 1)
+        kc = min(w.K_c, n_mid)
+        kg = min(w.K_g, kc * (w.C // w.g_s))
+        nsink = min(w.F, c)
+        rec_lo = max(c - max(w.L, 1), nsink)
+        keys = (nsink + (c - rec_lo)) * w.C + kg * w.g_s + (t - c * w.C + 1)
+        per_head = (n_mid * w.D * 4 + kc * (w.C // w.g_s) * w.D * 4 + keys * w.D * e * 2
+                    + w.G * w.D * e * 2 + 2 * w.D * e + 3 * w.D * e)
+        total += per_head * w.Hkv * w.B
+    return total / steps
+
+
+def bench_decode(args, dev, world):
+    """16 sequences with a 64K-token cache, 256 decode steps captured in one
+    CUDA graph; steps/s and the HBM roofline of a step."""
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_kv_routing_b200 as hga
+    from workloads import WORKLOADS, make_decode_inputs
+    w = WORKLOADS[DECODE_WORKLOAD]
+    S = w.steps
+    hp = params_of(w)
+    d = make_decode_inputs(w, seed=args.seed + 1000 * (int(os.environ.get("RANK", "0")) + 1),
+                           device=dev)
+    cap = w.T + S
+    cache = hga.KVCache(w.B, cap, w.Hkv, w.D, torch.bfloat16, hp, device=dev)
+    hga.hga_fill_cache(d["k_hist"], d["v_hist"], d["pos_hist"], cache, hp)
+    del d["k_hist"], d["v_hist"]
+    ws = hga.decode_workspace(w.B, cap, w.Hq, w.Hkv, w.D, torch.bfloat16, hp, device=dev)
+    outs = torch.empty(S, w.B, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+    q, kn, vn, pn = d["q"], d["k_new"], d["v_new"], d["pos_new"]
+
+    def run_steps():
+        for s in range(S):
+            hga.hga_forward_decode(q[s], kn[s], vn[s], pn[s], cache, hp, out=outs[s],
+                                   workspace=ws)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            cache.lens.fill_(w.T)
+            run_steps()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    cache.lens.fill_(w.T)
+    with torch.cuda.graph(graph):
+        run_steps()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        cache.lens.fill_(w.T)
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    times = []
+    for _ in range(args.decode_replays):
+        cache.lens.fill_(w.T)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+    assert int(cache.lens[0].item()) == cap
+    tot = torch.tensor([sum(times)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    ms_step = float(tot.item()) / (len(times) * S)
+    del graph
+    pk, src = peaks()
+    bps = decode_bytes_per_step(w, w.T, S)
+    achieved = bps / (ms_step / 1e3) / 1e9
+    return {"metric": "decode steps/s", "value": world * 1e3 / ms_step, "unit": "steps/s",
+            "tokens_per_s": world * w.B * 1e3 / ms_step, "ms_per_step": ms_step,
+            "steps_per_replay": S, "replays": len(times),
+            "config": {"workload": w.name, "B": w.B, "cache_tokens": f"{w.T}..{cap - 1}",
+                       "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
+                       "graph": f"{S} steps captured in one CUDA graph, lens reset between "
+                                "replays outside the timed events"},
+            "gpu_launches_per_step": 2,
+            "roofline": {"bound": "hbm", "achieved": achieved,
+                         "peak": pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]), "unit": "GB/s",
+                         "frac": achieved / pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]),
+                         "traffic": None, "bytes_per_step": bps,
+                         "peak_source": f"{src} hbm_gbs (copy)"}}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -349,6 +454,7 @@ def main():
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hpos))
     d2h = hout.numel() * hout.element_size()
 
+    dec = None if args.no_decode else bench_decode(args, dev, world)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -374,6 +480,8 @@ def main():
             "gpu_launches": 3 * args.steps,
             "stage_ms": {"summaries": stage_ms[0], "route": stage_ms[1], "attend": stage_ms[2]},
             "roofline": roof}
+    if dec is not None:
+        line["decode"] = dec
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.seed)
     if args.seq or args.no_e2e:

@@ -22,7 +22,8 @@ import torch
 
 __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "hga_route",
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
-           "hga_workspace_size", "hga_forward_prefill_noalloc", "HGAError", "PREFILL",
+           "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
+           "decode_workspace", "HGAError", "PREFILL",
            "DECODE"]
 
 PREFILL, DECODE = 0, 1
@@ -317,6 +318,25 @@ def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCa
                          None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
     _check(st, "hga_forward(prefill)")
     return res
+
+
+def hga_fill_cache(k, v, pos, cache: "KVCache", params: HGAParams, *, stream=None):
+    """Fill a decode cache from a prompt's raw keys, values and positions
+    (stage 1 only: rotated keys, values, positions, summaries, lens = T)."""
+    lib = load()
+    _need(k, "k")
+    B, T, Hkv, D = k.shape
+    _need(v, "v", (B, T, Hkv, D), k.dtype)
+    _need(pos, "pos", (B, T), torch.int32)
+    io = _IO()
+    io.k, io.v, io.pos = k.data_ptr(), v.data_ptr(), pos.data_ptr()
+    io.cache = cache.c()
+    dims = _dims(B, T, Hkv, Hkv, D, _dtype_code(k))
+    pc = params.c()
+    st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io), None, 0,
+                         _stream(stream))
+    _check(st, "hga_forward(prefill, cache fill)")
+    return cache
 
 
 def hga_forward_prefill_noalloc(q, k, v, pos, params: HGAParams, out: torch.Tensor, *,

@@ -3,6 +3,8 @@
 // enqueued on the caller's stream.
 #include <cmath>
 #include <cstring>
+#include <mutex>
+#include <unordered_map>
 
 #include "hga_internal.cuh"
 #include "route_common.cuh"
@@ -15,6 +17,18 @@ hga_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return HGA_OK;
     g_last_cuda_error = (int)e;
     return HGA_ERR_CUDA;
+}
+
+cudaError_t ensure_smem(const void *kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::unordered_map<const void *, size_t> granted;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &have = granted[kernel];
+    if (bytes <= have) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) have = bytes;
+    return e;
 }
 
 hga_status set_rope(Rope *r, int D, double theta, double hf_wavelength, int C) {
@@ -177,17 +191,22 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
     const size_t need = hga_workspace_size(mode, dims, prm);
-    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
-        return HGA_ERR_WORKSPACE;
+    const bool ws_ok =
+        need == 0 || (workspace && workspace_bytes >= need && !((uintptr_t)workspace & 255u));
     char *ws = static_cast<char *>(workspace);
 
     if (mode == HGA_PREFILL) {
         if (dims->T == 0) return HGA_OK;
-        if (!io->q || !io->k || !io->v || !io->pos || !io->out) return HGA_ERR_INVALID_ARG;
-        if (!aligned16(io->q) || !aligned16(io->k) || !aligned16(io->v) || !aligned16(io->out))
-            return HGA_ERR_INVALID_ARG;
         const hga_kv_cache &cc = io->cache;
         const bool fill = cc.k_rot != nullptr;
+        // cache fill only: no queries, no output (stage 1 into the cache)
+        const bool fill_only = fill && !io->q && !io->out;
+        if (!io->k || !io->v || !io->pos || (!fill_only && (!io->q || !io->out)))
+            return HGA_ERR_INVALID_ARG;
+        if ((io->q && !aligned16(io->q)) || !aligned16(io->k) || !aligned16(io->v) ||
+            (io->out && !aligned16(io->out)))
+            return HGA_ERR_INVALID_ARG;
+        if (!fill_only && !ws_ok) return HGA_ERR_WORKSPACE;   // fill only needs none
         if (fill) {
             if (cc.capacity < dims->T || cc.capacity % prm->C || !cc.v || !cc.pos || !cc.k_open ||
                 !cc.s_chunk || !cc.s_group || !cc.lens)
@@ -207,7 +226,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
         s = launch_summaries(g, r, dims->dtype, io->k, fill ? io->v : nullptr, io->pos, g.T, k_rot,
                              fill ? cc.v : nullptr, fill ? cc.pos : nullptr, k_T, s_chunk, s_group,
                              nc_cap, fill ? cc.k_open : nullptr, fill ? cc.lens : nullptr, st);
-        if (s != HGA_OK) return s;
+        if (s != HGA_OK || fill_only) return s;
         s = launch_route(g, r, dims->dtype, io->q, io->pos, s_chunk, s_group, nc_cap, sel_c, sel_g,
                          st);
         if (s != HGA_OK) return s;
@@ -215,6 +234,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
                                io->out, io->lse, st);
     }
     if (mode == HGA_DECODE) {
+        if (!ws_ok) return HGA_ERR_WORKSPACE;
         const hga_kv_cache &cc = io->cache;
         if (!io->q_new || !io->k_new || !io->v_new || !io->pos_new || !io->out) return HGA_ERR_INVALID_ARG;
         if (!cc.k_rot || !cc.v || !cc.pos || !cc.k_open || !cc.s_chunk || !cc.s_group || !cc.lens)

@@ -157,7 +157,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     const size_t smem = attend_simt_smem(g);
     if (smem > 200 * 1024) return HGA_ERR_UNSUPPORTED;
     auto kern = k_attend_simt<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     const int n_rc = (kChunk * g.G + kRows - 1) / kRows;
     dim3 grid(g.NB * n_rc, g.Hkv, g.B);

@@ -491,7 +491,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         return HGA_ERR_CUDA;
     const size_t smem = Cfg<D>::oEnd + 1024;
     auto kern = k_attend_tc<D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(g.NB * a.ctas_per_unit, g.Hkv, g.B);
     kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, a);

@@ -441,9 +441,9 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     if (smem_scan > 200 * 1024 || smem_att > 200 * 1024) return HGA_ERR_UNSUPPORTED;
     auto ks = k_decode_scan<T, D>;
     auto ka = k_decode_attend<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_scan);
+    cudaError_t e = ensure_smem((const void *)ks, smem_scan);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_att);
+        e = ensure_smem((const void *)ka, smem_att);
     if (e != cudaSuccess) return cuda_status(e);
     ks<<<dim3(A.ns_scan, g.Hkv, g.B), kThreads, smem_scan, st>>>(A);
     e = cudaGetLastError();

@@ -92,6 +92,11 @@ __device__ __forceinline__ int middle_hi(int c, int L) { return L == 0 ? c - 2 :
 hga_status set_rope(Rope *r, int D, double theta, double hf_wavelength, int C);
 hga_status cuda_status(cudaError_t e);
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes`, calling
+// cudaFuncSetAttribute only when the limit has to grow (so repeated launches,
+// including launches inside a stream capture, make no such call).
+cudaError_t ensure_smem(const void *kernel, size_t bytes);
+
 // Stage 1.  k_rot/v_out/pos_out/k_open/lens may be null.  in_T: tokens per
 // sequence of the inputs; out_T: token capacity of k_rot/v_out/pos_out;
 // nc_cap: chunk capacity of s_chunk/s_group.

@@ -127,8 +127,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     if (smem > 160 * 1024) return HGA_ERR_UNSUPPORTED;   // candidate table must fit on chip
     auto kern = k_route<T, D>;
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = ensure_smem((const void *)kern, smem);
         if (e != cudaSuccess) return cuda_status(e);
     }
     dim3 grid(g.NB, g.Hkv, g.B);

@@ -139,7 +139,7 @@ hga_status run(const Geo &g, const Rope &r, const void *k_raw, const void *v_raw
                int32_t *lens, cudaStream_t st) {
     const size_t smem = sizeof(float2) * kChunk * (D / 2) + sizeof(float) * kChunk * D;
     auto kern = k_summaries<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid((in_T + kChunk - 1) / kChunk, g.B);
     kern<<<grid, kThreads, smem, st>>>(

@@ -169,7 +169,9 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  * HGA_PREFILL: stages 1-3 over the T prompt tokens (K_rot, summaries and
  *   selections live in the workspace unless io.cache / io.sel_* are given).
  *   With io.cache.k_rot set (capacity >= T), the cache is filled for decoding:
- *   K_rot, V, pos, summaries, the open chunk's raw keys, and lens = T.
+ *   K_rot, V, pos, summaries, the open chunk's raw keys, and lens = T.  With
+ *   the cache set and io.q and io.out both NULL, only the cache is filled
+ *   (stage 1; no routing or attention is computed).
  * HGA_DECODE: dims.T must equal io.cache.capacity.  For each sequence b, appends the new token at t = lens[b]
  *   (rotated key, value, position, raw key of the open chunk), builds the
  *   summaries of chunk t/C if t closes it (page section 3, store operation

@@ -82,7 +82,7 @@ def test_null_buffers_rejected(lib):
     assert st == 1
     io = hga._IO()
     st = lib.hga_forward(0, ctypes.byref(d), ctypes.byref(p), ctypes.byref(io), None, 0, None)
-    assert st == 6  # workspace checked first (prefill needs one)
+    assert st == 1  # null inputs are rejected before the workspace is looked at
 
 
 def test_binding_fails_loudly_without_cuda():

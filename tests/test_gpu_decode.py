@@ -115,3 +115,85 @@ def test_decode_full_budget_is_dense(gpu_lib):
     Q[:, 300:] = d["q"].transpose(0, 1).double()
     O, _ = oracle.dense(Q, K, V, pos, w.theta)
     assert row_rel_err(_np(out)[:, 0], O[0, 300:]) <= 1e-5
+
+
+@pytest.mark.slow
+def test_decode_64k_full_size_graph(gpu_lib):
+    """The bench's decode configuration: 16 sequences with a 65536-token cache,
+    256 steps captured in one CUDA graph.  Every step's routed sets of two
+    sampled sequences and sampled steps' outputs are checked against the
+    oracle's full recompute; lens and the summaries of the chunks closed by
+    the run are checked for all sequences."""
+    hga = gpu_lib
+    w = QWEN
+    S = w.steps
+    dev = torch.device("cuda")
+    hp = _hp(hga, w)
+    d = make_decode_inputs(w, seed=21, device=dev)
+    cap = w.T + S
+    cache = hga.KVCache(w.B, cap, w.Hkv, w.D, torch.bfloat16, hp, device=dev)
+    hga.hga_fill_cache(d["k_hist"], d["v_hist"], d["pos_hist"], cache, hp)
+    ws = hga.decode_workspace(w.B, cap, w.Hq, w.Hkv, w.D, torch.bfloat16, hp, device=dev)
+    outs = torch.empty(S, w.B, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+    sels = torch.empty(S, w.B, w.Hkv, w.K_g, dtype=torch.int32, device=dev)
+    selc = torch.empty(S, w.B, w.Hkv, w.K_c, dtype=torch.int32, device=dev)
+    import ctypes
+
+    def run_steps():
+        for s in range(S):
+            io = hga._IO()
+            io.q_new, io.k_new = d["q"][s].data_ptr(), d["k_new"][s].data_ptr()
+            io.v_new, io.pos_new = d["v_new"][s].data_ptr(), d["pos_new"][s].data_ptr()
+            io.out = outs[s].data_ptr()
+            io.sel_chunk, io.sel_group = selc[s].data_ptr(), sels[s].data_ptr()
+            io.cache = cache.c()
+            dims = hga._Dims(w.B, cap, w.Hq, w.Hkv, w.D, 1)
+            pc = hp.c()
+            base = (ws.data_ptr() + 255) // 256 * 256
+            st = hga.load().hga_forward(hga.DECODE, ctypes.byref(dims), ctypes.byref(pc),
+                                        ctypes.byref(io), ctypes.c_void_p(base),
+                                        ws.numel() - 256, hga._stream(None))
+            assert st == 0
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run_steps()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    cache.lens.fill_(w.T)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_steps()
+    cache.lens.fill_(w.T)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert (cache.lens == cap).all()
+    p = oracle.Params.of(w)
+    tol = TOL[w.dtype]
+    for b in (3, 11):
+        K = torch.cat([d["k_hist"][b], d["k_new"][:, b]], 0)[None].cpu()
+        V = torch.cat([d["v_hist"][b], d["v_new"][:, b]], 0)[None].cpu()
+        pos = torch.cat([d["pos_hist"][b], d["pos_new"][:, b]], 0)[None].cpu()
+        steps = list(range(S))
+        Q = np.zeros((1, cap, w.Hq, w.D))
+        Q[0, w.T:] = d["q"][:, b].double().cpu().numpy()
+        units = [(0, w.T + s) for s in steps]
+        rr = oracle.hga(Q, K, V, pos, p, route_block=1, units=units, attend=False)
+        ref = RouteRef(Q, K, pos, p, w.Hkv)
+        sc, sg = selc[:, b].cpu().numpy(), sels[:, b].cpu().numpy()
+        for i, (_, t) in enumerate(units):
+            for h in range(w.Hkv):
+                ok, _ = check_unit_selection(ref, 0, h, t, t + 1, t // 64, sc[t - w.T, h],
+                                             sg[t - w.T, h], rr["sel_c"][i, h], rr["sel_g"][i, h])
+                assert ok, f"routing mismatch b={b} t={t} h={h}"
+        sample = [0, 1, 63, 64, 127, 128, 200, S - 1]
+        u2 = [(0, w.T + s) for s in sample]
+        force = np.stack([sg[s] for s in sample])
+        orc = oracle.hga(Q, K, V, pos, p, route_block=1, units=u2, sel_g_force=force)
+        O = outs[:, b].float().cpu().numpy()
+        for s in sample:
+            e = row_rel_err(O[s], orc["O"][0, w.T + s])
+            assert e <= tol, f"decode output rel err {e} at b={b} step={s}"
+        S_c, _ = oracle.build_summaries(K, pos, p)
+        assert row_rel_err(_np(cache.s_chunk[b:b + 1]), S_c) < 2e-6
