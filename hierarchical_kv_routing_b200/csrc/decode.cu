@@ -8,28 +8,32 @@
 // The pages check decode against a full recompute (Table 7); the tests here
 // do the same against the oracle.
 //
-// Two kernels per step, both HBM-bound:
-//   k_decode_scan   grid (scan splits, KV heads, sequences).  Split 0 of each
-//                   (sequence, KV head) appends the token (rotated key, value,
-//                   position, raw key into the open-chunk buffer) and, when the
-//                   token closes its chunk, writes that chunk's summaries.  Every
-//                   split scores its 64-chunk slice of the middle-chunk table
-//                   with the token's routing query (fp64 accumulation) and
-//                   keeps its top K_c keys; the last split to finish (atomic
-//                   counter) merges them, scores the groups of the chosen
-//                   chunks and keeps the top K_g.
-//   k_decode_attend grid (key splits, KV heads, sequences).  Each CTA takes a
-//                   slice of the token's visible key list, stages its K/V rows
-//                   in shared memory with 16-byte loads, and computes partial
-//                   softmax sums for the KV head's G query heads; the last CTA
-//                   per (sequence, KV head) combines the partials, and the last
-//                   of those per sequence increments lens.
+// Two kernels per step, both HBM-bound.  The visible set splits into a part
+// routing does not touch (sinks, recent chunks, the current chunk) and the
+// routed groups, so the first kernel attends over the fixed part while it
+// routes, and the second only has to add the routed groups.
+//   k_decode_a  grid (scan splits + fixed splits, KV heads, sequences)
+//     scan CTAs   split 0 appends the token (rotated key, value, position,
+//                 raw key of the open chunk) and, when the token closes its
+//                 chunk, writes that chunk's summaries.  Each scan CTA scores
+//                 256 middle chunks, one summary row per thread (fp64 dot
+//                 products), and keeps its top K_c keys; the last one to
+//                 finish (atomic counter) merges them, scores the groups of the
+//                 chosen chunks and keeps the top K_g.
+//     fixed CTAs  attend the KV head's G query heads over a slice of the fixed
+//                 keys (the new token's key and value straight from the step's
+//                 inputs, everything else from the cache) and write partial
+//                 softmax sums.
+//   k_decode_b  grid (routed splits, KV heads, sequences), launched as a
+//               programmatic dependent of k_decode_a: it rotates the queries,
+//               then waits for k_decode_a, attends over a slice of the routed
+//               groups, and the last CTA per (sequence, KV head) combines all
+//               partials; the last of those per sequence increments lens.
 // Counters live in the workspace; each last CTA resets its counter, so the
 // workspace only has to be zeroed before its first use.
 #include "hga_internal.cuh"
 #include "route_common.cuh"
 #include "vec.cuh"
-#include "visible.cuh"
 
 namespace hga {
 
@@ -38,11 +42,15 @@ __device__ int g_decode_error = 0;
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kScanChunks = 64;   // middle chunks per scan split
-constexpr int kAttSplits = 8;     // key-list splits per (sequence, KV head)
+constexpr int kScanChunks = 256;  // middle chunks per scan CTA (one per thread)
+constexpr int kFixSplits = 4;     // CTAs over the fixed keys per (sequence, KV head)
+constexpr int kRouteSplits = 4;   // CTAs over the routed keys
+constexpr int kParts = kFixSplits + kRouteSplits;
+constexpr int kMaxG = 16;
+constexpr int kMaxCand = 1024;    // merge and group candidate table
 
 struct DecodeArgs {
-    int B, Tc, Hq, Hkv, G, C, g_s, gpc, F, L, K_c, K_g, nc_cap, ns_scan, keys_max, per_max;
+    int B, Tc, Hq, Hkv, G, C, g_s, gpc, F, L, K_c, K_g, nc_cap, ns_scan;
     const void *q_new, *k_new, *v_new;
     const int32_t *pos_new;
     void *k_rot, *v;
@@ -54,16 +62,11 @@ struct DecodeArgs {
     float *lse;
     int32_t *sel_c, *sel_g;          // [B, Hkv, K]
     unsigned long long *cand;        // [B, Hkv, ns_scan, K_c]
-    float *part;                     // [B, Hq, kAttSplits, D + 2]
+    float *part;                     // [B, Hq, kParts, D + 2]
     int32_t *scan_done, *att_done, *seq_done;
     float scale_log2;
     Rope rope;
 };
-
-template <typename T>
-__device__ __forceinline__ float ld_elem(const T *p) {
-    return to_f(*p);
-}
 
 // Summaries of chunk c of (b, h) from the open-chunk raw keys (its last key
 // was written by this CTA just before), positions from the cache except the
@@ -83,7 +86,7 @@ __device__ void close_chunk(const DecodeArgs &A, int b, int h, int c, int32_t po
         for (int j = lo; j < lo + cnt; ++j) {
             const int32_t pj = j == A.C - 1 ? pos_last : pc[j];
             pm += (double)pj;
-            const float x = ld_elem(ko + (int64_t)j * D + i), y = ld_elem(ko + (int64_t)j * D + i + H);
+            const float x = to_f(ko[(int64_t)j * D + i]), y = to_f(ko[(int64_t)j * D + i + H]);
             if (hf) {
                 const float2 r = rope_cs(A.rope, (double)pj, i);
                 a += (double)(x * r.x - y * r.y);
@@ -109,15 +112,174 @@ __device__ void close_chunk(const DecodeArgs &A, int b, int h, int c, int32_t po
     }
 }
 
+// Rotated, pre-scaled queries of the KV head's G heads -> qs[G][D].
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) k_decode_scan(const DecodeArgs A) {
+__device__ __forceinline__ void load_queries(const DecodeArgs &A, int b, int h, int32_t pnew,
+                                             float *qs) {
     constexpr int H = D / 2;
-    extern __shared__ __align__(16) unsigned char smem[];
-    unsigned long long *cand = reinterpret_cast<unsigned long long *>(smem);
-    __shared__ double qr[D];
-    __shared__ RouteScratch rs;
-    __shared__ int s_last;
+    const T *qb = static_cast<const T *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
+    for (int e = threadIdx.x; e < A.G * H; e += blockDim.x) {
+        const int g = e / H, i = e % H;
+        const float2 r = rope_cs(A.rope, (double)pnew, i);
+        const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
+        qs[g * D + i] = (x * r.x - y * r.y) * A.scale_log2;
+        qs[g * D + i + H] = (y * r.x + x * r.y) * A.scale_log2;
+    }
+}
 
+// The step's new key, rotated and rounded to the cache's type exactly like
+// the appended row, into knew[D] (shared, cache type), by D/2 threads.
+template <typename T, int D>
+__device__ __forceinline__ void rotate_new_key(const DecodeArgs &A, int b, int h, int32_t pnew,
+                                               T *knew) {
+    constexpr int H = D / 2;
+    if (threadIdx.x < H) {
+        const int i = threadIdx.x;
+        const T *kn = static_cast<const T *>(A.k_new) + ((int64_t)b * A.Hkv + h) * D;
+        const float x = to_f(kn[i]), y = to_f(kn[i + H]);
+        const float2 r = rope_cs(A.rope, (double)pnew, i);
+        knew[i] = from_f<T>(x * r.x - y * r.y);
+        knew[i + H] = from_f<T>(y * r.x + x * r.y);
+    }
+}
+
+// q . k for one packed 16-byte slice of k (8 bf16 or 4 fp32 values).
+template <typename T>
+__device__ __forceinline__ float dot16(const uint4 &w, const float *q) {
+    if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
+        const float4 qa = *reinterpret_cast<const float4 *>(q);
+        const float4 qb = *reinterpret_cast<const float4 *>(q + 4);
+        const float2 a = __bfloat1622float2(h2[0]), b = __bfloat1622float2(h2[1]);
+        const float2 c = __bfloat1622float2(h2[2]), d = __bfloat1622float2(h2[3]);
+        float s = qa.x * a.x;
+        s = fmaf(qa.y, a.y, s);
+        s = fmaf(qa.z, b.x, s);
+        s = fmaf(qa.w, b.y, s);
+        s = fmaf(qb.x, c.x, s);
+        s = fmaf(qb.y, c.y, s);
+        s = fmaf(qb.z, d.x, s);
+        return fmaf(qb.w, d.y, s);
+    } else {
+        const float4 qa = *reinterpret_cast<const float4 *>(q);
+        float s = qa.x * __uint_as_float(w.x);
+        s = fmaf(qa.y, __uint_as_float(w.y), s);
+        s = fmaf(qa.z, __uint_as_float(w.z), s);
+        return fmaf(qa.w, __uint_as_float(w.w), s);
+    }
+}
+
+// Partial attention of the G heads over keys key_of(0..nk), nk <= blockDim:
+// scores one key per thread, softmax and P.V one warp per head with lanes
+// over dims; writes (m, l, o[D]) for part index `pi`.
+template <typename T, int D, typename KeyOf>
+__device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, KeyOf key_of,
+                            int pi, const float *qs, const T *knew, float *sc, int *kt_s) {
+    constexpr int DL = D / 32;
+    constexpr int NV = D * (int)sizeof(T) / 16;     // 16-byte slices per row
+    constexpr int EV = 16 / (int)sizeof(T);         // elements per slice
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int k = threadIdx.x; k < nk; k += blockDim.x) {
+        const int kt = key_of(k);
+        kt_s[k] = kt;
+        const uint4 *src = kt == t
+            ? reinterpret_cast<const uint4 *>(knew)
+            : reinterpret_cast<const uint4 *>(static_cast<const T *>(A.k_rot) +
+                                              (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D);
+        uint4 kw[NV];
+#pragma unroll
+        for (int e = 0; e < NV; ++e) kw[e] = kt == t ? src[e] : __ldg(src + e);
+#pragma unroll 1
+        for (int g = 0; g < A.G; ++g) {
+            const float *qg = qs + g * D;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < NV; e += 2) {
+                a0 += dot16<T>(kw[e], qg + e * EV);
+                a1 += dot16<T>(kw[e + 1], qg + (e + 1) * EV);
+            }
+            sc[g * kThreads + k] = a0 + a1;
+        }
+    }
+    __syncthreads();
+    const T *vbase = static_cast<const T *>(A.v);
+    const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
+    float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
+    for (int g = warp; g < A.G; g += nw) {
+        float m = -INFINITY;
+        for (int k = lane; k < nk; k += 32) m = fmaxf(m, sc[g * kThreads + k]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        for (int k = lane; k < nk; k += 32) {
+            const float p = exp2f(sc[g * kThreads + k] - m);
+            sc[g * kThreads + k] = p;
+            l += p;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        __syncwarp();
+        float acc[DL];
+#pragma unroll
+        for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+        for (int k = 0; k < nk; ++k) {
+            const float p = sc[g * kThreads + k];
+            const int kt = kt_s[k];
+            const T *vr = kt == t ? vn : vbase + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D;
+            float vv[DL];
+#pragma unroll
+            for (int e = 0; e < DL; ++e) vv[e] = to_f(vr[lane * DL + e]);
+#pragma unroll
+            for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
+        }
+        float *dst = part_b + ((int64_t)g * kParts + pi) * (D + 2);
+#pragma unroll
+        for (int e = 0; e < DL; ++e) dst[2 + lane * DL + e] = acc[e];
+        if (lane == 0) {
+            dst[0] = nk > 0 ? m : -INFINITY;
+            dst[1] = l;
+        }
+    }
+}
+
+// Shared memory of k_decode_a: the scan and fixed-attention roles never meet
+// in one CTA, so their buffers share one pool.
+template <typename T, int D>
+struct ScanSmem {
+    double qr[D];
+    unsigned long long cand[kMaxCand];
+    unsigned long long lists[kThreads];
+    RouteScratch rs;
+};
+template <typename T, int D>
+struct AttSmem {
+    float qs[kMaxG * D];
+    T knew[D];
+    float sc[kMaxG * kThreads];
+    int kt_s[kThreads];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
+    constexpr int H = D / 2;
+    constexpr size_t kPool = sizeof(ScanSmem<T, D>) > sizeof(AttSmem<T, D>)
+                                 ? sizeof(ScanSmem<T, D>) : sizeof(AttSmem<T, D>);
+    __shared__ __align__(16) unsigned char pool[kPool];
+    __shared__ int s_last;
+    ScanSmem<T, D> &ss = *reinterpret_cast<ScanSmem<T, D> *>(pool);
+    AttSmem<T, D> &as = *reinterpret_cast<AttSmem<T, D> *>(pool);
+    double *qr = ss.qr;
+    unsigned long long *cand = ss.cand;
+    unsigned long long *lists = ss.lists;
+    RouteScratch &rs = ss.rs;
+    int *sel_c = rs.sel_c, *sel_g = rs.sel_g;
+    float *qs = as.qs;
+    T *knew = as.knew;
+    float *sc = as.sc;
+    int *kt_s = as.kt_s;
+
+    // let the routed-keys kernel launch now; it waits for this grid itself
+    asm volatile("griddepcontrol.launch_dependents;");
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
     if (t < 0 || t >= A.Tc) {
@@ -127,7 +289,27 @@ __global__ void __launch_bounds__(kThreads) k_decode_scan(const DecodeArgs A) {
     const int c = t / A.C;
     const int32_t pnew = A.pos_new[b];
 
-    // ---- append (split 0 of each KV head)
+    if (s >= A.ns_scan) {
+        // ------------------------------------------- fixed-key attention --
+        const int f = s - A.ns_scan;
+        const int nsink = min(A.F, c);
+        const int rec_lo = max(c - max(A.L, 1), nsink);
+        const int n1 = nsink * A.C, n2 = n1 + (c - rec_lo) * A.C;
+        const int nfix = n2 + (t - c * A.C + 1);
+        const int per = (nfix + kFixSplits - 1) / kFixSplits;
+        const int k0 = min(nfix, f * per), nk = min(nfix, k0 + per) - k0;
+        load_queries<T, D>(A, b, h, pnew, qs);
+        rotate_new_key<T, D>(A, b, h, pnew, knew);
+        __syncthreads();
+        auto key_of = [&](int k) {
+            const int i = k0 + k;
+            return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
+        };
+        attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s);
+        return;
+    }
+
+    // ------------------------------------------------------------- scan --
     if (s == 0) {
         const T *kn = static_cast<const T *>(A.k_new) + ((int64_t)b * A.Hkv + h) * D;
         const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
@@ -149,7 +331,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_scan(const DecodeArgs A) {
         if (t % A.C == A.C - 1) close_chunk<T, D>(A, b, h, c, pnew);
     }
 
-    // ---- routing query of the token: sum over the KV head's query heads
+    // routing query of the token: the KV head's query heads summed, in fp64
     if (threadIdx.x < H) {
         const int i = threadIdx.x;
         const float2 r = rope_cs(A.rope, (double)pnew, i);
@@ -165,18 +347,22 @@ __global__ void __launch_bounds__(kThreads) k_decode_scan(const DecodeArgs A) {
     }
     __syncthreads();
 
-    // ---- this split's slice of the middle chunks, top K_c keys
+    // this CTA's slice of the middle chunks, one row per thread
     const int mlo = A.F, mhi = middle_hi(c, A.L);
     const int first = max(mlo, s * kScanChunks);
     const int last = min(mhi, s * kScanChunks + kScanChunks - 1);
     const int n = max(0, last - first + 1);
     const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
-    score_rows<D>(qr, Sc, first, n, cand);
+    if (threadIdx.x < n)
+        cand[threadIdx.x] = pack_key(
+            (float)thread_dot_row<D>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
+            first + threadIdx.x);
     __syncthreads();
     unsigned long long *mine = A.cand + (((int64_t)b * A.Hkv + h) * A.ns_scan + s) * A.K_c;
-    topk_keys(cand, n, A.K_c, mine, rs);
+    if (A.K_c <= 32) block_topk32_keys(cand, n, A.K_c, mine, lists);
+    else topk_keys(cand, n, A.K_c, mine, rs);
 
-    // ---- the last split merges and routes the groups
+    // the last scan CTA of (b, h) merges and routes the groups
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -190,164 +376,107 @@ __global__ void __launch_bounds__(kThreads) k_decode_scan(const DecodeArgs A) {
     const int ntot = A.ns_scan * A.K_c;
     for (int r = threadIdx.x; r < ntot; r += blockDim.x) cand[r] = __ldcg(all + r);
     __syncthreads();
-    // keys of 0 are padding: they never beat a real key, and only min(K_c,
-    // real) keys are kept, so count the real ones
-    int nreal = 0;
-    for (int r = 0; r < ntot; ++r) nreal += cand[r] != 0;
-    // compact (stable) so padding does not count as a candidate
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int w = 0;
-        for (int r = 0; r < ntot; ++r)
-            if (cand[r] != 0) cand[w++] = cand[r];
+    int kc;
+    if (A.K_c <= 32) {
+        block_topk32(cand, ntot, A.K_c, sel_c, lists);    // padding keys (0) never win
+        kc = 0;
+        for (int r = 0; r < A.K_c; ++r) kc += sel_c[r] >= 0;
+    } else {
+        if (threadIdx.x == 0) {               // drop the padding, keep the order
+            int w = 0;
+            for (int r = 0; r < ntot; ++r)
+                if (cand[r]) cand[w++] = cand[r];
+            s_last = w;
+        }
+        __syncthreads();
+        kc = topk_select(cand, s_last, A.K_c, sel_c, rs);
+        for (int r = kc + threadIdx.x; r < A.K_c; r += blockDim.x) sel_c[r] = -1;
+        __syncthreads();
+    }
+    int32_t *oc = A.sel_c + ((int64_t)b * A.Hkv + h) * A.K_c;
+    for (int r = threadIdx.x; r < A.K_c; r += blockDim.x) oc[r] = sel_c[r];
+    const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
+    const int ng = kc * A.gpc;
+    for (int r = threadIdx.x; r < ng; r += blockDim.x) {
+        const int gid = sel_c[r / A.gpc] * A.gpc + r % A.gpc;
+        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sg + (int64_t)gid * D), gid);
     }
     __syncthreads();
-    const int kc = topk_select(cand, nreal, A.K_c, rs.sel_c, rs);
-    int32_t *oc = A.sel_c + ((int64_t)b * A.Hkv + h) * A.K_c;
-    for (int r = threadIdx.x; r < A.K_c; r += blockDim.x) oc[r] = r < kc ? rs.sel_c[r] : -1;
-    const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
-    __syncthreads();
-    score_group_rows<D>(qr, Sg, rs.sel_c, A.gpc, kc * A.gpc, cand);
-    __syncthreads();
-    const int kg = topk_select(cand, kc * A.gpc, A.K_g, rs.sel_g, rs);
+    if (A.K_g <= 32) {
+        block_topk32(cand, ng, A.K_g, sel_g, lists);
+    } else {
+        const int kg = topk_select(cand, ng, A.K_g, sel_g, rs);
+        for (int r = kg + threadIdx.x; r < A.K_g; r += blockDim.x) sel_g[r] = -1;
+        __syncthreads();
+    }
     int32_t *og = A.sel_g + ((int64_t)b * A.Hkv + h) * A.K_g;
-    for (int r = threadIdx.x; r < A.K_g; r += blockDim.x) og[r] = r < kg ? rs.sel_g[r] : -1;
+    for (int r = threadIdx.x; r < A.K_g; r += blockDim.x) og[r] = sel_g[r];
     if (threadIdx.x == 0) A.scan_done[b * A.Hkv + h] = 0;
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) k_decode_attend(const DecodeArgs A) {
-    constexpr int H = D / 2, DL = D / 32;   // dims per lane
-    extern __shared__ __align__(16) unsigned char smem[];
-    // regions: keys (int, keys_max rounded to 4), q [G][D], scores [G][per_max]
-    // (per_max a multiple of 4), K and V rows [per_max][D]; all 16-byte aligned
-    int *keys = reinterpret_cast<int *>(smem);
-    float *qs = reinterpret_cast<float *>(smem + sizeof(int) * ((A.keys_max + 3) & ~3));
-    float *sc = qs + A.G * D;
-    T *Ks = reinterpret_cast<T *>(sc + A.G * A.per_max);
-    T *Vs = Ks + (size_t)A.per_max * D;
-    __shared__ RunList rl;
-    __shared__ int s_last, s_seq_last;
+__global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
+    constexpr int DL = D / 32;
+    __shared__ __align__(16) float qs[kMaxG * D];
+    __shared__ __align__(16) T knew[D];
+    __shared__ float sc[kMaxG * kThreads];
+    __shared__ int kt_s[kThreads];
+    __shared__ int sel[kMaxK];
+    __shared__ int s_last;
 
-    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    const int t = A.lens[b];
-    if (t < 0 || t >= A.Tc) return;
-    const int c = t / A.C;
+    const int t = A.lens[b];          // written only by the previous step
     const int32_t pnew = A.pos_new[b];
-
-    if (threadIdx.x == 0)
-        build_runs(rl, c, A.F, A.L, A.g_s, A.sel_g + ((int64_t)b * A.Hkv + h) * A.K_g, A.K_g,
-                   t - c * A.C + 1);
-    // rotated, pre-scaled queries of the G heads
-    const T *qb = static_cast<const T *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
-    for (int e = threadIdx.x; e < A.G * H; e += blockDim.x) {
-        const int g = e / H, i = e % H;
-        const float2 r = rope_cs(A.rope, (double)pnew, i);
-        const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
-        qs[g * D + i] = (x * r.x - y * r.y) * A.scale_log2;
-        qs[g * D + i + H] = (y * r.x + x * r.y) * A.scale_log2;
-    }
+    if (t >= 0 && t < A.Tc) load_queries<T, D>(A, b, h, pnew, qs);
+    // everything below reads what k_decode_a wrote
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (t < 0 || t >= A.Tc) return;
+    for (int j = threadIdx.x; j < A.K_g; j += blockDim.x)
+        sel[j] = A.sel_g[((int64_t)b * A.Hkv + h) * A.K_g + j];
     __syncthreads();
-    fill_keys(rl, keys);
-    const int nkeys = rl.off[rl.n];
-    const int per = (nkeys + kAttSplits - 1) / kAttSplits;
-    const int k0 = min(nkeys, s * per), nk = min(nkeys, k0 + per) - k0;
-    __syncthreads();
+    int kg = 0;
+    for (int j = 0; j < A.K_g; ++j) kg += sel[j] >= 0;
+    const int nrt = kg * A.g_s;
+    const int per = (nrt + kRouteSplits - 1) / kRouteSplits;
+    const int k0 = min(nrt, r * per), nk = min(nrt, k0 + per) - k0;
+    auto key_of = [&](int k) {
+        const int i = k0 + k;
+        return sel[i / A.g_s] * A.g_s + i % A.g_s;
+    };
+    attend_part<T, D>(A, b, h, t, nk, key_of, kFixSplits + r, qs, knew, sc, kt_s);
 
-    // stage this slice's K and V rows (16-byte loads)
-    constexpr int VPR = D * (int)sizeof(T) / 16;   // 16-byte vectors per row
-    const T *kbase = static_cast<const T *>(A.k_rot);
-    const T *vbase = static_cast<const T *>(A.v);
-    for (int e = threadIdx.x; e < nk * VPR; e += blockDim.x) {
-        const int k = e / VPR, part = e % VPR;
-        const int64_t row = ((int64_t)b * A.Tc + keys[k0 + k]) * A.Hkv + h;
-        reinterpret_cast<uint4 *>(Ks + (size_t)k * D)[part] =
-            __ldg(reinterpret_cast<const uint4 *>(kbase + row * D) + part);
-        reinterpret_cast<uint4 *>(Vs + (size_t)k * D)[part] =
-            __ldg(reinterpret_cast<const uint4 *>(vbase + row * D) + part);
-    }
-    __syncthreads();
-
-    // scores: one warp per key, lanes over dims, all G heads
-    for (int k = warp; k < nk; k += nw) {
-        float kv[DL];
-#pragma unroll
-        for (int e = 0; e < DL; ++e) kv[e] = to_f(Ks[(size_t)k * D + lane * DL + e]);
-        for (int g = 0; g < A.G; ++g) {
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < DL; ++e) a = fmaf(qs[g * D + lane * DL + e], kv[e], a);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            if (lane == 0) sc[g * A.per_max + k] = a;
-        }
-    }
-    __syncthreads();
-
-    // per head: max, exponentials, sum, then P.V over this slice
-    float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kAttSplits * (D + 2);
-    for (int g = warp; g < A.G; g += nw) {
-        float m = -INFINITY;
-        for (int k = lane; k < nk; k += 32) m = fmaxf(m, sc[g * A.per_max + k]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int k = lane; k < nk; k += 32) {
-            const float p = nk > 0 ? exp2f(sc[g * A.per_max + k] - m) : 0.f;
-            sc[g * A.per_max + k] = p;
-            l += p;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        __syncwarp();
-        float o_acc[DL];
-#pragma unroll
-        for (int e = 0; e < DL; ++e) o_acc[e] = 0.f;
-        for (int k = 0; k < nk; ++k) {
-            const float p = sc[g * A.per_max + k];
-#pragma unroll
-            for (int e = 0; e < DL; ++e)
-                o_acc[e] = fmaf(p, to_f(Vs[(size_t)k * D + lane * DL + e]), o_acc[e]);
-        }
-        float *dst = part_b + ((int64_t)g * kAttSplits + s) * (D + 2);
-#pragma unroll
-        for (int e = 0; e < DL; ++e) dst[2 + lane * DL + e] = o_acc[e];
-        if (lane == 0) {
-            dst[0] = nk > 0 ? m : -INFINITY;
-            dst[1] = l;
-        }
-    }
-
-    // ---- the last split of this (sequence, KV head) combines
+    // the last CTA of (b, h) combines the fixed and routed partials
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
         const int done = atomicAdd(&A.att_done[b * A.Hkv + h], 1);
-        s_last = done == kAttSplits - 1;
+        s_last = done == kRouteSplits - 1;
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
     for (int g = warp; g < A.G; g += nw) {
-        const float *src = part_b + (int64_t)g * kAttSplits * (D + 2);
+        const float *src = part_b + (int64_t)g * kParts * (D + 2);
         float M = -INFINITY;
-        for (int sp = 0; sp < kAttSplits; ++sp) M = fmaxf(M, __ldcg(src + sp * (D + 2)));
-        float L = 0.f, o_acc[DL];
+        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, __ldcg(src + sp * (D + 2)));
+        float L = 0.f, acc[DL];
 #pragma unroll
-        for (int e = 0; e < DL; ++e) o_acc[e] = 0.f;
-        for (int sp = 0; sp < kAttSplits; ++sp) {
+        for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+        for (int sp = 0; sp < kParts; ++sp) {
             const float ms = __ldcg(src + sp * (D + 2));
             if (ms == -INFINITY) continue;
             const float w = exp2f(ms - M);
             L += w * __ldcg(src + sp * (D + 2) + 1);
 #pragma unroll
-            for (int e = 0; e < DL; ++e) o_acc[e] += w * __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
+            for (int e = 0; e < DL; ++e)
+                acc[e] += w * __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
         }
         const float inv = 1.f / L;
         T *o = static_cast<T *>(A.out) + ((int64_t)b * A.Hq + (int64_t)h * A.G + g) * D;
 #pragma unroll
-        for (int e = 0; e < DL; ++e) o[lane * DL + e] = from_f<T>(o_acc[e] * inv);
+        for (int e = 0; e < DL; ++e) o[lane * DL + e] = from_f<T>(acc[e] * inv);
         if (A.lse && lane == 0)
             A.lse[(int64_t)b * A.Hq + (int64_t)h * A.G + g] = (M + __log2f(L)) * 0.6931471805599453f;
     }
@@ -356,8 +485,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_attend(const DecodeArgs A) 
         A.att_done[b * A.Hkv + h] = 0;
         __threadfence();
         const int done = atomicAdd(&A.seq_done[b], 1);
-        s_seq_last = done == A.Hkv - 1;
-        if (s_seq_last) {
+        if (done == A.Hkv - 1) {
             A.seq_done[b] = 0;
             A.lens[b] = t + 1;
         }
@@ -383,7 +511,7 @@ Ws layout(const Geo &g) {
     w.sel_g = o;
     o += up256(sizeof(int32_t) * (size_t)g.B * g.Hkv * g.K_g);
     w.part = o;
-    o += up256(sizeof(float) * (size_t)g.B * g.Hq * kAttSplits * (g.D + 2));
+    o += up256(sizeof(float) * (size_t)g.B * g.Hq * kParts * (g.D + 2));
     w.total = o;
     return w;
 }
@@ -407,9 +535,6 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.K_g = g.K_g;
     A.nc_cap = g.T / g.C;
     A.ns_scan = (A.nc_cap + kScanChunks - 1) / kScanChunks;
-    A.keys_max = (int)min((long long)(g.F + max(g.L, 1) + 1) * g.C + (long long)g.K_g * g.g_s,
-                          (long long)g.T);
-    A.per_max = (((A.keys_max + kAttSplits - 1) / kAttSplits) + 3) & ~3;
     A.q_new = io.q_new;
     A.k_new = io.k_new;
     A.v_new = io.v_new;
@@ -434,30 +559,40 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     A.rope = r;
 
-    const size_t smem_scan = sizeof(unsigned long long) *
-        (size_t)max(max(kScanChunks, A.ns_scan * g.K_c), g.K_c * g.gpc);
-    const size_t smem_att = sizeof(int) * (size_t)((A.keys_max + 3) & ~3) +
-        sizeof(float) * (size_t)(g.G * D + g.G * A.per_max) + 2 * sizeof(T) * (size_t)A.per_max * D;
-    if (smem_scan > 200 * 1024 || smem_att > 200 * 1024) return HGA_ERR_UNSUPPORTED;
-    auto ks = k_decode_scan<T, D>;
-    auto ka = k_decode_attend<T, D>;
-    cudaError_t e = ensure_smem((const void *)ks, smem_scan);
-    if (e == cudaSuccess)
-        e = ensure_smem((const void *)ka, smem_att);
+    k_decode_a<T, D><<<dim3(A.ns_scan + kFixSplits, g.Hkv, g.B), kThreads, 0, st>>>(A);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
-    ks<<<dim3(A.ns_scan, g.Hkv, g.B), kThreads, smem_scan, st>>>(A);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_status(e);
-    ka<<<dim3(kAttSplits, g.Hkv, g.B), kThreads, smem_att, st>>>(A);
-    return cuda_status(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kRouteSplits, g.Hkv, g.B);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_decode_b<T, D>, A);
+    return cuda_status(e);
 }
 
 }  // namespace
+
+// Shapes the fixed-size tables hold: per CTA at most kThreads keys, the
+// merge and group candidates fit kMaxCand.
+bool decode_supported(const Geo &g) {
+    const long long ns = ((g.T / g.C) + kScanChunks - 1) / kScanChunks;
+    const long long routed = min((long long)g.K_g * g.g_s, (long long)g.T);
+    return g.G <= kMaxG && ns * g.K_c <= kMaxCand && (long long)g.K_c * g.gpc <= kMaxCand &&
+           routed <= (long long)kRouteSplits * kThreads &&
+           (long long)(g.F + max(g.L, 1) + 1) * g.C <= (long long)kFixSplits * kThreads;
+}
 
 size_t decode_workspace_bytes(const Geo &g) { return layout(g).total; }
 
 hga_status launch_decode(const Geo &g, const Rope &r, int dtype, const hga_io &io, void *ws,
                          cudaStream_t st) {
+    if (!decode_supported(g)) return HGA_ERR_UNSUPPORTED;
     if (dtype == HGA_BF16)
         return g.D == 128 ? run<__nv_bfloat16, 128>(g, r, io, ws, st)
                           : run<__nv_bfloat16, 64>(g, r, io, ws, st);

@@ -8,12 +8,14 @@
 // and KV head is the block's RoPE-rotated queries summed over its tokens and
 // over the KV head's query heads.
 //
-// Design: one CTA per (block, KV head, sequence).  The routing query is
-// formed from one 16-byte-vectorised pass over the block's Q rows (heads are
-// summed before the rotation, which is linear), accumulated in fp64.  Scores
-// are fp64 dot products of fp32 summary rows (one warp per row, coalesced),
-// ranked as packed (fp32 score, id) keys; the top-K is taken by K rounds of a
-// CTA-wide max, which is cheap for the K <= 64 the method uses.
+// Design: one CTA per (block, KV head, sequence), HBM-bound on the Q stream.
+// Each thread sums its token's G query heads on a quarter of the pairs with
+// 16-byte loads (RoPE is linear, so heads are summed before rotating), the
+// rotated rows meet in shared memory and 128 threads reduce them over the
+// block's tokens in fp64.  Scores are fp64 dot products, one summary row per
+// thread (its 16-byte loads all in flight), ranked as packed (fp32 score, id)
+// keys; the top-K runs in registers (warp bitonic sort and merge) for K <= 32
+// and by CTA-wide rounds above that.
 #include "hga_internal.cuh"
 #include "route_common.cuh"
 
@@ -26,13 +28,14 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int Hq, int Hkv,
         const float *__restrict__ s_chunk, const float *__restrict__ s_group, int nc_cap,
-        int F, int L, int K_c, int K_g, int gpc, int32_t *__restrict__ sel_chunk,
+        int F, int L, int K_c, int K_g, int gpc, int ncand, int32_t *__restrict__ sel_chunk,
         int32_t *__restrict__ sel_group, Rope rope) {
     constexpr int H = D / 2, PS = H / 4;
     extern __shared__ __align__(16) unsigned char smem[];
-    unsigned long long *cand = reinterpret_cast<unsigned long long *>(smem);
-    __shared__ double qr[D];
-    __shared__ double part[kThreads / 32][D];
+    float *rot = reinterpret_cast<float *>(smem);                              // [64][D]
+    unsigned long long *cand = reinterpret_cast<unsigned long long *>(rot + kChunk * D);
+    __shared__ __align__(16) double qr[D];
+    __shared__ unsigned long long lists[kThreads];
     __shared__ RouteScratch rs;
 
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -44,13 +47,10 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
     // ---- routing query: sum_i sum_{h'} R_{p_i}(q_{i,h'})
     {
         const int j = threadIdx.x >> 2, sl = threadIdx.x & 3;
-        double acc[2 * PS];
+        float lo[PS], hi[PS];
 #pragma unroll
-        for (int e = 0; e < 2 * PS; ++e) acc[e] = 0.0;
+        for (int p = 0; p < PS; ++p) lo[p] = hi[p] = 0.f;
         if (j < n) {
-            float lo[PS], hi[PS];
-#pragma unroll
-            for (int p = 0; p < PS; ++p) lo[p] = hi[p] = 0.f;
             const T *row = q + (((int64_t)b * Tlen + t0 + j) * Hq + (int64_t)h * G) * D;
             for (int hh = 0; hh < G; ++hh) {
                 float a[PS], d2[PS];
@@ -66,32 +66,20 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
 #pragma unroll
             for (int p = 0; p < PS; ++p) {
                 const float2 r = rope_cs(rope, pj, sl * PS + p);
-                acc[p] = (double)(lo[p] * r.x - hi[p] * r.y);
-                acc[PS + p] = (double)(hi[p] * r.x + lo[p] * r.y);
+                const float x = lo[p], y = hi[p];
+                lo[p] = x * r.x - y * r.y;
+                hi[p] = y * r.x + x * r.y;
             }
         }
-        // reduce over the 8 tokens of this warp (lanes with the same slice)
 #pragma unroll
-        for (int e = 0; e < 2 * PS; ++e) {
-            double v = acc[e];
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            acc[e] = v;
-        }
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-        if (lane < 4) {
-#pragma unroll
-            for (int p = 0; p < PS; ++p) {
-                part[warp][lane * PS + p] = acc[p];
-                part[warp][H + lane * PS + p] = acc[PS + p];
-            }
+        for (int p = 0; p < PS; ++p) {
+            rot[j * D + sl * PS + p] = lo[p];
+            rot[j * D + H + sl * PS + p] = hi[p];
         }
         __syncthreads();
         if (threadIdx.x < D) {
             double s = 0.0;
-#pragma unroll
-            for (int w = 0; w < kThreads / 32; ++w) s += part[w][threadIdx.x];
+            for (int jj = 0; jj < n; ++jj) s += (double)rot[jj * D + threadIdx.x];
             qr[threadIdx.x] = s;
         }
         __syncthreads();
@@ -101,9 +89,12 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
     const int hi_m = middle_hi(c, L);
     const int n_mid = max(0, hi_m - F + 1);
     const float *Sc = s_chunk + ((int64_t)b * Hkv + h) * nc_cap * D;
-    score_rows<D>(qr, Sc, F, n_mid, cand);
+    for (int r = threadIdx.x; r < n_mid; r += kThreads)
+        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sc + (int64_t)(F + r) * D), F + r);
     __syncthreads();
-    const int kc = topk_select(cand, n_mid, K_c, rs.sel_c, rs);
+    const int kc = min(K_c, n_mid);
+    if (K_c <= 32) block_topk32(cand, n_mid, K_c, rs.sel_c, lists);
+    else topk_select(cand, n_mid, K_c, rs.sel_c, rs);
     int32_t *out_c = sel_chunk + (((int64_t)b * NB + c) * Hkv + h) * K_c;
     for (int r = threadIdx.x; r < K_c; r += kThreads) out_c[r] = r < kc ? rs.sel_c[r] : -1;
 
@@ -111,9 +102,14 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
     const float *Sg = s_group + ((int64_t)b * Hkv + h) * nc_cap * gpc * D;
     const int n_g = kc * gpc;
     __syncthreads();
-    score_group_rows<D>(qr, Sg, rs.sel_c, gpc, n_g, cand);
+    for (int r = threadIdx.x; r < n_g; r += kThreads) {
+        const int gid = rs.sel_c[r / gpc] * gpc + r % gpc;
+        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sg + (int64_t)gid * D), gid);
+    }
     __syncthreads();
-    const int kg = topk_select(cand, n_g, K_g, rs.sel_g, rs);
+    const int kg = min(K_g, n_g);
+    if (K_g <= 32) block_topk32(cand, n_g, K_g, rs.sel_g, lists);
+    else topk_select(cand, n_g, K_g, rs.sel_g, rs);
     int32_t *out_g = sel_group + (((int64_t)b * NB + c) * Hkv + h) * K_g;
     for (int r = threadIdx.x; r < K_g; r += kThreads) out_g[r] = r < kg ? rs.sel_g[r] : -1;
 }
@@ -123,17 +119,15 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                const float *s_chunk, const float *s_group, int nc_cap, int32_t *sel_chunk,
                int32_t *sel_group, cudaStream_t st) {
     const long long ncand = max(max((long long)g.NC, 1ll), (long long)min(g.K_c, g.NC) * g.gpc);
-    const size_t smem = sizeof(unsigned long long) * (size_t)ncand;
-    if (smem > 160 * 1024) return HGA_ERR_UNSUPPORTED;   // candidate table must fit on chip
+    const size_t smem = sizeof(float) * kChunk * D + sizeof(unsigned long long) * (size_t)ncand;
+    if (smem > 180 * 1024) return HGA_ERR_UNSUPPORTED;   // candidate table must fit on chip
     auto kern = k_route<T, D>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = ensure_smem((const void *)kern, smem);
-        if (e != cudaSuccess) return cuda_status(e);
-    }
+    cudaError_t e = ensure_smem((const void *)kern, smem);
+    if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(g.NB, g.Hkv, g.B);
     kern<<<grid, kThreads, smem, st>>>(static_cast<const T *>(q), pos, g.T, g.Hq, g.Hkv, s_chunk,
-                                       s_group, nc_cap, g.F, g.L, g.K_c, g.K_g, g.gpc, sel_chunk,
-                                       sel_group, r);
+                                       s_group, nc_cap, g.F, g.L, g.K_c, g.K_g, g.gpc,
+                                       (int)ncand, sel_chunk, sel_group, r);
     return cuda_status(cudaGetLastError());
 }
 

@@ -137,3 +137,134 @@ __device__ __forceinline__ int topk_keys(unsigned long long *cand, int n, int K,
 }
 
 }  // namespace hga
+
+namespace hga {
+
+// ---- register top-K for K <= 32: warp bitonic sort and merge of packed keys
+
+// Sort the warp's 32 keys, one per lane, descending (lane 0 = largest).
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long p = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool take_max = ((lane & j) == 0) == ((lane & k) == 0);
+            v = take_max ? (p > v ? p : v) : (p < v ? p : v);
+        }
+    }
+    return v;
+}
+
+// Top 32 of two descending lists a and b (one key per lane), descending.
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long a,
+                                                              unsigned long long b) {
+    const int lane = threadIdx.x & 31;
+    const unsigned long long br = __shfl_sync(0xffffffffu, b, 31 - lane);
+    unsigned long long v = a > br ? a : br;   // bitonic: the top 32 of the union
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const unsigned long long p = __shfl_xor_sync(0xffffffffu, v, j);
+        v = ((lane & j) == 0) ? (p > v ? p : v) : (p < v ? p : v);
+    }
+    return v;
+}
+
+// Ascending sort of 32 ints across a warp (padding = INT_MAX).
+__device__ __forceinline__ int warp_sort_asc_int(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int p = __shfl_xor_sync(0xffffffffu, v, j);
+            const bool take_min = ((lane & j) == 0) == ((lane & k) == 0);
+            v = take_min ? min(v, p) : max(v, p);
+        }
+    }
+    return v;
+}
+
+// The warp's top 32 of n keys in smem/global (strided by the warp count),
+// descending.  warp_index/n_warps split the candidates between warps.
+__device__ __forceinline__ unsigned long long warp_top32(const unsigned long long *cand, int n,
+                                                         int warp_index, int n_warps) {
+    const int lane = threadIdx.x & 31;
+    unsigned long long acc = 0;
+    for (int base = warp_index * 32; base < n; base += n_warps * 32) {
+        const unsigned long long x = base + lane < n ? cand[base + lane] : 0ull;
+        acc = warp_merge_desc(acc, warp_sort_desc(x));
+    }
+    return acc;
+}
+
+// Top-K (K <= 32) of n candidate keys with the whole CTA: every warp reduces
+// its share to a sorted top 32, warp 0 merges them.  Writes the chosen ids
+// ascending to out (K entries, the unused ones -1); returns min(K, n).
+// lists: shared scratch of 32 * (blockDim.x / 32) keys.
+__device__ __forceinline__ int block_topk32(const unsigned long long *cand, int n, int K, int *out,
+                                            unsigned long long *lists) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const unsigned long long mine = warp_top32(cand, n, warp, nw);
+    lists[warp * 32 + lane] = mine;
+    __syncthreads();
+    if (warp == 0) {
+        unsigned long long acc = lists[lane];
+        for (int w = 1; w < nw; ++w) acc = warp_merge_desc(acc, lists[w * 32 + lane]);
+        const bool take = lane < K && acc != 0ull;
+        const int id = warp_sort_asc_int(take ? key_id(acc) : 0x7fffffff);
+        if (lane < K) out[lane] = id == 0x7fffffff ? -1 : id;
+    }
+    __syncthreads();
+    return min(K, n);
+}
+
+}  // namespace hga
+
+namespace hga {
+
+// fp64 dot product of q (shared, fp64) with one fp32 row, by one thread
+// (the whole row streams through this thread's 16-byte loads).
+template <int D>
+__device__ __forceinline__ double thread_dot_row(const double *qr, const float *__restrict__ row) {
+    // 16 loads in flight per batch: enough to cover latency, few registers
+    constexpr int kBatch = 16;
+    const float4 *r4 = reinterpret_cast<const float4 *>(row);
+    const double2 *q2 = reinterpret_cast<const double2 *>(qr);
+    double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+    for (int base = 0; base < D / 4; base += kBatch) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) v[e] = __ldg(r4 + base + e);
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) {
+            const double2 a = q2[2 * (base + e)], b = q2[2 * (base + e) + 1];
+            s0 = fma(a.x, (double)v[e].x, s0);
+            s1 = fma(a.y, (double)v[e].y, s1);
+            s0 = fma(b.x, (double)v[e].z, s0);
+            s1 = fma(b.y, (double)v[e].w, s1);
+        }
+    }
+    return s0 + s1;
+}
+
+// Top-K (K <= 32) keys of n candidates with the whole CTA, written to out
+// (global or shared) descending, padded with 0.
+__device__ __forceinline__ void block_topk32_keys(const unsigned long long *cand, int n, int K,
+                                                  unsigned long long *out,
+                                                  unsigned long long *lists) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const unsigned long long mine = warp_top32(cand, n, warp, nw);
+    lists[warp * 32 + lane] = mine;
+    __syncthreads();
+    if (warp == 0) {
+        unsigned long long acc = lists[lane];
+        for (int w = 1; w < nw; ++w) acc = warp_merge_desc(acc, lists[w * 32 + lane]);
+        if (lane < K) out[lane] = acc;
+    }
+    __syncthreads();
+}
+
+}  // namespace hga
