@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-replays", type=int, default=10)
+    ap.add_argument("--decode-only", action="store_true",
+                    help="profiling variant: only the decode part")
     ap.add_argument("--seq", type=int, default=0,
                     help="override the prefill length (small profiling cases only)")
     return ap.parse_args()
@@ -375,6 +377,13 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     hga.load()
+    if args.decode_only:
+        dec = bench_decode(args, dev, world)
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"note": "profiling variant, not a bench line", "decode": dec}))
+        return
     w = WORKLOADS[WORKLOAD]
     if args.seq:
         w = w.replace(T=args.seq, name=f"{w.name}_T{args.seq}")

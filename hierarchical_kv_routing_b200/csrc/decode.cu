@@ -169,19 +169,39 @@ __device__ __forceinline__ float dot16(const uint4 &w, const float *q) {
     }
 }
 
-// Partial attention of the G heads over keys key_of(0..nk), nk <= blockDim:
-// scores one key per thread, softmax and P.V one warp per head with lanes
-// over dims; writes (m, l, o[D]) for part index `pi`.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
+// Partial attention of the G heads over keys key_of(0..nk), nk <= blockDim.
+// The value rows are staged in shared memory (Vs, [nk][D]) with cp.async
+// while the scores are computed, one key per thread with the key row's
+// 16-byte loads all in flight; softmax and P.V then run one warp per head
+// with lanes over dims.  Writes (m, l, o[D]) for part index `pi`.
 template <typename T, int D, typename KeyOf>
 __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, KeyOf key_of,
-                            int pi, const float *qs, const T *knew, float *sc, int *kt_s) {
+                            int pi, const float *qs, const T *knew, float *sc, int *kt_s, T *Vs) {
     constexpr int DL = D / 32;
     constexpr int NV = D * (int)sizeof(T) / 16;     // 16-byte slices per row
     constexpr int EV = 16 / (int)sizeof(T);         // elements per slice
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    for (int k = threadIdx.x; k < nk; k += blockDim.x) kt_s[k] = key_of(k);
+    __syncthreads();
+    const T *vbase = static_cast<const T *>(A.v);
+    const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
+    for (int idx = threadIdx.x; idx < nk * NV; idx += blockDim.x) {
+        const int k = idx / NV, part = idx % NV;
+        const int kt = kt_s[k];
+        const T *src = kt == t ? vn : vbase + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D;
+        cp_async16(reinterpret_cast<uint4 *>(Vs + (size_t)k * D) + part,
+                   reinterpret_cast<const uint4 *>(src) + part);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     for (int k = threadIdx.x; k < nk; k += blockDim.x) {
-        const int kt = key_of(k);
-        kt_s[k] = kt;
+        const int kt = kt_s[k];
         const uint4 *src = kt == t
             ? reinterpret_cast<const uint4 *>(knew)
             : reinterpret_cast<const uint4 *>(static_cast<const T *>(A.k_rot) +
@@ -201,9 +221,8 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
             sc[g * kThreads + k] = a0 + a1;
         }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    const T *vbase = static_cast<const T *>(A.v);
-    const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
     float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
     for (int g = warp; g < A.G; g += nw) {
         float m = -INFINITY;
@@ -222,15 +241,12 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
         float acc[DL];
 #pragma unroll
         for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+#pragma unroll 4
         for (int k = 0; k < nk; ++k) {
             const float p = sc[g * kThreads + k];
-            const int kt = kt_s[k];
-            const T *vr = kt == t ? vn : vbase + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D;
-            float vv[DL];
+            const T *vr = Vs + (size_t)k * D + lane * DL;
 #pragma unroll
-            for (int e = 0; e < DL; ++e) vv[e] = to_f(vr[lane * DL + e]);
-#pragma unroll
-            for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
+            for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e]);
         }
         float *dst = part_b + ((int64_t)g * kParts + pi) * (D + 2);
 #pragma unroll
@@ -266,6 +282,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
                                  ? sizeof(ScanSmem<T, D>) : sizeof(AttSmem<T, D>);
     __shared__ __align__(16) unsigned char pool[kPool];
     __shared__ int s_last;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
     ScanSmem<T, D> &ss = *reinterpret_cast<ScanSmem<T, D> *>(pool);
     AttSmem<T, D> &as = *reinterpret_cast<AttSmem<T, D> *>(pool);
     double *qr = ss.qr;
@@ -305,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
             const int i = k0 + k;
             return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
         };
-        attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s);
+        attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
         return;
     }
 
@@ -337,10 +355,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
         const float2 r = rope_cs(A.rope, (double)pnew, i);
         const T *qb = static_cast<const T *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
         double a = 0.0, d2 = 0.0;
-        for (int g = 0; g < A.G; ++g) {
-            const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
-            a += (double)(x * r.x - y * r.y);
-            d2 += (double)(y * r.x + x * r.y);
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g) {
+            if (g < A.G) {
+                const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
+                a += (double)(x * r.x - y * r.y);
+                d2 += (double)(y * r.x + x * r.y);
+            }
         }
         qr[i] = a;
         qr[i + H] = d2;
@@ -423,6 +444,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     __shared__ int kt_s[kThreads];
     __shared__ int sel[kMaxK];
     __shared__ int s_last;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
 
     const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -444,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
         const int i = k0 + k;
         return sel[i / A.g_s] * A.g_s + i % A.g_s;
     };
-    attend_part<T, D>(A, b, h, t, nk, key_of, kFixSplits + r, qs, knew, sc, kt_s);
+    attend_part<T, D>(A, b, h, t, nk, key_of, kFixSplits + r, qs, knew, sc, kt_s, Vs);
 
     // the last CTA of (b, h) combines the fixed and routed partials
     __threadfence();
@@ -559,13 +582,17 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     A.rope = r;
 
-    k_decode_a<T, D><<<dim3(A.ns_scan + kFixSplits, g.Hkv, g.B), kThreads, 0, st>>>(A);
-    cudaError_t e = cudaGetLastError();
+    const size_t vs_bytes = sizeof(T) * (size_t)kThreads * D;
+    cudaError_t e = ensure_smem((const void *)k_decode_a<T, D>, vs_bytes);
+    if (e == cudaSuccess) e = ensure_smem((const void *)k_decode_b<T, D>, vs_bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    k_decode_a<T, D><<<dim3(A.ns_scan + kFixSplits, g.Hkv, g.B), kThreads, vs_bytes, st>>>(A);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kRouteSplits, g.Hkv, g.B);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = vs_bytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -52,14 +52,35 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
         for (int p = 0; p < PS; ++p) lo[p] = hi[p] = 0.f;
         if (j < n) {
             const T *row = q + (((int64_t)b * Tlen + t0 + j) * Hq + (int64_t)h * G) * D;
-            for (int hh = 0; hh < G; ++hh) {
-                float a[PS], d2[PS];
-                load_slice<T, PS>(row + hh * D + sl * PS, a);
-                load_slice<T, PS>(row + hh * D + H + sl * PS, d2);
+            // several heads' rows in flight at a time, kept packed until summed
+            constexpr int kVec = PS * (int)sizeof(T) / 16;        // 16-byte words per half
+            constexpr int kBatch = sizeof(T) == 2 ? 4 : 2;
+            for (int h0 = 0; h0 < G; h0 += kBatch) {
+                uint4 wa[kBatch][kVec], wb[kBatch][kVec];
 #pragma unroll
-                for (int p = 0; p < PS; ++p) {
-                    lo[p] += a[p];
-                    hi[p] += d2[p];
+                for (int u = 0; u < kBatch; ++u) {
+                    if (h0 + u < G) {
+                        const uint4 *pa = reinterpret_cast<const uint4 *>(row + (h0 + u) * D + sl * PS);
+                        const uint4 *pb = reinterpret_cast<const uint4 *>(row + (h0 + u) * D + H + sl * PS);
+#pragma unroll
+                        for (int v = 0; v < kVec; ++v) {
+                            wa[u][v] = __ldg(pa + v);
+                            wb[u][v] = __ldg(pb + v);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    if (h0 + u < G) {
+                        float a[PS], d2[PS];
+                        unpack_words<T, PS>(wa[u], a);
+                        unpack_words<T, PS>(wb[u], d2);
+#pragma unroll
+                        for (int p = 0; p < PS; ++p) {
+                            lo[p] += a[p];
+                            hi[p] += d2[p];
+                        }
+                    }
                 }
             }
             const double pj = (double)pos[(int64_t)b * Tlen + t0 + j];

@@ -54,4 +54,29 @@ __device__ __forceinline__ void store_slice(T *__restrict__ p, const float (&x)[
     }
 }
 
+// Unpack N elements held as 16-byte words (8 bf16 or 4 fp32 per word).
+template <typename T, int N>
+__device__ __forceinline__ void unpack_words(const uint4 (&w)[N * sizeof(T) / 16], float (&x)[N]) {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int v = 0; v < N / 8; ++v) {
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&w[v]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                x[v * 8 + 2 * e] = f.x;
+                x[v * 8 + 2 * e + 1] = f.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int v = 0; v < N / 4; ++v) {
+            x[v * 4 + 0] = __uint_as_float(w[v].x);
+            x[v * 4 + 1] = __uint_as_float(w[v].y);
+            x[v * 4 + 2] = __uint_as_float(w[v].z);
+            x[v * 4 + 3] = __uint_as_float(w[v].w);
+        }
+    }
+}
+
 }  // namespace hga
