@@ -53,11 +53,12 @@ struct Cfg {
     static constexpr uint32_t oK = oQ + 2 * kTileBytes;
     static constexpr uint32_t oV = oK + kStages * kTileBytes;
     static constexpr uint32_t oEnd = oV + kStages * kTileBytes;
+    static constexpr uint32_t oCS = oEnd;                       // optional cos/sin table
 };
 
 struct Ctl {
     uint64_t q_full[2], q_ready[2], s_full[2], p_full[2], o_full[2];
-    uint64_t k_full[4], v_full[4], kv_empty[4];
+    uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
     uint64_t fin;
     uint32_t tmem_base;
     int nseg, first_cur;
@@ -68,6 +69,7 @@ struct Ctl {
 struct TcArgs {
     int T, Hq, Hkv, G, NB, F, L, K_g, g_s, k_T, v_T;
     int rows_per_unit, ctas_per_unit, tokM;
+    int cs_tokens;            // > 0: the CTA's (token, pair) cos/sin table is in smem
     const int32_t *sel_group;
     const int32_t *pos;
     __nv_bfloat16 *out;
@@ -89,7 +91,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-            const __grid_constant__ CUtensorMap tmV, const TcArgs A) {
+            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
+            const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmK64,
+            const __grid_constant__ CUtensorMap tmV64, const TcArgs A) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -117,11 +121,21 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         for (int i = 0; i < 4; ++i) {
             mbar_init(&ctl.k_full[i], 1);
             mbar_init(&ctl.v_full[i], 1);
-            mbar_init(&ctl.kv_empty[i], 1);
+            mbar_init(&ctl.k_empty[i], 1);
+            mbar_init(&ctl.v_empty[i], 1);
         }
         mbar_init(&ctl.fin, 1);
         ctl.abort = 0;
         fence_barrier_init();
+        // Q tiles first, so they load while the cos/sin table is computed
+        prefetch_tensormap(&tmQ);
+        for (int mt = 0; mt < NT; ++mt) {
+            const int tok_first = t0 + (row0 + mt * 128) / A.G;
+            mbar_arrive_expect_tx(&ctl.q_full[mt], (uint32_t)(A.G * A.tokM * D * 2));
+            for (int hf = 0; hf < C::kHalves; ++hf)
+                tma_load_3d(smem + C::oQ + mt * C::kTileBytes + hf * C::kHalfBytes, &tmQ,
+                            &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&ctl.tmem_base, 512);
@@ -157,6 +171,18 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
     }
     __syncthreads();
+    // cos/sin of every (token, pair) of this CTA's rows, shared by the G
+    // query heads of a token (each angle formed once instead of G times)
+    const int tok0 = t0 + row0 / A.G;
+    float2 *cs_tab = reinterpret_cast<float2 *>(smem + C::oCS);
+    if (A.cs_tokens > 0) {
+        constexpr int H = D / 2;
+        for (int e = threadIdx.x; e < A.cs_tokens * H; e += kThreads) {
+            const int tk = tok0 + e / H;
+            if (tk < A.T) cs_tab[e] = rope_cs(A.rope, (double)A.pos[(int64_t)b * A.T + tk], e % H);
+        }
+        __syncthreads();
+    }
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
     const int nseg = ctl.nseg;
@@ -166,19 +192,16 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     if (warp == 0) {
         // ------------------------------------------------------ producer --
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-            for (int mt = 0; mt < NT; ++mt) {
-                const int tok_first = t0 + (row0 + mt * 128) / A.G;
-                mbar_arrive_expect_tx(&ctl.q_full[mt], (uint32_t)(A.G * A.tokM * D * 2));
-                for (int hf = 0; hf < C::kHalves; ++hf)
-                    tma_load_3d(smem + C::oQ + mt * C::kTileBytes + hf * C::kHalfBytes, &tmQ,
-                                &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first);
-            }
+            prefetch_tensormap(&tmK16);
+            prefetch_tensormap(&tmV16);
+            prefetch_tensormap(&tmK64);
+            prefetch_tensormap(&tmV64);
             for (int j = 0; j < ntiles && !ctl.abort; ++j) {
                 const int s = j % C::kStages;
-                if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1)) {
+                const uint32_t ph = ((j / C::kStages) - 1) & 1;
+                if (j >= C::kStages && !mbar_wait(&ctl.k_empty[s], ph)) {
                     fail(ctl);
                     break;
                 }
@@ -186,22 +209,37 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const uint32_t bytes = (uint32_t)nsj * 8 * D * 2;
                 uint8_t *kt = smem + C::oK + s * C::kTileBytes;
                 uint8_t *vt = smem + C::oV + s * C::kTileBytes;
+                // runs of consecutive segments go as one 64- or 16-row box
+                auto issue = [&](uint8_t *tile, const CUtensorMap *m8, const CUtensorMap *m16,
+                                 const CUtensorMap *m64, uint64_t *bar, int kvT) {
+                    const int *sg = ctl.seg_tok + j * kSegPerTile;
+                    for (int e = 0; e < nsj;) {
+                        const int st = sg[e];
+                        int run = 1;
+                        if (st != kDummy) {
+                            if ((e & 7) == 0 && e + 8 <= nsj) {
+                                run = 8;
+                                for (int i = 1; i < 8; ++i)
+                                    if (sg[e + i] != st + 8 * i) { run = 1; break; }
+                            }
+                            if (run == 1 && (e & 1) == 0 && e + 2 <= nsj && sg[e + 1] == st + 8)
+                                run = 2;
+                        }
+                        const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
+                        const int z = b * kvT + (st == kDummy ? 0 : st);
+                        for (int hf = 0; hf < C::kHalves; ++hf)
+                            tma_load_3d(tile + hf * C::kHalfBytes + e * 1024, m, bar, hf * 64, h, z);
+                        e += run;
+                    }
+                };
                 mbar_arrive_expect_tx(&ctl.k_full[s], bytes);
-                for (int e = 0; e < nsj; ++e) {
-                    const int st = ctl.seg_tok[j * kSegPerTile + e];
-                    const int z = b * A.k_T + (st == kDummy ? 0 : st);
-                    for (int hf = 0; hf < C::kHalves; ++hf)
-                        tma_load_3d(kt + hf * C::kHalfBytes + e * 1024, &tmK, &ctl.k_full[s],
-                                    hf * 64, h, z);
+                issue(kt, &tmK, &tmK16, &tmK64, &ctl.k_full[s], A.k_T);
+                if (j >= C::kStages && !mbar_wait(&ctl.v_empty[s], ph)) {
+                    fail(ctl);
+                    break;
                 }
                 mbar_arrive_expect_tx(&ctl.v_full[s], bytes);
-                for (int e = 0; e < nsj; ++e) {
-                    const int st = ctl.seg_tok[j * kSegPerTile + e];
-                    const int z = b * A.v_T + (st == kDummy ? 0 : st);
-                    for (int hf = 0; hf < C::kHalves; ++hf)
-                        tma_load_3d(vt + hf * C::kHalfBytes + e * 1024, &tmV, &ctl.v_full[s],
-                                    hf * 64, h, z);
-                }
+                issue(vt, &tmV, &tmV16, &tmV64, &ctl.v_full[s], A.v_T);
             }
         }
     } else if (warp == 1) {
@@ -233,12 +271,11 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                            smem_desc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
                 }
             };
+            // per tile j: P.V of tile j-1 first (it needs no new data), then
+            // S of tile j once its K tile has landed; K stages are released
+            // after both S products, V stages after both P.V products
             for (int j = 0; j <= ntiles && ok; ++j) {
                 const int s = j % C::kStages;
-                if (j < ntiles) {
-                    if (!(ok = mbar_wait(&ctl.k_full[s], (j / C::kStages) & 1))) break;
-                    tc_fence_after();
-                }
                 for (int mt = 0; mt < NT && ok; ++mt) {
                     if (j > 0) {
                         if (!(ok = mbar_wait(&ctl.p_full[mt], (j - 1) & 1))) break;
@@ -250,11 +287,16 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         }
                         issue_pv(mt, j - 1);
                         if (j == ntiles) mma_commit(&ctl.o_full[mt]);
-                        else if (mt == NT - 1) mma_commit(&ctl.kv_empty[sp]);
+                        else if (mt == NT - 1) mma_commit(&ctl.v_empty[sp]);
                     }
                     if (j < ntiles) {
+                        if (mt == 0) {
+                            if (!(ok = mbar_wait(&ctl.k_full[s], (j / C::kStages) & 1))) break;
+                            tc_fence_after();
+                        }
                         issue_s(mt, j);
                         mma_commit(&ctl.s_full[mt]);
+                        if (mt == NT - 1) mma_commit(&ctl.k_empty[s]);
                     }
                 }
             }
@@ -295,8 +337,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = __bfloat1622float2(pa[e]);
                         const float2 y = __bfloat1622float2(pb[e]);
-                        const float2 c0 = rope_cs(A.rope, p, g * 8 + 2 * e);
-                        const float2 c1 = rope_cs(A.rope, p, g * 8 + 2 * e + 1);
+                        const float2 c0 = A.cs_tokens > 0 ? cs_tab[(tok - tok0) * (D / 2) + g * 8 + 2 * e]
+                                                          : rope_cs(A.rope, p, g * 8 + 2 * e);
+                        const float2 c1 = A.cs_tokens > 0 ? cs_tab[(tok - tok0) * (D / 2) + g * 8 + 2 * e + 1]
+                                                          : rope_cs(A.rope, p, g * 8 + 2 * e + 1);
                         pa[e] = __floats2bfloat162_rn(x.x * c0.x - y.x * c0.y, x.y * c1.x - y.y * c1.y);
                         pb[e] = __floats2bfloat162_rn(y.x * c0.x + x.x * c0.y, y.y * c1.x + x.y * c1.y);
                     }
@@ -324,65 +368,57 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     const int st = segs[col >> 3];
                     return st == kDummy || st + (col & 7) > tok;
                 };
-                // pass 1: row max
-                float mx = -INFINITY;
-                for (int cb = 0; cb < (nj + 31) / 32; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_base + cb * 32, v);
-                    tmem_ld_wait();
+                // one TMEM pass: the S row (up to 128 columns) into registers
+                uint32_t v[128];
+                tmem_ld32(lane_base + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tmem_ld32(lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+                tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+                tmem_ld_wait();
+                if (need_mask) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x = __uint_as_float(v[e]);
-                        if (!need_mask || !masked(cb * 32 + e)) mx = fmaxf(mx, x);
-                    }
+                    for (int e = 0; e < 128; ++e)
+                        if (masked(e)) v[e] = __float_as_uint(-INFINITY);
                 }
+                float mx = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
                 if (!valid) mx = -INFINITY;
                 const float mt_new = mx * sc;
-                // The rescale decision is per row, but tcgen05.ld/st are
-                // warp-collective: the warp rescales together, rows that
-                // keep their reference use factor 1.
+                // The reference grows only when the row max rises by more than
+                // 2^8; P uses the new reference, and O (accumulated under the
+                // old one) is rescaled below, before this tile's P.V.
                 const bool grow = mt_new > m_ref + 8.0f;
                 const bool rescale = grow && m_ref != -INFINITY;
+                const float f = rescale ? ex2(m_ref - mt_new) : 1.0f;
+                if (grow) m_ref = mt_new;
+                l *= f;
+                // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
+                const bool live = m_ref != -INFINITY;
+                const float neg = -m_ref;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (live) {
+                        p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, neg));
+                        p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, neg));
+                    }
+                    l += p0 + p1;
+                    v[e] = pack_bf16(p0, p1);
+                }
+                tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+                tmem_st32(lane_base + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+                // tcgen05.ld/st are warp-collective: the warp rescales O
+                // together when any of its rows needs it (factor 1 elsewhere)
                 if (__any_sync(0xffffffffu, rescale)) {
-                    const float f = rescale ? ex2(m_ref - mt_new) : 1.0f;
-                    l *= f;
                     for (int cb = 0; cb < D / 32; ++cb) {
-                        uint32_t v[32];
-                        tmem_ld32(lane_base + 128 + cb * 32, v);
+                        uint32_t o[32];
+                        tmem_ld32(lane_base + 128 + cb * 32, o);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-                        tmem_st32(lane_base + 128 + cb * 32, v);
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        tmem_st32(lane_base + 128 + cb * 32, o);
                     }
-                }
-                if (grow) m_ref = mt_new;
-                // pass 2: P = 2^(s*scale - m_ref) as bf16 over the S columns
-                const bool live = m_ref != -INFINITY;
-                for (int cb = 0; cb < (nj + 31) / 32; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_base + cb * 32, v);
-                    tmem_ld_wait();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float p0 = 0.f, p1 = 0.f;
-                        if (live) {
-                            const int c0 = cb * 32 + 2 * e;
-                            if (!need_mask || !masked(c0))
-                                p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, -m_ref));
-                            if (!need_mask || !masked(c0 + 1))
-                                p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, -m_ref));
-                        }
-                        l += p0 + p1;
-                        pk[e] = pack_bf16(p0, p1);
-                    }
-                    asm volatile(
-                        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, "
-                        "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(lane_base + cb * 16),
-                        "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]),
-                        "r"(pk[6]), "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]),
-                        "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-                        : "memory");
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -478,23 +514,33 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     a.rows_per_unit = kChunk * g.G;
     a.ctas_per_unit = (a.rows_per_unit + 255) / 256;
     a.tokM = min(128, kChunk * g.G) / g.G;
+    {
+        // the table costs tokens x D/2 x 8 bytes; keep the CTA inside 227 KB
+        const int tok_cta = (min(256, a.rows_per_unit) + g.G - 1) / g.G;
+        const size_t tab = (size_t)tok_cta * (D / 2) * sizeof(float2);
+        a.cs_tokens = Cfg<D>::oEnd + 1024 + tab + sizeof(Ctl) <= 232448 ? tok_cta : 0;
+    }
     a.sel_group = sel_group;
     a.pos = pos;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     a.rope = r;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mk16, mv16, mk64, mv64;
     if (!make_map(&mq, q, D, g.Hq, (long long)g.B * g.T, g.G, a.tokM) ||
         !make_map(&mk, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 8) ||
-        !make_map(&mv, v, D, g.Hkv, (long long)g.B * v_T, 1, 8))
+        !make_map(&mv, v, D, g.Hkv, (long long)g.B * v_T, 1, 8) ||
+        !make_map(&mk16, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 16) ||
+        !make_map(&mv16, v, D, g.Hkv, (long long)g.B * v_T, 1, 16) ||
+        !make_map(&mk64, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 64) ||
+        !make_map(&mv64, v, D, g.Hkv, (long long)g.B * v_T, 1, 64))
         return HGA_ERR_CUDA;
-    const size_t smem = Cfg<D>::oEnd + 1024;
+    const size_t smem = Cfg<D>::oEnd + 1024 + (size_t)a.cs_tokens * (D / 2) * sizeof(float2);
     auto kern = k_attend_tc<D>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(g.NB * a.ctas_per_unit, g.Hkv, g.B);
-    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mk16, mv16, mk64, mv64, a);
     return cuda_status(cudaGetLastError());
 }
 

@@ -169,6 +169,33 @@ __device__ __forceinline__ float dot16(const uint4 &w, const float *q) {
     }
 }
 
+// DL consecutive elements (shared memory) as one packed load.
+template <typename T, int DL>
+__device__ __forceinline__ void load_lane_slice(const T *p, float (&x)[DL]) {
+    if constexpr (sizeof(T) == 2 && DL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2 *>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+        const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+        x[0] = a.x;
+        x[1] = a.y;
+        x[2] = c.x;
+        x[3] = c.y;
+    } else if constexpr (sizeof(T) == 2 && DL == 2) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+        x[0] = a.x;
+        x[1] = a.y;
+    } else if constexpr (sizeof(T) == 4 && DL == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(p);
+        x[0] = a.x;
+        x[1] = a.y;
+        x[2] = a.z;
+        x[3] = a.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < DL; ++e) x[e] = to_f(p[e]);
+    }
+}
+
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                      static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -200,7 +227,11 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
                    reinterpret_cast<const uint4 *>(src) + part);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int k = threadIdx.x; k < nk; k += blockDim.x) {
+    // two threads per key (each half of the heads) when the slice is short
+    const int tpk = nk <= (int)blockDim.x / 2 ? 2 : 1;
+    const int gper = (A.G + tpk - 1) / tpk;
+    for (int idx = threadIdx.x; idx < nk * tpk; idx += blockDim.x) {
+        const int k = idx / tpk, part = idx % tpk;
         const int kt = kt_s[k];
         const uint4 *src = kt == t
             ? reinterpret_cast<const uint4 *>(knew)
@@ -209,8 +240,9 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
         uint4 kw[NV];
 #pragma unroll
         for (int e = 0; e < NV; ++e) kw[e] = kt == t ? src[e] : __ldg(src + e);
+        const int g1 = min(A.G, (part + 1) * gper);
 #pragma unroll 1
-        for (int g = 0; g < A.G; ++g) {
+        for (int g = part * gper; g < g1; ++g) {
             const float *qg = qs + g * D;
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
@@ -244,9 +276,10 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
 #pragma unroll 4
         for (int k = 0; k < nk; ++k) {
             const float p = sc[g * kThreads + k];
-            const T *vr = Vs + (size_t)k * D + lane * DL;
+            float vv[DL];
+            load_lane_slice<T, DL>(Vs + (size_t)k * D + lane * DL, vv);
 #pragma unroll
-            for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e]);
+            for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
         }
         float *dst = part_b + ((int64_t)g * kParts + pi) * (D + 2);
 #pragma unroll
@@ -296,8 +329,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     float *sc = as.sc;
     int *kt_s = as.kt_s;
 
-    // let the routed-keys kernel launch now; it waits for this grid itself
-    asm volatile("griddepcontrol.launch_dependents;");
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
     if (t < 0 || t >= A.Tc) {
@@ -324,6 +355,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
             return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
         };
         attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
+        // this CTA is done: the routed-keys kernel may start launching
+        asm volatile("griddepcontrol.launch_dependents;");
         return;
     }
 
@@ -391,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
         s_last = done == A.ns_scan - 1;
     }
     __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;");
     if (!s_last) return;
     __threadfence();
     const unsigned long long *all = A.cand + ((int64_t)b * A.Hkv + h) * A.ns_scan * A.K_c;
