@@ -189,57 +189,51 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
     const int first_cur = ctl.first_cur;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer --
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------ producers --
+        // warp 0 streams the K tiles, warp 2 the V tiles, each through its own
+        // stage ring: a K tile is needed one P.V earlier than its V tile, so
+        // the K stream must not wait behind V stage releases
         if (lane == 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            prefetch_tensormap(&tmK16);
-            prefetch_tensormap(&tmV16);
-            prefetch_tensormap(&tmK64);
-            prefetch_tensormap(&tmV64);
+            const bool is_k = warp == 0;
+            const CUtensorMap *m8 = is_k ? &tmK : &tmV;
+            const CUtensorMap *m16 = is_k ? &tmK16 : &tmV16;
+            const CUtensorMap *m64 = is_k ? &tmK64 : &tmV64;
+            prefetch_tensormap(m8);
+            prefetch_tensormap(m16);
+            prefetch_tensormap(m64);
+            const int kvT = is_k ? A.k_T : A.v_T;
             for (int j = 0; j < ntiles && !ctl.abort; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t ph = ((j / C::kStages) - 1) & 1;
-                if (j >= C::kStages && !mbar_wait(&ctl.k_empty[s], ph)) {
+                uint64_t *empty = is_k ? &ctl.k_empty[s] : &ctl.v_empty[s];
+                uint64_t *full = is_k ? &ctl.k_full[s] : &ctl.v_full[s];
+                if (j >= C::kStages && !mbar_wait(empty, ph)) {
                     fail(ctl);
                     break;
                 }
                 const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
-                const uint32_t bytes = (uint32_t)nsj * 8 * D * 2;
-                uint8_t *kt = smem + C::oK + s * C::kTileBytes;
-                uint8_t *vt = smem + C::oV + s * C::kTileBytes;
+                uint8_t *tile = smem + (is_k ? C::oK : C::oV) + s * C::kTileBytes;
+                mbar_arrive_expect_tx(full, (uint32_t)nsj * 8 * D * 2);
                 // runs of consecutive segments go as one 64- or 16-row box
-                auto issue = [&](uint8_t *tile, const CUtensorMap *m8, const CUtensorMap *m16,
-                                 const CUtensorMap *m64, uint64_t *bar, int kvT) {
-                    const int *sg = ctl.seg_tok + j * kSegPerTile;
-                    for (int e = 0; e < nsj;) {
-                        const int st = sg[e];
-                        int run = 1;
-                        if (st != kDummy) {
-                            if ((e & 7) == 0 && e + 8 <= nsj) {
-                                run = 8;
-                                for (int i = 1; i < 8; ++i)
-                                    if (sg[e + i] != st + 8 * i) { run = 1; break; }
-                            }
-                            if (run == 1 && (e & 1) == 0 && e + 2 <= nsj && sg[e + 1] == st + 8)
-                                run = 2;
+                const int *sg = ctl.seg_tok + j * kSegPerTile;
+                for (int e = 0; e < nsj;) {
+                    const int st = sg[e];
+                    int run = 1;
+                    if (st != kDummy) {
+                        if ((e & 7) == 0 && e + 8 <= nsj) {
+                            run = 8;
+                            for (int i = 1; i < 8; ++i)
+                                if (sg[e + i] != st + 8 * i) { run = 1; break; }
                         }
-                        const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
-                        const int z = b * kvT + (st == kDummy ? 0 : st);
-                        for (int hf = 0; hf < C::kHalves; ++hf)
-                            tma_load_3d(tile + hf * C::kHalfBytes + e * 1024, m, bar, hf * 64, h, z);
-                        e += run;
+                        if (run == 1 && (e & 1) == 0 && e + 2 <= nsj && sg[e + 1] == st + 8) run = 2;
                     }
-                };
-                mbar_arrive_expect_tx(&ctl.k_full[s], bytes);
-                issue(kt, &tmK, &tmK16, &tmK64, &ctl.k_full[s], A.k_T);
-                if (j >= C::kStages && !mbar_wait(&ctl.v_empty[s], ph)) {
-                    fail(ctl);
-                    break;
+                    const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
+                    const int z = b * kvT + (st == kDummy ? 0 : st);
+                    for (int hf = 0; hf < C::kHalves; ++hf)
+                        tma_load_3d(tile + hf * C::kHalfBytes + e * 1024, m, full, hf * 64, h, z);
+                    e += run;
                 }
-                mbar_arrive_expect_tx(&ctl.v_full[s], bytes);
-                issue(vt, &tmV, &tmV16, &tmV64, &ctl.v_full[s], A.v_T);
             }
         }
     } else if (warp == 1) {
@@ -380,9 +374,14 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     for (int e = 0; e < 128; ++e)
                         if (masked(e)) v[e] = __float_as_uint(-INFINITY);
                 }
-                float mx = -INFINITY;
+                // row max with 8 independent chains (no 128-long dependency)
+                float mx8[8];
 #pragma unroll
-                for (int e = 0; e < 128; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+                for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(v[u]);
+#pragma unroll
+                for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
+                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 if (!valid) mx = -INFINITY;
                 const float mt_new = mx * sc;
                 // The reference grows only when the row max rises by more than
@@ -396,6 +395,9 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
                 const bool live = m_ref != -INFINITY;
                 const float neg = -m_ref;
+                float l8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) l8[u] = 0.f;
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     float p0 = 0.f, p1 = 0.f;
@@ -403,9 +405,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                         p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, neg));
                         p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, neg));
                     }
-                    l += p0 + p1;
+                    l8[e & 7] += p0 + p1;
                     v[e] = pack_bf16(p0, p1);
                 }
+                l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
                 tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
                 tmem_st32(lane_base + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
                 // tcgen05.ld/st are warp-collective: the warp rescales O
