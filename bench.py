@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-hosttier", action="store_true")
     ap.add_argument("--decode-replays", type=int, default=10)
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling variant: only the decode part")
@@ -357,6 +358,78 @@ def bench_decode(args, dev, world):
                          "peak_source": f"{src} hbm_gbs (copy)"}}
 
 
+HOSTTIER_WORKLOAD = "qwen3_30b_a3b_bf16_hosttier_prefill_64k"
+
+
+def hosttier_link_bytes(w, sel_group):
+    """Algorithmic bytes over the host link for one host-tier prefill: raw K
+    once (summaries), K and V of every token once (sinks and fixed windows;
+    window chunks shared by consecutive waves move on the device), and K and
+    V of every routed group of every (block, KV head)."""
+    row = w.Hkv * w.D * 2
+    routed = int((sel_group >= 0).sum().item()) * w.g_s * w.D * 2 * 2
+    return w.B * w.T * row + 2 * w.B * w.T * row + routed
+
+
+def bench_hosttier(args, dev, world):
+    """The 64K prefill with K/V in pinned host RAM; tokens/s and the fraction
+    of the host-to-device copy bandwidth measured in the same run."""
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_kv_routing_b200 as hga
+    from workloads import WORKLOADS, make_prefill_inputs
+    w = WORKLOADS[HOSTTIER_WORKLOAD]
+    hp = params_of(w)
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=args.seed + 77, device=dev)
+    kh, vh = k.cpu().pin_memory(), v.cpu().pin_memory()
+    del k, v
+    stream = torch.cuda.current_stream(dev)
+    n = hga.hga_workspace_size(hga.PREFILL_HOSTKV, w.B, w.T, w.Hq, w.Hkv, w.D, torch.bfloat16, hp)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    res = hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, want_sel=True, workspace=ws)
+    link = hosttier_link_bytes(w, res["sel_group"])
+    for _ in range(max(2, min(args.warmup, 3))):
+        hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    steps = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = torch.tensor([e0.elapsed_time(e1) / steps], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    # host-to-device peak of this box: copy engine, pinned source, 256 MiB
+    src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    best = 0.0
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dst.copy_(src, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        best = max(best, src.numel() / (a.elapsed_time(b) / 1e3) / 1e9)
+    achieved = link / (ms / 1e3) / 1e9
+    return {"metric": "host-tier prefill tokens/s", "value": world * w.B * w.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+                       "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
+                       "tier": "raw K and V in pinned host RAM; summaries, Q, O and two "
+                               "32-block staging buffers in HBM"},
+            "roofline": {"bound": "host link", "achieved": achieved, "peak": best,
+                         "unit": "GB/s", "frac": achieved / best, "bytes_per_step": link,
+                         "peak_source": "measured in this run: pinned host -> device copy "
+                                        "of 256 MiB, best of 5"}}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -464,6 +537,7 @@ def main():
     d2h = hout.numel() * hout.element_size()
 
     dec = None if args.no_decode else bench_decode(args, dev, world)
+    tier = None if args.no_hosttier else bench_hosttier(args, dev, world)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -491,6 +565,8 @@ def main():
             "roofline": roof}
     if dec is not None:
         line["decode"] = dec
+    if tier is not None:
+        line["hosttier"] = tier
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.seed)
     if args.seq or args.no_e2e:

@@ -23,10 +23,10 @@ import torch
 __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "hga_route",
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
            "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
-           "decode_workspace", "HGAError", "PREFILL",
-           "DECODE"]
+           "decode_workspace", "hga_forward_prefill_hostkv", "HGAError", "PREFILL",
+           "DECODE", "PREFILL_HOSTKV"]
 
-PREFILL, DECODE = 0, 1
+PREFILL, DECODE, PREFILL_HOSTKV = 0, 1, 2
 _F32, _BF16 = 0, 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libhga.so")
@@ -320,6 +320,46 @@ def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCa
     return res
 
 
+def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out=None,
+                               want_lse=False, want_sel=False, workspace=None, stream=None):
+    """Prefill with the token K/V history in host RAM (the host-resident
+    tier).  q [B,T,Hq,D] and pos [B,T] are CUDA tensors; k_host and v_host
+    [B,T,Hkv,D] are pinned CPU tensors (raw keys, values).  Returns the same
+    dict as hga_forward_prefill; the outputs equal that call's."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    Hkv = k_host.shape[2]
+    for t, name in ((k_host, "k_host"), (v_host, "v_host")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+            raise HGAError(f"{name} must be a pinned CPU tensor")
+        if not t.is_contiguous() or tuple(t.shape) != (B, T, Hkv, D) or t.dtype != q.dtype:
+            raise HGAError(f"{name} must be contiguous {(B, T, Hkv, D)} {q.dtype}")
+    _need(pos, "pos", (B, T), torch.int32)
+    NB = (T + params.C - 1) // params.C
+    res = {"out": torch.empty_like(q) if out is None else out}
+    io = _IO()
+    io.q, io.k, io.v, io.pos = q.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), pos.data_ptr()
+    io.out = res["out"].data_ptr()
+    if want_lse:
+        res["lse"] = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+        io.lse = res["lse"].data_ptr()
+    if want_sel:
+        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+        io.sel_chunk = res["sel_chunk"].data_ptr()
+        io.sel_group = res["sel_group"].data_ptr()
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    nbytes = int(lib.hga_workspace_size(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc)))
+    ws = _workspace(nbytes, q.device, workspace, zero=False)
+    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
+    st = lib.hga_forward(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    _check(st, "hga_forward(prefill, host K/V)")
+    return res
+
+
 def hga_fill_cache(k, v, pos, cache: "KVCache", params: HGAParams, *, stream=None):
     """Fill a decode cache from a prompt's raw keys, values and positions
     (stage 1 only: rotated keys, values, positions, summaries, lens = T)."""
@@ -409,10 +449,13 @@ def decode_workspace(B, capacity, Hq, Hkv, D, dtype, params: HGAParams, device="
 
 
 def hga_forward(mode: int, *args, **kw):
-    """hga_forward(PREFILL, q, k, v, pos, params, ...) or
-    hga_forward(DECODE, q_new, k_new, v_new, pos_new, cache, params, ...)."""
+    """hga_forward(PREFILL, q, k, v, pos, params, ...),
+    hga_forward(DECODE, q_new, k_new, v_new, pos_new, cache, params, ...) or
+    hga_forward(PREFILL_HOSTKV, q, k_host, v_host, pos, params, ...)."""
     if mode == PREFILL:
         return hga_forward_prefill(*args, **kw)
     if mode == DECODE:
         return hga_forward_decode(*args, **kw)
+    if mode == PREFILL_HOSTKV:
+        return hga_forward_prefill_hostkv(*args, **kw)
     raise HGAError(f"unknown mode {mode}")

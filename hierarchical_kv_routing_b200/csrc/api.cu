@@ -178,6 +178,7 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
     const Geo g = make_geo(dims, prm);
     if (mode == HGA_PREFILL) return prefill_ws(g, dims->dtype).total;
     if (mode == HGA_DECODE) return decode_workspace_bytes(g);
+    if (mode == HGA_PREFILL_HOSTKV) return hostkv_workspace_bytes(g);
     return 0;
 }
 
@@ -246,6 +247,16 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
             !aligned16(cc.k_open) || !aligned16(cc.s_chunk) || !aligned16(cc.s_group))
             return HGA_ERR_INVALID_ARG;
         return launch_decode(g, r, dims->dtype, *io, workspace, st);
+    }
+    if (mode == HGA_PREFILL_HOSTKV) {
+        if (dims->T == 0) return HGA_OK;
+        if (!ws_ok) return HGA_ERR_WORKSPACE;
+        if (dims->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
+        if (!io->q || !io->k || !io->v || !io->pos || !io->out || io->cache.k_rot)
+            return HGA_ERR_INVALID_ARG;
+        if (!aligned16(io->q) || !aligned16(io->k) || !aligned16(io->v) || !aligned16(io->out))
+            return HGA_ERR_INVALID_ARG;
+        return launch_prefill_hostkv(g, r, *io, workspace, st);
     }
     return HGA_ERR_INVALID_ARG;
 }

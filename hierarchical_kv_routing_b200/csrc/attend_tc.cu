@@ -70,6 +70,12 @@ struct TcArgs {
     int T, Hq, Hkv, G, NB, F, L, K_g, g_s, k_T, v_T;
     int rows_per_unit, ctas_per_unit, tokM;
     int cs_tokens;            // > 0: the CTA's (token, pair) cos/sin table is in smem
+    int c0;                   // first query block of this launch
+    // Host-resident tier: K/V rows come from a wave's staging buffer, not from
+    // the token layout.  Tokens below sink_rows sit at row = token; other
+    // tokens at row = win_row0 + token - win_tok0; group slot j of block c at
+    // rows rt_row0 + ((c - c0) * K_g + j) * g_s.
+    int tier, sink_rows, win_tok0, win_row0, rt_row0;
     const int32_t *sel_group;
     const int32_t *pos;
     __nv_bfloat16 *out;
@@ -101,7 +107,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     __shared__ Ctl ctl;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x / A.ctas_per_unit, cu = blockIdx.x % A.ctas_per_unit;
+    const int c = A.c0 + blockIdx.x / A.ctas_per_unit, cu = blockIdx.x % A.ctas_per_unit;
     const int h = blockIdx.y, b = blockIdx.z;
     const int t0 = c * kChunk;
     const int row0 = cu * 256;
@@ -147,8 +153,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int nsink = min(A.F, c);
         const int rec_lo = max(c - max(A.L, 1), nsink);
         const int n_fixed = 8 * (nsink + (c - rec_lo));
+        // load row of a token: itself, or its place in the tier's window
+        auto row_of = [&](int tok) {
+            return (!A.tier || tok < A.sink_rows) ? tok : A.win_row0 + tok - A.win_tok0;
+        };
         for (int s = lane; s < n_fixed; s += 32)
-            ctl.seg_tok[s] = s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8;
+            ctl.seg_tok[s] = row_of(s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8);
         const int32_t *sel = A.sel_group + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_g;
         const int gseg = A.g_s / 8;
         int kg = 0;
@@ -157,12 +167,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             kg += __popc(__ballot_sync(0xffffffffu, v >= 0));
         }
         for (int j = lane; j < kg; j += 32) {
-            const int g = sel[j];
-            for (int e = 0; e < gseg; ++e) ctl.seg_tok[n_fixed + j * gseg + e] = g * A.g_s + e * 8;
+            const int r0 = A.tier ? A.rt_row0 + ((c - A.c0) * A.K_g + j) * A.g_s : sel[j] * A.g_s;
+            for (int e = 0; e < gseg; ++e) ctl.seg_tok[n_fixed + j * gseg + e] = r0 + e * 8;
         }
         const int n_route = n_fixed + kg * gseg;
         const int ncur = (max_tok - t0) / 8 + 1;
-        for (int e = lane; e < ncur; e += 32) ctl.seg_tok[n_route + e] = t0 + e * 8;
+        for (int e = lane; e < ncur; e += 32) ctl.seg_tok[n_route + e] = row_of(t0 + e * 8);
         int nseg = n_route + ncur;
         if (lane == 0) {
             if (nseg & 1) ctl.seg_tok[nseg++] = kDummy;
@@ -308,6 +318,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int tok = t0 + R / A.G;
         const int head = R % A.G;
         const bool valid = mt < NT && (mt * 128 + r) < rows && tok < A.T;
+        // token of a current-chunk row: row + cur_shift
+        const int cur_shift = (A.tier && t0 >= A.sink_rows) ? A.win_tok0 - A.win_row0 : 0;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
         if (mt < NT) {
             // RoPE of this row's query, in place in the swizzled Q tile
@@ -357,10 +369,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const int nj = nsj * 8;
                 const bool need_mask = (j + 1) * kSegPerTile > first_cur;
                 const int *segs = ctl.seg_tok + j * kSegPerTile;
+                // only the current chunk's segments can lie after the query
                 auto masked = [&](int col) -> bool {
                     if (col >= nj) return true;
                     const int st = segs[col >> 3];
-                    return st == kDummy || st + (col & 7) > tok;
+                    if (st == kDummy) return true;
+                    return j * kSegPerTile + (col >> 3) >= first_cur && st + cur_shift + (col & 7) > tok;
                 };
                 // one TMEM pass: the S row (up to 128 columns) into registers
                 uint32_t v[128];
@@ -501,8 +515,15 @@ bool make_map(CUtensorMap *m, const void *base, int D, int heads, long long n_ro
 template <int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, const void *k_rot,
                int k_T, const void *v, int v_T, const int32_t *sel_group, void *out, float *lse,
-               cudaStream_t st) {
+               cudaStream_t st, const TierWave *tw) {
     TcArgs a;
+    a.c0 = tw ? tw->c0 : 0;
+    a.tier = tw != nullptr;
+    a.sink_rows = tw ? tw->sink_rows : 0;
+    a.win_tok0 = tw ? tw->win_tok0 : 0;
+    a.win_row0 = tw ? tw->win_row0 : 0;
+    a.rt_row0 = tw ? tw->rt_row0 : 0;
+    const int nblk = tw ? tw->c1 - tw->c0 : g.NB;
     a.T = g.T;
     a.Hq = g.Hq;
     a.Hkv = g.Hkv;
@@ -542,7 +563,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     auto kern = k_attend_tc<D>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
-    dim3 grid(g.NB * a.ctas_per_unit, g.Hkv, g.B);
+    dim3 grid(nblk * a.ctas_per_unit, g.Hkv, g.B);
     kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mk16, mv16, mk64, mv64, a);
     return cuda_status(cudaGetLastError());
 }
@@ -559,10 +580,11 @@ bool attend_tc_supported(const Geo &g, int dtype) {
 
 hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                             const void *k_rot, int k_T, const void *v, int v_T,
-                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st) {
-    if (g.NB <= 0) return HGA_OK;
-    return g.D == 128 ? run<128>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st)
-                      : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
+                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st,
+                            const TierWave *tw) {
+    if (g.NB <= 0 || (tw && tw->c1 <= tw->c0)) return HGA_OK;
+    return g.D == 128 ? run<128>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw)
+                      : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw);
 }
 
 }  // namespace hga

@@ -89,8 +89,9 @@ __device__ void close_chunk(const DecodeArgs &A, int b, int h, int c, int32_t po
             const float x = to_f(ko[(int64_t)j * D + i]), y = to_f(ko[(int64_t)j * D + i + H]);
             if (hf) {
                 const float2 r = rope_cs(A.rope, (double)pj, i);
-                a += (double)(x * r.x - y * r.y);
-                d2 += (double)(y * r.x + x * r.y);
+                const float2 rr = rot_pair(x, y, r);
+                a += (double)rr.x;
+                d2 += (double)rr.y;
             } else {
                 a += (double)x;
                 d2 += (double)y;
@@ -138,8 +139,9 @@ __device__ __forceinline__ void rotate_new_key(const DecodeArgs &A, int b, int h
         const T *kn = static_cast<const T *>(A.k_new) + ((int64_t)b * A.Hkv + h) * D;
         const float x = to_f(kn[i]), y = to_f(kn[i + H]);
         const float2 r = rope_cs(A.rope, (double)pnew, i);
-        knew[i] = from_f<T>(x * r.x - y * r.y);
-        knew[i + H] = from_f<T>(y * r.x + x * r.y);
+        const float2 rr = rot_pair(x, y, r);
+        knew[i] = from_f<T>(rr.x);
+        knew[i + H] = from_f<T>(rr.y);
     }
 }
 
@@ -371,8 +373,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
         for (int i = threadIdx.x; i < H; i += blockDim.x) {
             const float x = to_f(kn[i]), y = to_f(kn[i + H]);
             const float2 r = rope_cs(A.rope, (double)pnew, i);
-            kr[i] = from_f<T>(x * r.x - y * r.y);
-            kr[i + H] = from_f<T>(y * r.x + x * r.y);
+            const float2 rr = rot_pair(x, y, r);
+            kr[i] = from_f<T>(rr.x);
+            kr[i + H] = from_f<T>(rr.y);
             ko[i] = kn[i];
             ko[i + H] = kn[i + H];
         }

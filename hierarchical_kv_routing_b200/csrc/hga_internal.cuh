@@ -57,6 +57,14 @@ __device__ __forceinline__ float2 rope_cs(const Rope &r, double p, int i) {
 
 __device__ __forceinline__ bool is_high(const Rope &r, int i) { return (r.high >> i) & 1ull; }
 
+// Rotate the pair (x, y) by the angle whose (cos, sin) is cs.  The rounding
+// is spelled out (one product rounded, then one fused multiply-add) so every
+// kernel that writes rotated keys produces the same bits for the same input.
+__device__ __forceinline__ float2 rot_pair(float x, float y, float2 cs) {
+    return make_float2(__fmaf_rn(x, cs.x, -__fmul_rn(y, cs.y)),
+                       __fmaf_rn(y, cs.x, __fmul_rn(x, cs.y)));
+}
+
 // Routing keys: a score and a candidate id packed so that a larger key means
 // a higher score, and on equal scores the lower id.  0 = no candidate.
 __device__ __forceinline__ unsigned long long pack_key(float score, int id) {
@@ -99,12 +107,13 @@ cudaError_t ensure_smem(const void *kernel, size_t bytes);
 
 // Stage 1.  k_rot/v_out/pos_out/k_open/lens may be null.  in_T: tokens per
 // sequence of the inputs; out_T: token capacity of k_rot/v_out/pos_out;
-// nc_cap: chunk capacity of s_chunk/s_group.
+// nc_cap: chunk capacity of s_chunk/s_group.  host_src: k_raw is the device
+// address of pinned host memory (read with plain loads; bf16, summaries only).
 hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *k_raw,
                             const void *v_raw, const int32_t *pos, int in_T, void *k_rot,
                             void *v_out, int32_t *pos_out, int out_T, float *s_chunk,
                             float *s_group, int nc_cap, void *k_open, int32_t *lens,
-                            cudaStream_t st);
+                            cudaStream_t st, bool host_src = false);
 
 // Stage 2 (prefill blocks).
 hga_status launch_route(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
@@ -120,9 +129,26 @@ hga_status launch_attend_simt(const Geo &g, const Rope &r, int dtype, const void
                               cudaStream_t st);
 size_t attend_simt_smem(const Geo &g);
 bool attend_tc_supported(const Geo &g, int dtype);
+
+// One wave of query blocks [c0, c1) whose keys and values sit in a staging
+// buffer of the host-resident tier (rows per sequence: the buffer's k_T):
+// tokens below sink_rows at row = token, other fixed-window and current
+// tokens at row = win_row0 + token - win_tok0, and group slot j of block c at
+// rows rt_row0 + ((c - c0) * K_g + j) * g_s (slot j holds the j-th routed id).
+struct TierWave {
+    int c0, c1, sink_rows, win_tok0, win_row0, rt_row0;
+};
+
+// tw == nullptr: every query block, keys at their token rows.
 hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                             const void *k_rot, int k_T, const void *v, int v_T,
-                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st);
+                            const int32_t *sel_group, void *out, float *lse, cudaStream_t st,
+                            const TierWave *tw = nullptr);
+
+// Prefill with K and V in pinned host memory (hga_forward HGA_PREFILL_HOSTKV).
+size_t hostkv_workspace_bytes(const Geo &g);
+hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, void *ws,
+                                 cudaStream_t st);
 
 // Decode step (append, close-chunk summaries, route, split attention).
 size_t decode_workspace_bytes(const Geo &g);

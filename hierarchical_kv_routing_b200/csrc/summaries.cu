@@ -7,145 +7,226 @@
 // low-frequency pairs are the mean raw key rotated at the set's mean position.
 // Summaries are routing keys only; they never enter the attention output.
 //
-// Design (HBM-bound stream): one CTA per (chunk, sequence) handles all KV
-// heads, so each (token, pair) angle is computed once into shared memory and
-// reused Hkv times.  Each key row is read once with 16-byte vector loads and
-// written once (K_rot); set sums are accumulated in fp64 from shared memory.
+// Design (HBM-bound stream): one CTA per (chunk, sequence).  The chunk's key
+// rows (all KV heads, or a slab of heads when they do not fit) arrive in
+// shared memory as one bulk copy while the CTA computes every (token, pair)
+// angle once for all heads.  Then each thread owns one (head, pair): it walks
+// the 64 tokens, rotates in place, and keeps the group and chunk sums in fp64
+// registers, so no shared-memory reduction is needed; the rotated rows leave
+// as one bulk store (K_rot).  Keys that live in pinned host memory (the
+// host-resident tier) are read with plain loads instead of the bulk copy.
 #include "hga_internal.cuh"
-#include "vec.cuh"
+#include "sm100.cuh"
 
 namespace hga {
+
+__device__ int g_summaries_error = 0;
+
 namespace {
 
-constexpr int kThreads = 256;
+using namespace sm100;
 
-// Shared memory: cos/sin per (token, pair) [64][D/2] float2, then the values
-// to be averaged per (token, dim) [64][D] float (rotated on high pairs, raw on
-// low pairs).
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-k_summaries(const T *__restrict__ k_raw, const T *__restrict__ v_raw,
-            const int32_t *__restrict__ pos, int in_T, int Hkv, T *__restrict__ k_rot,
-            T *__restrict__ v_out, int32_t *__restrict__ pos_out, int out_T,
-            float *__restrict__ s_chunk, float *__restrict__ s_group, int nc_cap,
-            T *__restrict__ k_open, int32_t *__restrict__ lens, int g_s, Rope rope) {
-    constexpr int C = kChunk, H = D / 2, PS = H / 4;  // pairs per thread slice
-    extern __shared__ __align__(16) unsigned char smem[];
-    float2 *cs = reinterpret_cast<float2 *>(smem);                // [C][H]
-    float *val = reinterpret_cast<float *>(smem + sizeof(float2) * C * H);  // [C][D]
+constexpr int kThreads = 256;
+constexpr int kSlabBytes = 64 * 1024;   // key rows of one head slab of one chunk
+
+struct SumArgs {
+    const void *k_raw, *v_raw;
+    const int32_t *pos;
+    int in_T, Hkv, HS;          // HS: heads per slab
+    void *k_rot, *v_out;
+    int32_t *pos_out;
+    int out_T;
+    float *s_chunk, *s_group;
+    int nc_cap;
+    void *k_open;
+    int32_t *lens;
+    int g_s;
+    Rope rope;
+};
+
+// Plain 16-byte load (no read-only path; used for pinned host memory).
+__device__ __forceinline__ uint4 ld16_plain(const void *p) {
+    uint4 w;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                 : "l"(p));
+    return w;
+}
+
+// Summary of one set for pair i from its fp64 sums: high pairs are the mean
+// of the rotated keys; low pairs the mean raw key rotated at the set's mean
+// position.
+__device__ __forceinline__ void write_summary(const Rope &rope, bool hf, int i, int H, double sx,
+                                              double sy, int cnt, double pmid, float *dst) {
+    const double a = sx / (double)cnt, c2 = sy / (double)cnt;
+    float o0, o1;
+    if (hf) {
+        o0 = (float)a;
+        o1 = (float)c2;
+    } else {
+        const float2 r = rope_cs(rope, pmid, i);
+        o0 = (float)(a * (double)r.x - c2 * (double)r.y);
+        o1 = (float)(c2 * (double)r.x + a * (double)r.y);
+    }
+    dst[i] = o0;
+    dst[i + H] = o1;
+}
+
+template <typename T, int D, bool kHost>
+__global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
+    constexpr int C = kChunk, H = D / 2;
+    extern __shared__ __align__(128) unsigned char smem[];
+    T *kb = reinterpret_cast<T *>(smem);                          // [n][nh][D]
+    float2 *cs = reinterpret_cast<float2 *>(smem + kSlabBytes);   // [n][H]
     __shared__ double s_pmid[C + 1];
+    __shared__ __align__(8) uint64_t bar;
 
     const int m = blockIdx.x, b = blockIdx.y;
     const int t0 = m * C;
-    const int n = min(C, in_T - t0);
-    const bool closed = (n == C);
-    const int gpc = C / g_s;
-    const int32_t *pb = pos + (int64_t)b * in_T + t0;
+    const int n = min(C, A.in_T - t0);
+    const bool closed = n == C;
+    const int gpc = C / A.g_s;
+    const int32_t *pb = A.pos + (int64_t)b * A.in_T + t0;
+    const T *kin = static_cast<const T *>(A.k_raw);
 
-    for (int e = threadIdx.x; e < C * H; e += kThreads) {
-        const int j = e / H, i = e % H;
-        if (j < n) cs[e] = rope_cs(rope, (double)pb[j], i);
-    }
-    if (pos_out)
-        for (int j = threadIdx.x; j < n; j += kThreads) pos_out[(int64_t)b * out_T + t0 + j] = pb[j];
-    if (lens && m == 0 && threadIdx.x == 0) lens[b] = in_T;
-    // mean positions: chunk (index gpc) and groups (0..gpc-1)
-    if (closed && threadIdx.x <= gpc) {
-        const int g = threadIdx.x;
-        const int lo = g < gpc ? g * g_s : 0, cnt = g < gpc ? g_s : C;
-        double acc = 0.0;
-        for (int j = 0; j < cnt; ++j) acc += (double)pb[lo + j];
-        s_pmid[g] = acc / (double)cnt;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
     }
     __syncthreads();
 
-    const int j = threadIdx.x >> 2, sl = threadIdx.x & 3;
-    for (int h = 0; h < Hkv; ++h) {
-        if (j < n) {
-            const int64_t in_row = ((int64_t)b * in_T + t0 + j) * Hkv + h;
-            const int64_t out_row = ((int64_t)b * out_T + t0 + j) * Hkv + h;
-            float lo[PS], hi[PS], rlo[PS], rhi[PS];
-            load_slice<T, PS>(k_raw + in_row * D + sl * PS, lo);
-            load_slice<T, PS>(k_raw + in_row * D + H + sl * PS, hi);
-#pragma unroll
-            for (int p = 0; p < PS; ++p) {
-                const float2 c = cs[j * H + sl * PS + p];
-                rlo[p] = lo[p] * c.x - hi[p] * c.y;
-                rhi[p] = hi[p] * c.x + lo[p] * c.y;
-            }
-            if (k_rot) {
-                store_slice<T, PS>(k_rot + out_row * D + sl * PS, rlo);
-                store_slice<T, PS>(k_rot + out_row * D + H + sl * PS, rhi);
-            }
-            if (v_out) {
-                float a[PS], c2[PS];
-                load_slice<T, PS>(v_raw + in_row * D + sl * PS, a);
-                load_slice<T, PS>(v_raw + in_row * D + H + sl * PS, c2);
-                store_slice<T, PS>(v_out + out_row * D + sl * PS, a);
-                store_slice<T, PS>(v_out + out_row * D + H + sl * PS, c2);
-            }
-            if (!closed && k_open) {
-                T *ko = k_open + (((int64_t)b * Hkv + h) * C + j) * D;
-                store_slice<T, PS>(ko + sl * PS, lo);
-                store_slice<T, PS>(ko + H + sl * PS, hi);
-            }
-            if (closed) {
-#pragma unroll
-                for (int p = 0; p < PS; ++p) {
-                    const int i = sl * PS + p;
-                    const bool hf = is_high(rope, i);
-                    val[j * D + i] = hf ? rlo[p] : lo[p];
-                    val[j * D + i + H] = hf ? rhi[p] : hi[p];
+    int pass = 0;
+    for (int hs0 = 0; hs0 < A.Hkv; hs0 += A.HS, ++pass) {
+        const int nh = min(A.HS, A.Hkv - hs0);
+        const uint32_t row_bytes = (uint32_t)(nh * D * sizeof(T));
+        const T *src0 = kin + (((int64_t)b * A.in_T + t0) * A.Hkv + hs0) * D;
+        if constexpr (!kHost) {
+            if (threadIdx.x == 0) {
+                mbar_arrive_expect_tx(&bar, row_bytes * n);
+                if (nh == A.Hkv) {
+                    bulk_load(kb, src0, row_bytes * n, &bar);       // contiguous rows
+                } else {
+                    for (int j = 0; j < n; ++j)
+                        bulk_load(kb + (size_t)j * nh * D, src0 + (int64_t)j * A.Hkv * D, row_bytes,
+                                  &bar);
                 }
+            }
+        } else {
+            // eight independent loads in flight per thread (the link's latency
+            // is microseconds), then the shared-memory stores
+            const int wpr = (int)(row_bytes / 16), nw = n * wpr;
+            for (int base = 0; base < nw; base += 8 * kThreads) {
+                uint4 w[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int idx = base + u * kThreads + threadIdx.x;
+                    if (idx < nw)
+                        w[u] = ld16_plain(reinterpret_cast<const uint4 *>(
+                                              src0 + (int64_t)(idx / wpr) * A.Hkv * D) + idx % wpr);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int idx = base + u * kThreads + threadIdx.x;
+                    if (idx < nw) reinterpret_cast<uint4 *>(kb)[idx] = w[u];
+                }
+            }
+        }
+        if (pass == 0) {
+            // while the keys are in flight: angles, mean positions, copies
+            for (int e = threadIdx.x; e < n * H; e += kThreads)
+                cs[e] = rope_cs(A.rope, (double)pb[e / H], e % H);
+            if (closed && threadIdx.x <= gpc) {
+                const int g = threadIdx.x;
+                const int lo = g < gpc ? g * A.g_s : 0, cnt = g < gpc ? A.g_s : C;
+                double acc = 0.0;
+                for (int j = 0; j < cnt; ++j) acc += (double)pb[lo + j];
+                s_pmid[g] = acc / (double)cnt;
+            }
+            if (A.pos_out)
+                for (int j = threadIdx.x; j < n; j += kThreads)
+                    A.pos_out[(int64_t)b * A.out_T + t0 + j] = pb[j];
+            if (A.lens && m == 0 && threadIdx.x == 0) A.lens[b] = A.in_T;
+            if (A.v_out) {
+                const int wpr = A.Hkv * D * (int)sizeof(T) / 16;
+                const uint4 *vs = reinterpret_cast<const uint4 *>(
+                    static_cast<const T *>(A.v_raw) + ((int64_t)b * A.in_T + t0) * A.Hkv * D);
+                uint4 *vd = reinterpret_cast<uint4 *>(
+                    static_cast<T *>(A.v_out) + ((int64_t)b * A.out_T + t0) * A.Hkv * D);
+                for (int w = threadIdx.x; w < n * wpr; w += kThreads) vd[w] = __ldg(vs + w);
             }
         }
         __syncthreads();
-        if (closed) {
-            // one work item per (set, pair): sets 0..gpc-1 are groups, gpc the chunk
-            for (int e = threadIdx.x; e < (gpc + 1) * H; e += kThreads) {
-                const int set = e / H, i = e % H;
-                const int lo = set < gpc ? set * g_s : 0, cnt = set < gpc ? g_s : C;
-                double a = 0.0, c2 = 0.0;
-                for (int jj = 0; jj < cnt; ++jj) {
-                    a += (double)val[(lo + jj) * D + i];
-                    c2 += (double)val[(lo + jj) * D + i + H];
-                }
-                a /= (double)cnt;
-                c2 /= (double)cnt;
-                float o0, o1;
-                if (is_high(rope, i)) {
-                    o0 = (float)a;
-                    o1 = (float)c2;
-                } else {
-                    const float2 r = rope_cs(rope, s_pmid[set], i);
-                    o0 = (float)(a * (double)r.x - c2 * (double)r.y);
-                    o1 = (float)(c2 * (double)r.x + a * (double)r.y);
-                }
-                float *dst = set < gpc
-                    ? s_group + ((((int64_t)b * Hkv + h) * nc_cap + m) * gpc + set) * D
-                    : s_chunk + (((int64_t)b * Hkv + h) * nc_cap + m) * D;
-                dst[i] = o0;
-                dst[i + H] = o1;
+        if constexpr (!kHost) {
+            if (!mbar_wait(&bar, pass & 1)) {
+                if (threadIdx.x == 0) atomicExch(&g_summaries_error, (int)HGA_ERR_TIMEOUT);
+                return;
             }
-            __syncthreads();
         }
+
+        // one (head, pair) per thread: rotate in place, fp64 set sums
+        for (int e = threadIdx.x; e < nh * H; e += kThreads) {
+            const int hh = e / H, i = e % H;
+            const int h = hs0 + hh;
+            const bool hf = is_high(A.rope, i);
+            T *ko = (!closed && A.k_open)
+                ? static_cast<T *>(A.k_open) + ((int64_t)b * A.Hkv + h) * C * D : nullptr;
+            float *sg = A.s_group + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * gpc * D;
+            double gx = 0.0, gy = 0.0, cx = 0.0, cy = 0.0;
+            for (int j = 0; j < n; ++j) {
+                T *px = kb + ((size_t)j * nh + hh) * D + i;
+                const float x = to_f(px[0]), y = to_f(px[H]);
+                const float2 rr = rot_pair(x, y, cs[j * H + i]);
+                if (ko) {
+                    ko[(int64_t)j * D + i] = px[0];
+                    ko[(int64_t)j * D + i + H] = px[H];
+                }
+                px[0] = from_f<T>(rr.x);
+                px[H] = from_f<T>(rr.y);
+                if (closed) {
+                    gx += (double)(hf ? rr.x : x);
+                    gy += (double)(hf ? rr.y : y);
+                    if ((j + 1) % A.g_s == 0) {
+                        const int set = j / A.g_s;
+                        write_summary(A.rope, hf, i, H, gx, gy, A.g_s, s_pmid[set],
+                                      sg + (int64_t)set * D);
+                        cx += gx;
+                        cy += gy;
+                        gx = gy = 0.0;
+                    }
+                }
+            }
+            if (closed)
+                write_summary(A.rope, hf, i, H, cx, cy, C, s_pmid[gpc],
+                              A.s_chunk + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * D);
+        }
+        // rotated rows out
+        if (A.k_rot) {
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                T *dst0 = static_cast<T *>(A.k_rot) + (((int64_t)b * A.out_T + t0) * A.Hkv + hs0) * D;
+                if (nh == A.Hkv) {
+                    bulk_store(dst0, kb, row_bytes * n);
+                } else {
+                    for (int j = 0; j < n; ++j)
+                        bulk_store(dst0 + (int64_t)j * A.Hkv * D, kb + (size_t)j * nh * D, row_bytes);
+                }
+                bulk_commit();
+                bulk_wait_read();
+            }
+        }
+        __syncthreads();
     }
 }
 
-template <typename T, int D>
-hga_status run(const Geo &g, const Rope &r, const void *k_raw, const void *v_raw,
-               const int32_t *pos, int in_T, void *k_rot, void *v_out, int32_t *pos_out,
-               int out_T, float *s_chunk, float *s_group, int nc_cap, void *k_open,
-               int32_t *lens, cudaStream_t st) {
-    const size_t smem = sizeof(float2) * kChunk * (D / 2) + sizeof(float) * kChunk * D;
-    auto kern = k_summaries<T, D>;
+template <typename T, int D, bool kHost>
+hga_status run(const Geo &g, const SumArgs &a, int in_T, cudaStream_t st) {
+    const size_t smem = kSlabBytes + sizeof(float2) * kChunk * (D / 2);
+    auto kern = k_summaries<T, D, kHost>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid((in_T + kChunk - 1) / kChunk, g.B);
-    kern<<<grid, kThreads, smem, st>>>(
-        static_cast<const T *>(k_raw), static_cast<const T *>(v_raw), pos, in_T, g.Hkv,
-        static_cast<T *>(k_rot), static_cast<T *>(v_out), pos_out, out_T, s_chunk, s_group,
-        nc_cap, static_cast<T *>(k_open), lens, g.g_s, r);
+    kern<<<grid, kThreads, smem, st>>>(a);
     return cuda_status(cudaGetLastError());
 }
 
@@ -155,20 +236,38 @@ hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *
                             const void *v_raw, const int32_t *pos, int in_T, void *k_rot,
                             void *v_out, int32_t *pos_out, int out_T, float *s_chunk,
                             float *s_group, int nc_cap, void *k_open, int32_t *lens,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool host_src) {
     if (in_T <= 0) return HGA_OK;
-    if (dtype == HGA_BF16) {
-        if (g.D == 128)
-            return run<__nv_bfloat16, 128>(g, r, k_raw, v_raw, pos, in_T, k_rot, v_out, pos_out,
-                                           out_T, s_chunk, s_group, nc_cap, k_open, lens, st);
-        return run<__nv_bfloat16, 64>(g, r, k_raw, v_raw, pos, in_T, k_rot, v_out, pos_out, out_T,
-                                      s_chunk, s_group, nc_cap, k_open, lens, st);
+    const size_t es = dtype == HGA_BF16 ? 2 : 4;
+    SumArgs a;
+    a.k_raw = k_raw;
+    a.v_raw = v_raw;
+    a.pos = pos;
+    a.in_T = in_T;
+    a.Hkv = g.Hkv;
+    const int fit = (int)(kSlabBytes / (kChunk * g.D * es));
+    a.HS = fit < 1 ? 1 : (fit < g.Hkv ? fit : g.Hkv);
+    a.k_rot = k_rot;
+    a.v_out = v_out;
+    a.pos_out = pos_out;
+    a.out_T = out_T;
+    a.s_chunk = s_chunk;
+    a.s_group = s_group;
+    a.nc_cap = nc_cap;
+    a.k_open = k_open;
+    a.lens = lens;
+    a.g_s = g.g_s;
+    a.rope = r;
+    if (host_src) {
+        // the host-resident tier: bf16 keys only, no copies to the device
+        if (dtype != HGA_BF16 || v_raw || v_out || k_open) return HGA_ERR_UNSUPPORTED;
+        return g.D == 128 ? run<__nv_bfloat16, 128, true>(g, a, in_T, st)
+                          : run<__nv_bfloat16, 64, true>(g, a, in_T, st);
     }
-    if (g.D == 128)
-        return run<float, 128>(g, r, k_raw, v_raw, pos, in_T, k_rot, v_out, pos_out, out_T, s_chunk,
-                               s_group, nc_cap, k_open, lens, st);
-    return run<float, 64>(g, r, k_raw, v_raw, pos, in_T, k_rot, v_out, pos_out, out_T, s_chunk,
-                          s_group, nc_cap, k_open, lens, st);
+    if (dtype == HGA_BF16)
+        return g.D == 128 ? run<__nv_bfloat16, 128, false>(g, a, in_T, st)
+                          : run<__nv_bfloat16, 64, false>(g, a, in_T, st);
+    return g.D == 128 ? run<float, 128, false>(g, a, in_T, st) : run<float, 64, false>(g, a, in_T, st);
 }
 
 }  // namespace hga

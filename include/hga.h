@@ -62,7 +62,7 @@ typedef enum hga_status {
 
 typedef enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
 
-typedef enum hga_mode { HGA_PREFILL = 0, HGA_DECODE = 1 } hga_mode;
+typedef enum hga_mode { HGA_PREFILL = 0, HGA_DECODE = 1, HGA_PREFILL_HOSTKV = 2 } hga_mode;
 
 /* Method parameters (page section 3 and its setup table in section 6). */
 typedef struct hga_params {
@@ -178,6 +178,22 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   "append closed chunk"), routes with the token's own query (summed over the
  *   KV head's query heads), attends over the visible set of token t and
  *   increments lens[b].  Requires lens[b] < dims.T.
+ * HGA_PREFILL_HOSTKV: the prefill of HGA_PREFILL with the token K/V history
+ *   in host RAM (page section 3, the three-tier K/V store: the summaries stay
+ *   on the GPU and only routed groups are fetched).  io.k and io.v are HOST
+ *   pointers to pinned, mapped memory (cudaHostAlloc / cudaMallocHost /
+ *   cudaHostRegister with mapping) holding raw K and V [B, T, Hkv, D]; q,
+ *   pos and out (and lse, sel_chunk, sel_group when given) are device
+ *   pointers; io.cache must be empty.  bf16 only, shapes the tensor-core
+ *   attention takes (g_s a multiple of 8, Hq/Hkv a power of two <= 16).
+ *   Stage 1 reads K over the host link once; stage 3 runs in waves of 32
+ *   query blocks whose sink, recent, current and routed K/V rows are fetched
+ *   by the GPU over the link into two HBM staging buffers in the workspace,
+ *   on a library-owned side stream (one per device, created on the first
+ *   such call), the next wave's fetch overlapping this wave's attention; the
+ *   call joins that stream back into `stream` before returning, so the
+ *   caller sees ordinary stream order.  Host memory that is not pinned and
+ *   mapped returns HGA_ERR_INVALID_ARG.  The outputs equal HGA_PREFILL's.
  * workspace: hga_workspace_size(mode) bytes of device memory, 256-byte
  * aligned.  For HGA_DECODE it must be zero-filled before its first use; the
  * library leaves it zeroed between calls.  Calls that share a workspace must

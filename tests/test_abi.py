@@ -92,3 +92,25 @@ def test_binding_fails_loudly_without_cuda():
     with pytest.raises(hga.HGAError):
         hga.hga_build_summaries(torch.zeros(1, 64, 1, 64), torch.zeros(1, 64, dtype=torch.int32),
                                 hga.HGAParams())
+
+
+def test_hostkv_mode_host_checks(lib):
+    """HGA_PREFILL_HOSTKV: workspace sized on the host; fp32 and missing
+    buffers rejected before anything is launched (the workspace pointer
+    below is never dereferenced)."""
+    p = hga.HGAParams(F=2, L=8, K_c=16, K_g=32, rope_theta=1e6).c()
+    d = _dims(T=4096, Hq=32, Hkv=4, D=128, dtype=1)
+    n = lib.hga_workspace_size(2, ctypes.byref(d), ctypes.byref(p))
+    # two staging buffers of K and V for a 32-block wave dominate
+    rows = 2 * 64 + (32 + 8) * 64 + 32 * 32 * 16
+    assert n >= 4 * rows * 4 * 128 * 2
+    io = hga._IO()
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.hga_forward(2, ctypes.byref(d), ctypes.byref(p), ctypes.byref(io), fake, n, None)
+    assert st == 1
+    st = lib.hga_forward(2, ctypes.byref(d), ctypes.byref(p), ctypes.byref(io), None, 0, None)
+    assert st == 6
+    d32 = _dims(T=4096, Hq=32, Hkv=4, D=128, dtype=0)
+    n32 = lib.hga_workspace_size(2, ctypes.byref(d32), ctypes.byref(p))
+    st = lib.hga_forward(2, ctypes.byref(d32), ctypes.byref(p), ctypes.byref(io), fake, n32, None)
+    assert st == 2
