@@ -38,6 +38,10 @@ hga_status set_rope(Rope *r, int D, double theta, double hf_wavelength, int C) {
     for (int i = 0; i < D / 2; ++i) {
         r->omega[i] = std::pow(theta, -2.0 * (double)i / (double)D);
         if (2.0 * M_PI / r->omega[i] < hf) r->high |= 1ull << i;
+        // turns per position as a 64-bit fraction (extended precision on the host)
+        const long double two_pi = 6.283185307179586476925286766559L;
+        const long double t = (long double)r->omega[i] / two_pi * 18446744073709551616.0L;
+        r->turn[i] = (unsigned long long)llroundl(t);
     }
     return HGA_OK;
 }

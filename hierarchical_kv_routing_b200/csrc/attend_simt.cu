@@ -62,10 +62,10 @@ k_attend_simt(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen
         float lo[PS], hi[PS];
         load_slice<T, PS>(qrow + sl * PS, lo);
         load_slice<T, PS>(qrow + H + sl * PS, hi);
-        const double pp = (double)pos[(int64_t)b * Tlen + tok];
+        const int32_t pp = pos[(int64_t)b * Tlen + tok];
 #pragma unroll
         for (int p = 0; p < PS; ++p) {
-            const float2 cs = rope_cs(rope, pp, sl * PS + p);
+            const float2 cs = rope_cs_int(rope, pp, sl * PS + p);
             qv[p] = (lo[p] * cs.x - hi[p] * cs.y) * scale_log2;
             qv[PS + p] = (hi[p] * cs.x + lo[p] * cs.y) * scale_log2;
         }

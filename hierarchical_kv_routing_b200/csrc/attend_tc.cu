@@ -39,6 +39,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
+constexpr uint32_t kRegsLaunch = 168;   // 65536 / 384, rounded down to 8
+constexpr uint32_t kRegsCtl = 56;       // warps 0-3: TMA producers, MMA issuer
+constexpr uint32_t kRegsSoftmax = 224;  // warps 4-11: softmax and epilogue
 constexpr int kMaxSeg = 2048;
 constexpr int kSegPerTile = 16;          // 16 x 8 tokens = 128 keys
 constexpr int kDummy = 0x7fffffff;       // padding segment
@@ -63,6 +66,7 @@ struct Ctl {
     uint32_t tmem_base;
     int nseg, first_cur;
     volatile int abort;
+    int s_pos[kChunk];        // positions of this CTA's query tokens
     int seg_tok[kMaxSeg];
 };
 
@@ -147,6 +151,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         tmem_alloc(&ctl.tmem_base, 512);
         tc_fence_before();
     }
+    if (warp == 3) {
+        // positions of the CTA's tokens, one coalesced load
+        const int tk0 = t0 + row0 / A.G;
+        for (int j = lane; j < kChunk; j += 32)
+            ctl.s_pos[j] = tk0 + j < A.T ? A.pos[(int64_t)b * A.T + tk0 + j] : 0;
+    }
     if (warp == 2) {
         // the visible set as 8-token segments: sinks, recent, routed groups,
         // then the current chunk up to this CTA's last query token
@@ -186,19 +196,26 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     const int tok0 = t0 + row0 / A.G;
     float2 *cs_tab = reinterpret_cast<float2 *>(smem + C::oCS);
     if (A.cs_tokens > 0) {
+        // rows padded to H + 1 entries: the 4 tokens a warp reads differ in bank
         constexpr int H = D / 2;
         for (int e = threadIdx.x; e < A.cs_tokens * H; e += kThreads) {
-            const int tk = tok0 + e / H;
-            if (tk < A.T) cs_tab[e] = rope_cs(A.rope, (double)A.pos[(int64_t)b * A.T + tk], e % H);
+            const int tj = e / H;
+            if (tok0 + tj < A.T) cs_tab[tj * (H + 1) + e % H] = rope_cs_int(A.rope, ctl.s_pos[tj], e % H);
         }
         __syncthreads();
     }
     tc_fence_after();
+    // Registers: the producer / MMA warpgroup needs few, the two softmax
+    // warpgroups hold a 128-column S row each.  128 x 56 + 256 x 224 equals
+    // the launch allocation of 384 x 168.
+    static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
     const uint32_t tmem = ctl.tmem_base;
     const int nseg = ctl.nseg;
     const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
     const int first_cur = ctl.first_cur;
 
+    if (warp < 4) {
+    regs_dec<kRegsCtl>();
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------------ producers --
         // warp 0 streams the K tiles, warp 2 the V tiles, each through its own
@@ -309,7 +326,9 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             mma_commit(&ctl.fin);
             if (!mbar_wait(&ctl.fin, 0)) fail(ctl);
         }
-    } else if (warp >= 4) {
+    }
+    } else {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------- softmax --
         const int mt = (warp - 4) >> 2;
         const int q4 = warp & 3;
@@ -318,8 +337,11 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int tok = t0 + R / A.G;
         const int head = R % A.G;
         const bool valid = mt < NT && (mt * 128 + r) < rows && tok < A.T;
-        // token of a current-chunk row: row + cur_shift
-        const int cur_shift = (A.tier && t0 >= A.sink_rows) ? A.win_tok0 - A.win_row0 : 0;
+        // Visible keys of this row, in key-list order: every fixed and routed
+        // key (first_cur segments), then the current chunk's tokens up to the
+        // row's own; only the trailing padding follows.  So a key column is
+        // visible iff its index in the list is below nvis.
+        const int nvis = first_cur * 8 + (tok - t0 + 1);
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
         if (mt < NT) {
             // RoPE of this row's query, in place in the swizzled Q tile
@@ -327,7 +349,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             if (!ok) fail(ctl);
             if (ok && valid) {
                 uint8_t *qt = smem + C::oQ + mt * C::kTileBytes;
-                const double p = (double)A.pos[(int64_t)b * A.T + tok];
+                const int32_t p = ctl.s_pos[tok - tok0];
+                const float2 *csr = cs_tab + (tok - tok0) * (D / 2 + 1);
                 constexpr int kGroups = D / 16;       // 8 pairs per 16-byte chunk
                 for (int g = 0; g < kGroups; ++g) {
                     const int lo_half = 0, hi_half = D == 128 ? 1 : 0;
@@ -343,10 +366,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     for (int e = 0; e < 4; ++e) {
                         const float2 x = __bfloat1622float2(pa[e]);
                         const float2 y = __bfloat1622float2(pb[e]);
-                        const float2 c0 = A.cs_tokens > 0 ? cs_tab[(tok - tok0) * (D / 2) + g * 8 + 2 * e]
-                                                          : rope_cs(A.rope, p, g * 8 + 2 * e);
-                        const float2 c1 = A.cs_tokens > 0 ? cs_tab[(tok - tok0) * (D / 2) + g * 8 + 2 * e + 1]
-                                                          : rope_cs(A.rope, p, g * 8 + 2 * e + 1);
+                        const float2 c0 = A.cs_tokens > 0 ? csr[g * 8 + 2 * e]
+                                                          : rope_cs_int(A.rope, p, g * 8 + 2 * e);
+                        const float2 c1 = A.cs_tokens > 0 ? csr[g * 8 + 2 * e + 1]
+                                                          : rope_cs_int(A.rope, p, g * 8 + 2 * e + 1);
                         pa[e] = __floats2bfloat162_rn(x.x * c0.x - y.x * c0.y, x.y * c1.x - y.y * c1.y);
                         pb[e] = __floats2bfloat162_rn(y.x * c0.x + x.x * c0.y, y.y * c1.x + x.y * c1.y);
                     }
@@ -365,17 +388,9 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     break;
                 }
                 tc_fence_after();
-                const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
-                const int nj = nsj * 8;
-                const bool need_mask = (j + 1) * kSegPerTile > first_cur;
-                const int *segs = ctl.seg_tok + j * kSegPerTile;
-                // only the current chunk's segments can lie after the query
-                auto masked = [&](int col) -> bool {
-                    if (col >= nj) return true;
-                    const int st = segs[col >> 3];
-                    if (st == kDummy) return true;
-                    return j * kSegPerTile + (col >> 3) >= first_cur && st + cur_shift + (col & 7) > tok;
-                };
+                // the row's visible keys are the first nvis columns of the list
+                const int gc0 = j * kSegPerTile * 8;
+                const bool need_mask = gc0 + kSegPerTile * 8 > nvis;
                 // one TMEM pass: the S row (up to 128 columns) into registers
                 uint32_t v[128];
                 tmem_ld32(lane_base + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
@@ -386,7 +401,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 if (need_mask) {
 #pragma unroll
                     for (int e = 0; e < 128; ++e)
-                        if (masked(e)) v[e] = __float_as_uint(-INFINITY);
+                        if (gc0 + e >= nvis) v[e] = __float_as_uint(-INFINITY);
                 }
                 // row max with 8 independent chains (no 128-long dependency)
                 float mx8[8];
@@ -453,20 +468,23 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 const float inv = valid && l > 0.f ? 1.f / l : 0.f;
                 __nv_bfloat16 *orow =
                     A.out + (((int64_t)b * A.T + tok) * A.Hq + (int64_t)h * A.G + head) * D;
-                for (int cb = 0; cb < D / 32; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(lane_base + 128 + cb * 32, v);
+#pragma unroll
+                for (int hb = 0; hb < D / 64; ++hb) {
+                    uint32_t v[64];
+                    tmem_ld32(lane_base + 128 + hb * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                    tmem_ld32(lane_base + 128 + hb * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
                     tmem_ld_wait();
                     if (valid) {
-                        uint4 w[4];
-                        uint32_t *wp = reinterpret_cast<uint32_t *>(w);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            wp[e] = pack_bf16(__uint_as_float(v[2 * e]) * inv,
-                                              __uint_as_float(v[2 * e + 1]) * inv);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cb * 32);
+                        for (int q8 = 0; q8 < 8; ++q8) {
+                            uint4 w;
+                            uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = w[e];
+                            for (int e = 0; e < 4; ++e)
+                                wp[e] = pack_bf16(__uint_as_float(v[q8 * 8 + 2 * e]) * inv,
+                                                  __uint_as_float(v[q8 * 8 + 2 * e + 1]) * inv);
+                            reinterpret_cast<uint4 *>(orow)[hb * 8 + q8] = w;
+                        }
                     }
                 }
                 if (valid && A.lse)
@@ -541,7 +559,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     {
         // the table costs tokens x D/2 x 8 bytes; keep the CTA inside 227 KB
         const int tok_cta = (min(256, a.rows_per_unit) + g.G - 1) / g.G;
-        const size_t tab = (size_t)tok_cta * (D / 2) * sizeof(float2);
+        const size_t tab = (size_t)tok_cta * (D / 2 + 1) * sizeof(float2);
         a.cs_tokens = Cfg<D>::oEnd + 1024 + tab + sizeof(Ctl) <= 232448 ? tok_cta : 0;
     }
     a.sel_group = sel_group;
@@ -559,7 +577,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         !make_map(&mk64, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 64) ||
         !make_map(&mv64, v, D, g.Hkv, (long long)g.B * v_T, 1, 64))
         return HGA_ERR_CUDA;
-    const size_t smem = Cfg<D>::oEnd + 1024 + (size_t)a.cs_tokens * (D / 2) * sizeof(float2);
+    const size_t smem = Cfg<D>::oEnd + 1024 + (size_t)a.cs_tokens * (D / 2 + 1) * sizeof(float2);
     auto kern = k_attend_tc<D>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);

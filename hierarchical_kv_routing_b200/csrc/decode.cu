@@ -88,7 +88,7 @@ __device__ void close_chunk(const DecodeArgs &A, int b, int h, int c, int32_t po
             pm += (double)pj;
             const float x = to_f(ko[(int64_t)j * D + i]), y = to_f(ko[(int64_t)j * D + i + H]);
             if (hf) {
-                const float2 r = rope_cs(A.rope, (double)pj, i);
+                const float2 r = rope_cs_int(A.rope, pj, i);
                 const float2 rr = rot_pair(x, y, r);
                 a += (double)rr.x;
                 d2 += (double)rr.y;
@@ -121,7 +121,7 @@ __device__ __forceinline__ void load_queries(const DecodeArgs &A, int b, int h, 
     const T *qb = static_cast<const T *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
     for (int e = threadIdx.x; e < A.G * H; e += blockDim.x) {
         const int g = e / H, i = e % H;
-        const float2 r = rope_cs(A.rope, (double)pnew, i);
+        const float2 r = rope_cs_int(A.rope, pnew, i);
         const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
         qs[g * D + i] = (x * r.x - y * r.y) * A.scale_log2;
         qs[g * D + i + H] = (y * r.x + x * r.y) * A.scale_log2;
@@ -138,7 +138,7 @@ __device__ __forceinline__ void rotate_new_key(const DecodeArgs &A, int b, int h
         const int i = threadIdx.x;
         const T *kn = static_cast<const T *>(A.k_new) + ((int64_t)b * A.Hkv + h) * D;
         const float x = to_f(kn[i]), y = to_f(kn[i + H]);
-        const float2 r = rope_cs(A.rope, (double)pnew, i);
+        const float2 r = rope_cs_int(A.rope, pnew, i);
         const float2 rr = rot_pair(x, y, r);
         knew[i] = from_f<T>(rr.x);
         knew[i + H] = from_f<T>(rr.y);
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
         T *ko = static_cast<T *>(A.k_open) + (((int64_t)b * A.Hkv + h) * A.C + t % A.C) * D;
         for (int i = threadIdx.x; i < H; i += blockDim.x) {
             const float x = to_f(kn[i]), y = to_f(kn[i + H]);
-            const float2 r = rope_cs(A.rope, (double)pnew, i);
+            const float2 r = rope_cs_int(A.rope, pnew, i);
             const float2 rr = rot_pair(x, y, r);
             kr[i] = from_f<T>(rr.x);
             kr[i + H] = from_f<T>(rr.y);
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     // routing query of the token: the KV head's query heads summed, in fp64
     if (threadIdx.x < H) {
         const int i = threadIdx.x;
-        const float2 r = rope_cs(A.rope, (double)pnew, i);
+        const float2 r = rope_cs_int(A.rope, pnew, i);
         const T *qb = static_cast<const T *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
         double a = 0.0, d2 = 0.0;
 #pragma unroll

@@ -20,6 +20,7 @@ constexpr int kMaxHalf = 64;    // D/2 for D <= 128
 // parameter.
 struct Rope {
     double omega[kMaxHalf];
+    unsigned long long turn[kMaxHalf];  // round(omega_i / (2 pi) * 2^64): turns per position
     unsigned long long high;  // bit i set: pair i is high-frequency
     int half;                 // D / 2
 };
@@ -52,6 +53,20 @@ __device__ __forceinline__ float2 rope_cs(const Rope &r, double p, int i) {
     red = fma(-k, 2.4492935982947064e-16, red);                // 2 pi, low part
     float s, c;
     sincosf((float)red, &s, &c);
+    return make_float2(c, s);
+}
+
+// (cos, sin) of p * omega_i for an integer position p, without floating
+// point range reduction: the angle in turns, p * omega_i / (2 pi), is formed
+// modulo 1 in 64-bit fixed point (an integer product that wraps), its top 32
+// bits taken as a signed fraction of a half turn, and passed to sincospif.
+// The angle error is below pi * 2^-24 for |p| < 2^31, the same as rounding
+// the reduced angle to fp32.
+__device__ __forceinline__ float2 rope_cs_int(const Rope &r, int32_t p, int i) {
+    const unsigned long long u = (unsigned long long)(long long)p * r.turn[i];
+    const float x = (float)(int)(u >> 32) * 0x1p-31f;     // angle / pi in [-1, 1)
+    float s, c;
+    sincospif(x, &s, &c);
     return make_float2(c, s);
 }
 

@@ -83,10 +83,10 @@ k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int 
                     }
                 }
             }
-            const double pj = (double)pos[(int64_t)b * Tlen + t0 + j];
+            const int32_t pj = pos[(int64_t)b * Tlen + t0 + j];
 #pragma unroll
             for (int p = 0; p < PS; ++p) {
-                const float2 r = rope_cs(rope, pj, sl * PS + p);
+                const float2 r = rope_cs_int(rope, pj, sl * PS + p);
                 const float x = lo[p], y = hi[p];
                 lo[p] = x * r.x - y * r.y;
                 hi[p] = y * r.x + x * r.y;

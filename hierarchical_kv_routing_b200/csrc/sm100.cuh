@@ -232,6 +232,16 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Per-warpgroup register rebalancing (every warp of the warpgroup executes
+// the same one).  The shares must add up to no more than the block's launch
+// allocation, or an increase never completes.
+template <uint32_t N> __device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N> __device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Named barrier over a subset of warps (id 1..15; count = threads).
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

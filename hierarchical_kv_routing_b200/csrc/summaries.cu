@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
         if (pass == 0) {
             // while the keys are in flight: angles, mean positions, copies
             for (int e = threadIdx.x; e < n * H; e += kThreads)
-                cs[e] = rope_cs(A.rope, (double)pb[e / H], e % H);
+                cs[e] = rope_cs_int(A.rope, pb[e / H], e % H);
             if (closed && threadIdx.x <= gpc) {
                 const int g = threadIdx.x;
                 const int lo = g < gpc ? g * A.g_s : 0, cnt = g < gpc ? A.g_s : C;
@@ -163,41 +163,73 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
             }
         }
 
-        // one (head, pair) per thread: rotate in place, fp64 set sums
+        // one (head, pair) per thread: rotate in place, fp64 set sums with
+        // four independent accumulators (tokens j, j+1, j+2, j+3 in flight)
         for (int e = threadIdx.x; e < nh * H; e += kThreads) {
             const int hh = e / H, i = e % H;
             const int h = hs0 + hh;
             const bool hf = is_high(A.rope, i);
-            T *ko = (!closed && A.k_open)
-                ? static_cast<T *>(A.k_open) + ((int64_t)b * A.Hkv + h) * C * D : nullptr;
-            float *sg = A.s_group + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * gpc * D;
-            double gx = 0.0, gy = 0.0, cx = 0.0, cy = 0.0;
-            for (int j = 0; j < n; ++j) {
-                T *px = kb + ((size_t)j * nh + hh) * D + i;
-                const float x = to_f(px[0]), y = to_f(px[H]);
-                const float2 rr = rot_pair(x, y, cs[j * H + i]);
-                if (ko) {
-                    ko[(int64_t)j * D + i] = px[0];
-                    ko[(int64_t)j * D + i + H] = px[H];
+            T *col = kb + (size_t)hh * D + i;          // token j at col + j * js
+            const size_t js = (size_t)nh * D;
+            if (!closed) {
+                T *ko = A.k_open ? static_cast<T *>(A.k_open) + ((int64_t)b * A.Hkv + h) * C * D
+                                 : nullptr;
+                for (int j = 0; j < n; ++j) {
+                    T *px = col + j * js;
+                    const T x0 = px[0], y0 = px[H];
+                    const float2 rr = rot_pair(to_f(x0), to_f(y0), cs[j * H + i]);
+                    if (ko) {
+                        ko[(int64_t)j * D + i] = x0;
+                        ko[(int64_t)j * D + i + H] = y0;
+                    }
+                    px[0] = from_f<T>(rr.x);
+                    px[H] = from_f<T>(rr.y);
                 }
-                px[0] = from_f<T>(rr.x);
-                px[H] = from_f<T>(rr.y);
-                if (closed) {
-                    gx += (double)(hf ? rr.x : x);
-                    gy += (double)(hf ? rr.y : y);
-                    if ((j + 1) % A.g_s == 0) {
-                        const int set = j / A.g_s;
-                        write_summary(A.rope, hf, i, H, gx, gy, A.g_s, s_pmid[set],
-                                      sg + (int64_t)set * D);
-                        cx += gx;
-                        cy += gy;
-                        gx = gy = 0.0;
+                continue;
+            }
+            float *sg = A.s_group + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * gpc * D;
+            double cx = 0.0, cy = 0.0;
+            for (int set = 0; set < gpc; ++set) {
+                double ax[4] = {0.0, 0.0, 0.0, 0.0}, ay[4] = {0.0, 0.0, 0.0, 0.0};
+                const int j0 = set * A.g_s;
+                int jj = 0;
+                for (; jj + 4 <= A.g_s; jj += 4) {
+                    float x[4], y[4];
+                    float2 c4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const T *px = col + (j0 + jj + u) * js;
+                        x[u] = to_f(px[0]);
+                        y[u] = to_f(px[H]);
+                        c4[u] = cs[(j0 + jj + u) * H + i];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 rr = rot_pair(x[u], y[u], c4[u]);
+                        T *px = col + (j0 + jj + u) * js;
+                        px[0] = from_f<T>(rr.x);
+                        px[H] = from_f<T>(rr.y);
+                        ax[u] += (double)(hf ? rr.x : x[u]);
+                        ay[u] += (double)(hf ? rr.y : y[u]);
                     }
                 }
+                for (; jj < A.g_s; ++jj) {
+                    T *px = col + (j0 + jj) * js;
+                    const float x = to_f(px[0]), y = to_f(px[H]);
+                    const float2 rr = rot_pair(x, y, cs[(j0 + jj) * H + i]);
+                    px[0] = from_f<T>(rr.x);
+                    px[H] = from_f<T>(rr.y);
+                    ax[0] += (double)(hf ? rr.x : x);
+                    ay[0] += (double)(hf ? rr.y : y);
+                }
+                const double gx = (ax[0] + ax[1]) + (ax[2] + ax[3]);
+                const double gy = (ay[0] + ay[1]) + (ay[2] + ay[3]);
+                write_summary(A.rope, hf, i, H, gx, gy, A.g_s, s_pmid[set], sg + (int64_t)set * D);
+                cx += gx;
+                cy += gy;
             }
-            if (closed)
-                write_summary(A.rope, hf, i, H, cx, cy, C, s_pmid[gpc],
-                              A.s_chunk + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * D);
+            write_summary(A.rope, hf, i, H, cx, cy, C, s_pmid[gpc],
+                          A.s_chunk + (((int64_t)b * A.Hkv + h) * A.nc_cap + m) * D);
         }
         // rotated rows out
         if (A.k_rot) {

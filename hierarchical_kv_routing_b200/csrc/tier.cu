@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kGatherThreads) k_tier_gather(const GatherArgs
         const uint4 v0 = ld16(A.v_host + src + 8 * q), v1 = ld16(A.v_host + src + H + 8 * q);
         dv[q] = v0;
         dv[q + TPU] = v1;
-        const double p = (double)A.pos[(long long)b * A.T + tok];
+        const int32_t p = A.pos[(long long)b * A.T + tok];
         const __nv_bfloat162 *x2 = reinterpret_cast<const __nv_bfloat162 *>(&k0);
         const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&k1);
         uint4 o0, o1;
@@ -129,8 +129,8 @@ __global__ void __launch_bounds__(kGatherThreads) k_tier_gather(const GatherArgs
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 x = __bfloat1622float2(x2[e]), y = __bfloat1622float2(y2[e]);
-            const float2 r0 = rot_pair(x.x, y.x, rope_cs(A.rope, p, 8 * q + 2 * e));
-            const float2 r1 = rot_pair(x.y, y.y, rope_cs(A.rope, p, 8 * q + 2 * e + 1));
+            const float2 r0 = rot_pair(x.x, y.x, rope_cs_int(A.rope, p, 8 * q + 2 * e));
+            const float2 r1 = rot_pair(x.y, y.y, rope_cs_int(A.rope, p, 8 * q + 2 * e + 1));
             a2[e] = __floats2bfloat162_rn(r0.x, r1.x);
             c2[e] = __floats2bfloat162_rn(r0.y, r1.y);
         }
