@@ -8,14 +8,19 @@
 // and KV head is the block's RoPE-rotated queries summed over its tokens and
 // over the KV head's query heads.
 //
-// Design: one CTA per (block, KV head, sequence), HBM-bound on the Q stream.
-// Each thread sums its token's G query heads on a quarter of the pairs with
-// 16-byte loads (RoPE is linear, so heads are summed before rotating), the
-// rotated rows meet in shared memory and 128 threads reduce them over the
-// block's tokens in fp64.  Scores are fp64 dot products, one summary row per
-// thread (its 16-byte loads all in flight), ranked as packed (fp32 score, id)
-// keys; the top-K runs in registers (warp bitonic sort and merge) for K <= 32
-// and by CTA-wide rounds above that.
+// Design: one CTA per (run of up to 8 consecutive query blocks, KV head,
+// sequence).  Phase 1 streams the run's queries from HBM (the only large
+// read: every thread keeps one token's G head rows in flight as 16-byte
+// loads, sums the heads in fp32 (RoPE is linear), rotates, and accumulates
+// over tokens in fp64; warp shuffles and one shared-memory pass reduce over
+// tokens).  All of a run's CTAs stream at once, so the GPU's whole load
+// capacity works on Q.  Phase 2 reads each middle-chunk summary row once and
+// scores it against all the run's routing queries (fp64 dot products, the
+// query broadcast from shared memory), which cuts the chunk table's L2
+// traffic by the run length; one warp per block then takes its top K_c
+// (warp bitonic sort and merge of packed (fp32 score, id) keys), scores the
+// groups of its chunks and takes the top K_g.  K above 32 falls back to
+// CTA-wide selection rounds, one block at a time.
 #include "hga_internal.cuh"
 #include "route_common.cuh"
 
@@ -23,132 +28,242 @@ namespace hga {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kBlk = 8;                          // query blocks per CTA at most
+constexpr size_t kCandBytes = 160 * 1024;        // shared candidate table budget
+
+struct RouteArgs {
+    const void *q;
+    const int32_t *pos;
+    int T, Hq, Hkv, G, NB, F, L, K_c, K_g, gpc, nc_cap, nblk, ncap;
+    const float *s_chunk, *s_group;
+    int32_t *sel_chunk, *sel_group;
+    Rope rope;
+};
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-k_route(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, int Hq, int Hkv,
-        const float *__restrict__ s_chunk, const float *__restrict__ s_group, int nc_cap,
-        int F, int L, int K_c, int K_g, int gpc, int ncand, int32_t *__restrict__ sel_chunk,
-        int32_t *__restrict__ sel_group, Rope rope) {
-    constexpr int H = D / 2, PS = H / 4;
+__global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
+    constexpr int H = D / 2;
+    constexpr int EPW = 16 / (int)sizeof(T);     // elements per 16-byte word
+    constexpr int NS = H / EPW;                  // words per half row
+    constexpr int TP = kThreads / NS;            // tokens per pass
+    constexpr int HB = sizeof(T) == 2 ? 8 : 4;   // head rows in flight per thread
     extern __shared__ __align__(16) unsigned char smem[];
-    float *rot = reinterpret_cast<float *>(smem);                              // [64][D]
-    unsigned long long *cand = reinterpret_cast<unsigned long long *>(rot + kChunk * D);
-    __shared__ __align__(16) double qr[D];
+    double *qr = reinterpret_cast<double *>(smem);                            // [kBlk][D]
+    unsigned long long *cand = reinterpret_cast<unsigned long long *>(qr + kBlk * D);
+    __shared__ double part[kThreads / 32][D];
+    __shared__ int sel_s[kBlk][32];
+    __shared__ int kc_s[kBlk];
     __shared__ unsigned long long lists[kThreads];
     __shared__ RouteScratch rs;
 
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int NB = gridDim.x;
-    const int G = Hq / Hkv;
-    const int t0 = c * kChunk;
-    const int n = min(kChunk, Tlen - t0);
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int c0 = blockIdx.x * A.nblk;
+    const int nb = min(A.nblk, A.NB - c0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *q = static_cast<const T *>(A.q);
 
-    // ---- routing query: sum_i sum_{h'} R_{p_i}(q_{i,h'})
-    {
-        const int j = threadIdx.x >> 2, sl = threadIdx.x & 3;
-        float lo[PS], hi[PS];
+    // ---- phase 1: routing queries sum_i sum_{h'} R_{p_i}(q_{i,h'}), per block
+    const int w = threadIdx.x % NS, jt = threadIdx.x / NS;
+    for (int blk = 0; blk < nb; ++blk) {
+        const int t0 = (c0 + blk) * kChunk;
+        const int n = min(kChunk, A.T - t0);
+        double al[EPW], ah[EPW];
 #pragma unroll
-        for (int p = 0; p < PS; ++p) lo[p] = hi[p] = 0.f;
-        if (j < n) {
-            const T *row = q + (((int64_t)b * Tlen + t0 + j) * Hq + (int64_t)h * G) * D;
-            // several heads' rows in flight at a time, kept packed until summed
-            constexpr int kVec = PS * (int)sizeof(T) / 16;        // 16-byte words per half
-            constexpr int kBatch = sizeof(T) == 2 ? 4 : 2;
-            for (int h0 = 0; h0 < G; h0 += kBatch) {
-                uint4 wa[kBatch][kVec], wb[kBatch][kVec];
+        for (int e = 0; e < EPW; ++e) al[e] = ah[e] = 0.0;
+        for (int j = jt; j < n; j += TP) {
+            const T *row = q + (((int64_t)b * A.T + t0 + j) * A.Hq + (int64_t)h * A.G) * D;
+            float lo[EPW], hi[EPW];
 #pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    if (h0 + u < G) {
-                        const uint4 *pa = reinterpret_cast<const uint4 *>(row + (h0 + u) * D + sl * PS);
-                        const uint4 *pb = reinterpret_cast<const uint4 *>(row + (h0 + u) * D + H + sl * PS);
+            for (int e = 0; e < EPW; ++e) lo[e] = hi[e] = 0.f;
+            for (int g0 = 0; g0 < A.G; g0 += HB) {
+                uint4 wl[HB], wh[HB];
 #pragma unroll
-                        for (int v = 0; v < kVec; ++v) {
-                            wa[u][v] = __ldg(pa + v);
-                            wb[u][v] = __ldg(pb + v);
+                for (int u = 0; u < HB; ++u)
+                    if (g0 + u < A.G) {
+                        wl[u] = __ldg(reinterpret_cast<const uint4 *>(row + (g0 + u) * D) + w);
+                        wh[u] = __ldg(reinterpret_cast<const uint4 *>(row + (g0 + u) * D + H) + w);
+                    }
+#pragma unroll
+                for (int u = 0; u < HB; ++u)
+                    if (g0 + u < A.G) {
+                        float a[EPW], c[EPW];
+                        unpack_words<T, EPW>(reinterpret_cast<const uint4(&)[1]>(wl[u]), a);
+                        unpack_words<T, EPW>(reinterpret_cast<const uint4(&)[1]>(wh[u]), c);
+#pragma unroll
+                        for (int e = 0; e < EPW; ++e) {
+                            lo[e] += a[e];
+                            hi[e] += c[e];
                         }
                     }
-                }
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    if (h0 + u < G) {
-                        float a[PS], d2[PS];
-                        unpack_words<T, PS>(wa[u], a);
-                        unpack_words<T, PS>(wb[u], d2);
-#pragma unroll
-                        for (int p = 0; p < PS; ++p) {
-                            lo[p] += a[p];
-                            hi[p] += d2[p];
-                        }
-                    }
-                }
             }
-            const int32_t pj = pos[(int64_t)b * Tlen + t0 + j];
+            const int32_t p = A.pos[(int64_t)b * A.T + t0 + j];
 #pragma unroll
-            for (int p = 0; p < PS; ++p) {
-                const float2 r = rope_cs_int(rope, pj, sl * PS + p);
-                const float x = lo[p], y = hi[p];
-                lo[p] = x * r.x - y * r.y;
-                hi[p] = y * r.x + x * r.y;
+            for (int e = 0; e < EPW; ++e) {
+                const float2 rr = rot_pair(lo[e], hi[e], rope_cs_int(A.rope, p, w * EPW + e));
+                al[e] += (double)rr.x;
+                ah[e] += (double)rr.y;
             }
         }
+        // lanes holding the same word: reduce over their tokens
 #pragma unroll
-        for (int p = 0; p < PS; ++p) {
-            rot[j * D + sl * PS + p] = lo[p];
-            rot[j * D + H + sl * PS + p] = hi[p];
-        }
+        for (int off = NS; off < 32; off <<= 1)
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) {
+                al[e] += __shfl_xor_sync(0xffffffffu, al[e], off);
+                ah[e] += __shfl_xor_sync(0xffffffffu, ah[e], off);
+            }
+        if (lane < NS)
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) {
+                part[warp][w * EPW + e] = al[e];
+                part[warp][H + w * EPW + e] = ah[e];
+            }
         __syncthreads();
         if (threadIdx.x < D) {
-            double s = 0.0;
-            for (int jj = 0; jj < n; ++jj) s += (double)rot[jj * D + threadIdx.x];
-            qr[threadIdx.x] = s;
+            double sum = 0.0;
+#pragma unroll
+            for (int wp = 0; wp < kThreads / 32; ++wp) sum += part[wp][threadIdx.x];
+            qr[blk * D + threadIdx.x] = sum;
         }
         __syncthreads();
     }
 
-    // ---- chunk level: middle chunks F..hi, top K_c
-    const int hi_m = middle_hi(c, L);
-    const int n_mid = max(0, hi_m - F + 1);
-    const float *Sc = s_chunk + ((int64_t)b * Hkv + h) * nc_cap * D;
-    for (int r = threadIdx.x; r < n_mid; r += kThreads)
-        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sc + (int64_t)(F + r) * D), F + r);
-    __syncthreads();
-    const int kc = min(K_c, n_mid);
-    if (K_c <= 32) block_topk32(cand, n_mid, K_c, rs.sel_c, lists);
-    else topk_select(cand, n_mid, K_c, rs.sel_c, rs);
-    int32_t *out_c = sel_chunk + (((int64_t)b * NB + c) * Hkv + h) * K_c;
-    for (int r = threadIdx.x; r < K_c; r += kThreads) out_c[r] = r < kc ? rs.sel_c[r] : -1;
-
-    // ---- group level: the groups of the selected chunks, top K_g
-    const float *Sg = s_group + ((int64_t)b * Hkv + h) * nc_cap * gpc * D;
-    const int n_g = kc * gpc;
-    __syncthreads();
-    for (int r = threadIdx.x; r < n_g; r += kThreads) {
-        const int gid = rs.sel_c[r / gpc] * gpc + r % gpc;
-        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sg + (int64_t)gid * D), gid);
+    // ---- phase 2: chunk scores for every block of the run, one row read once
+    const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
+    const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
+    const int n_rows = max(0, middle_hi(c0 + nb - 1, A.L) - A.F + 1);
+    for (int r = threadIdx.x; r < n_rows; r += kThreads) {
+        const float4 *r4 = reinterpret_cast<const float4 *>(Sc + (int64_t)(A.F + r) * D);
+        double acc[kBlk];
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k) acc[k] = 0.0;
+#pragma unroll 1
+        for (int base = 0; base < D / 4; base += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __ldg(r4 + base + e);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int d = 4 * (base + e);
+#pragma unroll
+                for (int k = 0; k < kBlk; ++k) {
+                    if (k < nb) {
+                        const double *qk = qr + k * D + d;
+                        acc[k] = fma(qk[0], (double)v[e].x, acc[k]);
+                        acc[k] = fma(qk[1], (double)v[e].y, acc[k]);
+                        acc[k] = fma(qk[2], (double)v[e].z, acc[k]);
+                        acc[k] = fma(qk[3], (double)v[e].w, acc[k]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kBlk; ++k)
+            if (k < nb)
+                cand[k * A.ncap + r] = A.F + r <= middle_hi(c0 + k, A.L)
+                                           ? pack_key((float)acc[k], A.F + r) : 0ull;
     }
     __syncthreads();
-    const int kg = min(K_g, n_g);
-    if (K_g <= 32) block_topk32(cand, n_g, K_g, rs.sel_g, lists);
-    else topk_select(cand, n_g, K_g, rs.sel_g, rs);
-    int32_t *out_g = sel_group + (((int64_t)b * NB + c) * Hkv + h) * K_g;
-    for (int r = threadIdx.x; r < K_g; r += kThreads) out_g[r] = r < kg ? rs.sel_g[r] : -1;
+
+    if (A.K_c <= 32 && A.K_g <= 32) {
+        // one warp per block: top K_c chunks, then its groups and top K_g
+        for (int k = warp; k < nb; k += kThreads / 32) {
+            const int c = c0 + k;
+            const int n_mid = max(0, middle_hi(c, A.L) - A.F + 1);
+            const unsigned long long top = warp_top32(cand + k * A.ncap, n_mid, 0, 1);
+            const bool take = lane < A.K_c && top != 0ull;
+            const int id = warp_sort_asc_int(take ? key_id(top) : 0x7fffffff);
+            const int kc = min(A.K_c, n_mid);
+            sel_s[k][lane] = id;
+            int32_t *oc = A.sel_chunk + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_c;
+            if (lane < A.K_c) oc[lane] = lane < kc ? id : -1;
+            if (lane == 0) kc_s[k] = kc;
+        }
+        __syncthreads();
+        // group candidates of every block at once (the chunk table is free)
+        const int slots = A.K_c * A.gpc;
+        for (int x = threadIdx.x; x < nb * slots; x += kThreads) {
+            const int k = x / slots, r = x % slots;
+            if (r < kc_s[k] * A.gpc) {
+                const int gid = sel_s[k][r / A.gpc] * A.gpc + r % A.gpc;
+                cand[k * A.ncap + r] =
+                    pack_key((float)thread_dot_row<D>(qr + k * D, Sg + (int64_t)gid * D), gid);
+            }
+        }
+        __syncthreads();
+        for (int k = warp; k < nb; k += kThreads / 32) {
+            const int c = c0 + k;
+            const int ng = kc_s[k] * A.gpc;
+            const unsigned long long top = warp_top32(cand + k * A.ncap, ng, 0, 1);
+            const bool take = lane < A.K_g && top != 0ull;
+            const int id = warp_sort_asc_int(take ? key_id(top) : 0x7fffffff);
+            const int kg = min(A.K_g, ng);
+            int32_t *og = A.sel_group + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_g;
+            if (lane < A.K_g) og[lane] = lane < kg ? id : -1;
+        }
+        return;
+    }
+
+    // K above 32: CTA-wide selection rounds, one block at a time
+    for (int k = 0; k < nb; ++k) {
+        const int c = c0 + k;
+        const int n_mid = max(0, middle_hi(c, A.L) - A.F + 1);
+        unsigned long long *ck = cand + k * A.ncap;
+        const int kc = min(A.K_c, n_mid);
+        if (A.K_c <= 32) block_topk32(ck, n_mid, A.K_c, rs.sel_c, lists);
+        else topk_select(ck, n_mid, A.K_c, rs.sel_c, rs);
+        int32_t *oc = A.sel_chunk + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_c;
+        for (int r = threadIdx.x; r < A.K_c; r += kThreads) oc[r] = r < kc ? rs.sel_c[r] : -1;
+        __syncthreads();
+        const int ng = kc * A.gpc;
+        for (int r = threadIdx.x; r < ng; r += kThreads) {
+            const int gid = rs.sel_c[r / A.gpc] * A.gpc + r % A.gpc;
+            ck[r] = pack_key((float)thread_dot_row<D>(qr + k * D, Sg + (int64_t)gid * D), gid);
+        }
+        __syncthreads();
+        const int kg = min(A.K_g, ng);
+        if (A.K_g <= 32) block_topk32(ck, ng, A.K_g, rs.sel_g, lists);
+        else topk_select(ck, ng, A.K_g, rs.sel_g, rs);
+        int32_t *og = A.sel_group + (((int64_t)b * A.NB + c) * A.Hkv + h) * A.K_g;
+        for (int r = threadIdx.x; r < A.K_g; r += kThreads) og[r] = r < kg ? rs.sel_g[r] : -1;
+        __syncthreads();
+    }
 }
 
 template <typename T, int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                const float *s_chunk, const float *s_group, int nc_cap, int32_t *sel_chunk,
                int32_t *sel_group, cudaStream_t st) {
-    const long long ncand = max(max((long long)g.NC, 1ll), (long long)min(g.K_c, g.NC) * g.gpc);
-    const size_t smem = sizeof(float) * kChunk * D + sizeof(unsigned long long) * (size_t)ncand;
-    if (smem > 180 * 1024) return HGA_ERR_UNSUPPORTED;   // candidate table must fit on chip
+    RouteArgs a;
+    a.q = q;
+    a.pos = pos;
+    a.T = g.T;
+    a.Hq = g.Hq;
+    a.Hkv = g.Hkv;
+    a.G = g.G;
+    a.NB = g.NB;
+    a.F = g.F;
+    a.L = g.L;
+    a.K_c = g.K_c;
+    a.K_g = g.K_g;
+    a.gpc = g.gpc;
+    a.nc_cap = nc_cap;
+    // candidate rows per block: middle chunks, or the selected chunks' groups
+    a.ncap = (int)max(max((long long)g.NC, 1ll), (long long)min(g.K_c, g.NC) * g.gpc);
+    const size_t row_bytes = sizeof(unsigned long long) * (size_t)a.ncap;
+    if (row_bytes > kCandBytes) return HGA_ERR_UNSUPPORTED;   // must fit on chip
+    a.nblk = (int)min((size_t)kBlk, kCandBytes / row_bytes);
+    a.s_chunk = s_chunk;
+    a.s_group = s_group;
+    a.sel_chunk = sel_chunk;
+    a.sel_group = sel_group;
+    a.rope = r;
+    const size_t smem = sizeof(double) * kBlk * D + row_bytes * a.nblk;
     auto kern = k_route<T, D>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
-    dim3 grid(g.NB, g.Hkv, g.B);
-    kern<<<grid, kThreads, smem, st>>>(static_cast<const T *>(q), pos, g.T, g.Hq, g.Hkv, s_chunk,
-                                       s_group, nc_cap, g.F, g.L, g.K_c, g.K_g, g.gpc,
-                                       (int)ncand, sel_chunk, sel_group, r);
+    dim3 grid((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
+    kern<<<grid, kThreads, smem, st>>>(a);
     return cuda_status(cudaGetLastError());
 }
 

@@ -228,8 +228,9 @@ namespace hga {
 // (the whole row streams through this thread's 16-byte loads).
 template <int D>
 __device__ __forceinline__ double thread_dot_row(const double *qr, const float *__restrict__ row) {
-    // 16 loads in flight per batch: enough to cover latency, few registers
-    constexpr int kBatch = 16;
+    // 8 loads in flight per batch: several rows per thread and CTAs per SM
+    // cover the latency, and the routers stay within 80 registers
+    constexpr int kBatch = 8;
     const float4 *r4 = reinterpret_cast<const float4 *>(row);
     const double2 *q2 = reinterpret_cast<const double2 *>(qr);
     double s0 = 0.0, s1 = 0.0;
