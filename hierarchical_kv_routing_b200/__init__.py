@@ -24,7 +24,7 @@ __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "h
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
            "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
            "decode_workspace", "hga_forward_prefill_hostkv", "HGAError", "PREFILL",
-           "DECODE", "PREFILL_HOSTKV"]
+           "DECODE", "PREFILL_HOSTKV", "hga_device_status"]
 
 PREFILL, DECODE, PREFILL_HOSTKV = 0, 1, 2
 _F32, _BF16 = 0, 1
@@ -111,6 +111,8 @@ def load():
         lib.hga_status_string.argtypes = [ctypes.c_int]
         lib.hga_status_string.restype = ctypes.c_char_p
         lib.hga_last_cuda_error.restype = ctypes.c_int
+        lib.hga_device_status.argtypes = [P, ctypes.c_int]
+        lib.hga_device_status.restype = ctypes.c_int
         for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -235,6 +237,14 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
                         _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "hga_attend")
     return (out, lse) if want_lse or lse is not None else out
+
+
+def hga_device_status(clear: bool = True, stream=None) -> int:
+    """The status the kernels recorded on the device since the last reset
+    (0 = none; 4 = a bounded wait timed out; 5 = a bounds check refused an
+    access).  Waits for the work queued on `stream`."""
+    lib = load()
+    return int(lib.hga_device_status(_stream(stream), 1 if clear else 0))
 
 
 def hga_workspace_size(mode: int, B: int, T: int, Hq: int, Hkv: int, D: int, dtype,

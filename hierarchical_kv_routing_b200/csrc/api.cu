@@ -280,4 +280,15 @@ const char *hga_status_string(hga_status s) {
 
 int hga_last_cuda_error(void) { return g_last_cuda_error; }
 
+hga_status hga_device_status(void *stream, int clear) {
+    const cudaStream_t st = (cudaStream_t)stream;
+    hga_status first = HGA_OK;
+    const hga_status parts[3] = {summaries_error_take(st, clear != 0),
+                                 attend_tc_error_take(st, clear != 0),
+                                 decode_error_take(st, clear != 0)};
+    for (hga_status p : parts)
+        if (p != HGA_OK && first == HGA_OK) first = p;
+    return first;
+}
+
 }  // extern "C"

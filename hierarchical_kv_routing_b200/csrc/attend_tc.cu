@@ -605,4 +605,20 @@ hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const in
                       : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw);
 }
 
+
+// Reads this file's device error word on `st` (after the work queued on it)
+// and optionally resets it; returns the recorded status (HGA_OK if none).
+hga_status attend_tc_error_take(cudaStream_t st, bool clear) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_attend_tc_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear && v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_attend_tc_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return cuda_status(e);
+    return (hga_status)v;
+}
+
 }  // namespace hga

@@ -663,4 +663,20 @@ hga_status launch_decode(const Geo &g, const Rope &r, int dtype, const hga_io &i
     return g.D == 128 ? run<float, 128>(g, r, io, ws, st) : run<float, 64>(g, r, io, ws, st);
 }
 
+
+// Reads this file's device error word on `st` (after the work queued on it)
+// and optionally resets it; returns the recorded status (HGA_OK if none).
+hga_status decode_error_take(cudaStream_t st, bool clear) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_decode_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear && v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_decode_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return cuda_status(e);
+    return (hga_status)v;
+}
+
 }  // namespace hga

@@ -165,6 +165,12 @@ size_t hostkv_workspace_bytes(const Geo &g);
 hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, void *ws,
                                  cudaStream_t st);
 
+// Device error words (bounded-wait timeouts, bounds checks) of each kernel
+// file: read on a stream after its queued work, optionally reset.
+hga_status attend_tc_error_take(cudaStream_t st, bool clear);
+hga_status decode_error_take(cudaStream_t st, bool clear);
+hga_status summaries_error_take(cudaStream_t st, bool clear);
+
 // Decode step (append, close-chunk summaries, route, split attention).
 size_t decode_workspace_bytes(const Geo &g);
 hga_status launch_decode(const Geo &g, const Rope &r, int dtype, const hga_io &io, void *ws,

@@ -302,4 +302,20 @@ hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *
     return g.D == 128 ? run<float, 128, false>(g, a, in_T, st) : run<float, 64, false>(g, a, in_T, st);
 }
 
+
+// Reads this file's device error word on `st` (after the work queued on it)
+// and optionally resets it; returns the recorded status (HGA_OK if none).
+hga_status summaries_error_take(cudaStream_t st, bool clear) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_summaries_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear && v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_summaries_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return cuda_status(e);
+    return (hga_status)v;
+}
+
 }  // namespace hga

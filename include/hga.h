@@ -228,6 +228,18 @@ hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hga_params *p
                                        const void *q, const void *k, const void *v,
                                        const int32_t *pos, void *out, float *lse, void *stream);
 
+/* Status recorded by the kernels themselves since the last reset: a bounded
+ * wait that gave up (HGA_ERR_TIMEOUT: the kernel recorded it, released what
+ * it held and returned without finishing its tile) or a device-side index
+ * check that refused an access (HGA_ERR_BOUNDS, e.g. a decode step for a
+ * sequence whose lens[b] is outside [0, capacity); that sequence is skipped,
+ * the others proceed).  Kernels never trap: a launch that met such a
+ * condition still completes, and only this call reports it.  Waits for the
+ * work already queued on `stream`, then reads the library's error words;
+ * clear != 0 resets them.  Returns HGA_OK when none is set, the first set
+ * status otherwise, or HGA_ERR_CUDA if the copies fail. */
+hga_status hga_device_status(void *stream, int clear);
+
 /* Static description of a status code. */
 const char *hga_status_string(hga_status s);
 

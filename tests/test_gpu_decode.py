@@ -197,3 +197,35 @@ def test_decode_64k_full_size_graph(gpu_lib):
             assert e <= tol, f"decode output rel err {e} at b={b} step={s}"
         S_c, _ = oracle.build_summaries(K, pos, p)
         assert row_rel_err(_np(cache.s_chunk[b:b + 1]), S_c) < 2e-6
+
+
+def test_decode_bounds_status_is_recorded(gpu_lib):
+    """A sequence whose cache is already full is refused by the kernels' own
+    index checks (before any access): the step leaves it untouched, records
+    HGA_ERR_BOUNDS for hga_device_status, and the other sequences are served
+    exactly as in a step without it."""
+    w = QWEN.replace(B=2, Hq=8, Hkv=2)
+    T_hist, cap = 640, 704
+    d = make_decode_inputs(w, seed=3, T=T_hist, steps=1)
+    dev = torch.device("cuda")
+    hga = gpu_lib
+    hp = _hp(hga, w)
+    dt = d["k_hist"].dtype
+    caches = []
+    for _ in range(2):
+        c = hga.KVCache(w.B, cap, w.Hkv, w.D, dt, hp, device=dev)
+        hga.hga_fill_cache(d["k_hist"].to(dev), d["v_hist"].to(dev), d["pos_hist"].to(dev), c, hp)
+        caches.append(c)
+    assert hga.hga_device_status(clear=True) == 0
+    caches[1].lens[0] = cap            # sequence 0 of the second cache: no room left
+    args = (d["q"][0].to(dev), d["k_new"][0].to(dev), d["v_new"][0].to(dev),
+            d["pos_new"][0].to(dev))
+    good = hga.hga_forward_decode(*args, caches[0], hp)
+    assert hga.hga_device_status(clear=True) == 0
+    bad = hga.hga_forward_decode(*args, caches[1], hp)
+    assert hga.hga_device_status(clear=False) == 5          # HGA_ERR_BOUNDS
+    assert hga.hga_device_status(clear=True) == 5
+    assert hga.hga_device_status(clear=True) == 0           # reset
+    torch.cuda.synchronize()
+    assert int(caches[1].lens[0]) == cap and int(caches[1].lens[1]) == T_hist + 1
+    assert torch.equal(good["out"][1].view(torch.int16), bad["out"][1].view(torch.int16))

@@ -130,3 +130,22 @@ def test_qwen_32k_full_size(gpu_lib):
     NB = w.T // 64
     blocks = list(range(0, w.F + w.L + 2)) + list(range(40, NB, 61)) + [NB - 1]
     run_and_check(gpu_lib, w, seed=11, units=[(0, u) for u in blocks])
+
+
+def test_exact_token_chunk_variant(gpu_lib):
+    """The exact-token chunk variant (groups off: every group of each routed
+    chunk opened, page section 3, routing policy) is K_g = K_c * C / g_s: the
+    routed groups are exactly the groups of the routed chunks, and outputs
+    match the oracle."""
+    w = QWEN.replace(T=64 * 40 + 17, K_c=6, K_g=6 * 4)
+    run_and_check(gpu_lib, w, seed=21)
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=21)
+    dev = torch.device("cuda")
+    res = gpu_lib.hga_forward_prefill(*(x.to(dev) for x in (q, k, v, pos)), _hp(w), want_sel=True)
+    sc, sg = res["sel_chunk"].cpu().numpy(), res["sel_group"].cpu().numpy()
+    gpc = w.C // w.g_s
+    for blk in range(sc.shape[1]):
+        for h in range(w.Hkv):
+            chunks = sc[0, blk, h][sc[0, blk, h] >= 0]
+            groups = sg[0, blk, h][sg[0, blk, h] >= 0]
+            assert sorted(groups.tolist()) == sorted((chunks[:, None] * gpc + np.arange(gpc)).ravel().tolist())
