@@ -12,18 +12,20 @@
 // routing does not touch (sinks, recent chunks, the current chunk) and the
 // routed groups, so the first kernel attends over the fixed part while it
 // routes, and the second only has to add the routed groups.
-//   k_decode_a  grid (scan splits + fixed splits, KV heads, sequences)
-//     scan CTAs   split 0 appends the token (rotated key, value, position,
-//                 raw key of the open chunk) and, when the token closes its
-//                 chunk, writes that chunk's summaries.  Each scan CTA scores
-//                 256 middle chunks, one summary row per thread (fp64 dot
-//                 products), and keeps its top K_c keys; the last one to
-//                 finish (atomic counter) merges them, scores the groups of the
-//                 chosen chunks and keeps the top K_g.
-//     fixed CTAs  attend the KV head's G query heads over a slice of the fixed
-//                 keys (the new token's key and value straight from the step's
-//                 inputs, everything else from the cache) and write partial
-//                 softmax sums.
+//   k_decode_a  grid (max(scan splits, fixed splits), KV heads, sequences);
+//               each CTA takes one slice of both jobs, so the whole grid is
+//               resident at once (one wave):
+//     fixed keys  CTA s < 4 attends the KV head's G query heads over a slice
+//                 of the fixed keys (the new token's key and value straight
+//                 from the step's inputs, everything else from the cache) and
+//                 writes partial softmax sums;
+//     scan        CTA s < scan splits: split 0 appends the token (rotated key,
+//                 value, position, raw key of the open chunk) and, when the
+//                 token closes its chunk, writes that chunk's summaries.  Each
+//                 scores its 256 middle chunks, one summary row per thread
+//                 (fp64 dot products), and keeps its top K_c keys; the last one
+//                 to finish (atomic counter) merges them, scores the groups of
+//                 the chosen chunks and keeps the top K_g.
 //   k_decode_b  grid (routed splits, KV heads, sequences), launched as a
 //               programmatic dependent of k_decode_a: it rotates the queries,
 //               then waits for k_decode_a, attends over a slice of the routed
@@ -219,29 +221,37 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int k = threadIdx.x; k < nk; k += blockDim.x) kt_s[k] = key_of(k);
     __syncthreads();
+    // Every thread handles at most one key (nk * tpk <= blockDim): its key
+    // row's loads go out first, then the value rows' asynchronous copies, and
+    // only then does the thread wait on its key row for the dot products.
+    const int tpk = nk <= (int)blockDim.x / 2 ? 2 : 1;
+    const int gper = (A.G + tpk - 1) / tpk;
+    const int kk = threadIdx.x / tpk, part = threadIdx.x % tpk;
+    const bool has_key = kk < nk;
+    const int kt = has_key ? kt_s[kk] : 0;
+    uint4 kw[NV];
+    if (has_key) {
+        if (kt == t) {
+#pragma unroll
+            for (int e = 0; e < NV; ++e) kw[e] = reinterpret_cast<const uint4 *>(knew)[e];
+        } else {
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                static_cast<const T *>(A.k_rot) + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D);
+#pragma unroll
+            for (int e = 0; e < NV; ++e) kw[e] = __ldg(src + e);
+        }
+    }
     const T *vbase = static_cast<const T *>(A.v);
     const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
     for (int idx = threadIdx.x; idx < nk * NV; idx += blockDim.x) {
-        const int k = idx / NV, part = idx % NV;
-        const int kt = kt_s[k];
-        const T *src = kt == t ? vn : vbase + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D;
-        cp_async16(reinterpret_cast<uint4 *>(Vs + (size_t)k * D) + part,
-                   reinterpret_cast<const uint4 *>(src) + part);
+        const int k = idx / NV, pv = idx % NV;
+        const int kv = kt_s[k];
+        const T *src = kv == t ? vn : vbase + (((int64_t)b * A.Tc + kv) * A.Hkv + h) * D;
+        cp_async16(reinterpret_cast<uint4 *>(Vs + (size_t)k * D) + pv,
+                   reinterpret_cast<const uint4 *>(src) + pv);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    // two threads per key (each half of the heads) when the slice is short
-    const int tpk = nk <= (int)blockDim.x / 2 ? 2 : 1;
-    const int gper = (A.G + tpk - 1) / tpk;
-    for (int idx = threadIdx.x; idx < nk * tpk; idx += blockDim.x) {
-        const int k = idx / tpk, part = idx % tpk;
-        const int kt = kt_s[k];
-        const uint4 *src = kt == t
-            ? reinterpret_cast<const uint4 *>(knew)
-            : reinterpret_cast<const uint4 *>(static_cast<const T *>(A.k_rot) +
-                                              (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D);
-        uint4 kw[NV];
-#pragma unroll
-        for (int e = 0; e < NV; ++e) kw[e] = kt == t ? src[e] : __ldg(src + e);
+    if (has_key) {
         const int g1 = min(A.G, (part + 1) * gper);
 #pragma unroll 1
         for (int g = part * gper; g < g1; ++g) {
@@ -252,7 +262,7 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
                 a0 += dot16<T>(kw[e], qg + e * EV);
                 a1 += dot16<T>(kw[e + 1], qg + (e + 1) * EV);
             }
-            sc[g * kThreads + k] = a0 + a1;
+            sc[g * kThreads + kk] = a0 + a1;
         }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -293,8 +303,8 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
     }
 }
 
-// Shared memory of k_decode_a: the scan and fixed-attention roles never meet
-// in one CTA, so their buffers share one pool.
+// Shared memory of k_decode_a: a CTA runs its fixed-key attention first and
+// its scan afterwards, so the two jobs' buffers share one pool.
 template <typename T, int D>
 struct ScanSmem {
     double qr[D];
@@ -340,9 +350,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     const int c = t / A.C;
     const int32_t pnew = A.pos_new[b];
 
-    if (s >= A.ns_scan) {
+    if (s < kFixSplits) {
         // ------------------------------------------- fixed-key attention --
-        const int f = s - A.ns_scan;
+        const int f = s;
         const int nsink = min(A.F, c);
         const int rec_lo = max(c - max(A.L, 1), nsink);
         const int n1 = nsink * A.C, n2 = n1 + (c - rec_lo) * A.C;
@@ -357,7 +367,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
             return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
         };
         attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
-        // this CTA is done: the routed-keys kernel may start launching
+        __syncthreads();          // the scan below reuses the shared pool
+    }
+    if (s >= A.ns_scan) {
+        // no chunk rows for this CTA: the routed-keys kernel may start launching
         asm volatile("griddepcontrol.launch_dependents;");
         return;
     }
@@ -519,19 +532,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
     for (int g = warp; g < A.G; g += nw) {
         const float *src = part_b + (int64_t)g * kParts * (D + 2);
+        // every partial's (m, l, o slice) in one round trip to L2
+        float ms[kParts], ls[kParts], vs[kParts][DL];
+#pragma unroll
+        for (int sp = 0; sp < kParts; ++sp) {
+            ms[sp] = __ldcg(src + sp * (D + 2));
+            ls[sp] = __ldcg(src + sp * (D + 2) + 1);
+#pragma unroll
+            for (int e = 0; e < DL; ++e) vs[sp][e] = __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
+        }
         float M = -INFINITY;
-        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, __ldcg(src + sp * (D + 2)));
+#pragma unroll
+        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, ms[sp]);
         float L = 0.f, acc[DL];
 #pragma unroll
         for (int e = 0; e < DL; ++e) acc[e] = 0.f;
-        for (int sp = 0; sp < kParts; ++sp) {
-            const float ms = __ldcg(src + sp * (D + 2));
-            if (ms == -INFINITY) continue;
-            const float w = exp2f(ms - M);
-            L += w * __ldcg(src + sp * (D + 2) + 1);
 #pragma unroll
-            for (int e = 0; e < DL; ++e)
-                acc[e] += w * __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
+        for (int sp = 0; sp < kParts; ++sp) {
+            const float w = ms[sp] == -INFINITY ? 0.f : exp2f(ms[sp] - M);
+            L += w * ls[sp];
+#pragma unroll
+            for (int e = 0; e < DL; ++e) acc[e] += w * vs[sp][e];
         }
         const float inv = 1.f / L;
         T *o = static_cast<T *>(A.out) + ((int64_t)b * A.Hq + (int64_t)h * A.G + g) * D;
@@ -556,10 +577,17 @@ struct Ws {
     size_t counters, cand, sel_c, sel_g, part, total;
 };
 
+// Scan CTAs: scan CTA s holds middle chunks [256 s, 256 s + 256); the highest
+// middle chunk a step can have is nc - L - 2 (nc - 3 with L = 0).
+int scan_splits(const Geo &g) {
+    const int nc = g.T / g.C;
+    return max(0, nc - 2 - g.L) / kScanChunks + 1;
+}
+
 inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 Ws layout(const Geo &g) {
-    const int ns = ((g.T / g.C) + kScanChunks - 1) / kScanChunks;
+    const int ns = scan_splits(g);
     Ws w;
     size_t o = 0;
     w.counters = o;
@@ -594,7 +622,7 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.K_c = g.K_c;
     A.K_g = g.K_g;
     A.nc_cap = g.T / g.C;
-    A.ns_scan = (A.nc_cap + kScanChunks - 1) / kScanChunks;
+    A.ns_scan = scan_splits(g);
     A.q_new = io.q_new;
     A.k_new = io.k_new;
     A.v_new = io.v_new;
@@ -623,7 +651,7 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     cudaError_t e = ensure_smem((const void *)k_decode_a<T, D>, vs_bytes);
     if (e == cudaSuccess) e = ensure_smem((const void *)k_decode_b<T, D>, vs_bytes);
     if (e != cudaSuccess) return cuda_status(e);
-    k_decode_a<T, D><<<dim3(A.ns_scan + kFixSplits, g.Hkv, g.B), kThreads, vs_bytes, st>>>(A);
+    k_decode_a<T, D><<<dim3(max(A.ns_scan, kFixSplits), g.Hkv, g.B), kThreads, vs_bytes, st>>>(A);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg = {};
@@ -645,7 +673,7 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
 // Shapes the fixed-size tables hold: per CTA at most kThreads keys, the
 // merge and group candidates fit kMaxCand.
 bool decode_supported(const Geo &g) {
-    const long long ns = ((g.T / g.C) + kScanChunks - 1) / kScanChunks;
+    const long long ns = scan_splits(g);
     const long long routed = min((long long)g.K_g * g.g_s, (long long)g.T);
     return g.G <= kMaxG && ns * g.K_c <= kMaxCand && (long long)g.K_c * g.gpc <= kMaxCand &&
            routed <= (long long)kRouteSplits * kThreads &&
