@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
     T *kb = reinterpret_cast<T *>(smem);                          // [n][nh][D]
     float2 *cs = reinterpret_cast<float2 *>(smem + kSlabBytes);   // [n][H]
     __shared__ double s_pmid[C + 1];
+    __shared__ int32_t s_pos[C];
     __shared__ __align__(8) uint64_t bar;
 
     const int m = blockIdx.x, b = blockIdx.y;
@@ -93,6 +94,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
         mbar_init(&bar, 1);
         fence_barrier_init();
     }
+    // the chunk's positions, one coalesced load
+    if (threadIdx.x < n) s_pos[threadIdx.x] = pb[threadIdx.x];
     __syncthreads();
 
     int pass = 0;
@@ -134,17 +137,28 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
         if (pass == 0) {
             // while the keys are in flight: angles, mean positions, copies
             for (int e = threadIdx.x; e < n * H; e += kThreads)
-                cs[e] = rope_cs_int(A.rope, pb[e / H], e % H);
-            if (closed && threadIdx.x <= gpc) {
-                const int g = threadIdx.x;
-                const int lo = g < gpc ? g * A.g_s : 0, cnt = g < gpc ? A.g_s : C;
-                double acc = 0.0;
-                for (int j = 0; j < cnt; ++j) acc += (double)pb[lo + j];
-                s_pmid[g] = acc / (double)cnt;
+                cs[e] = rope_cs_int(A.rope, s_pos[e / H], e % H);
+            if (closed && threadIdx.x < 32) {
+                // mean positions: lane l holds positions l and l + 32 (64-bit
+                // sums are exact); each set is a run of lanes
+                const int l = threadIdx.x;
+                const long long p0 = s_pos[l], p1 = s_pos[l + 32];
+                long long tot = p0 + p1;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                if (l == 0) s_pmid[gpc] = (double)tot / (double)C;
+                for (int g = 0; g < gpc; ++g) {
+                    const int lo = g * A.g_s;
+                    long long part = 0;
+                    for (int j = l; j < A.g_s; j += 32) part += s_pos[lo + j];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                    if (l == 0) s_pmid[g] = (double)part / (double)A.g_s;
+                }
             }
             if (A.pos_out)
                 for (int j = threadIdx.x; j < n; j += kThreads)
-                    A.pos_out[(int64_t)b * A.out_T + t0 + j] = pb[j];
+                    A.pos_out[(int64_t)b * A.out_T + t0 + j] = s_pos[j];
             if (A.lens && m == 0 && threadIdx.x == 0) A.lens[b] = A.in_T;
             if (A.v_out) {
                 const int wpr = A.Hkv * D * (int)sizeof(T) / 16;
