@@ -52,6 +52,24 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's);
+    every rank calls it at the same point."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -335,16 +353,13 @@ def bench_decode(args, dev, world):
         torch.cuda.synchronize(dev)
         times.append(e0.elapsed_time(e1))
     assert int(cache.lens[0].item()) == cap
-    tot = torch.tensor([sum(times)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    ms_step = float(tot.item()) / (len(times) * S)
+    ms_step = max_over_ranks(sum(times), dev, world) / (len(times) * S)
     del graph
     pk, src = peaks()
     bps = decode_bytes_per_step(w, w.T, S)
     achieved = bps / (ms_step / 1e3) / 1e9
-    return {"metric": "decode steps/s", "value": world * 1e3 / ms_step, "unit": "steps/s",
-            "tokens_per_s": world * w.B * 1e3 / ms_step, "ms_per_step": ms_step,
+    return {"metric": "decode steps/s", "value": whole_job_rate(1, world, ms_step), "unit": "steps/s",
+            "tokens_per_s": whole_job_rate(w.B, world, ms_step), "ms_per_step": ms_step,
             "steps_per_replay": S, "replays": len(times),
             "config": {"workload": w.name, "B": w.B, "cache_tokens": f"{w.T}..{cap - 1}",
                        "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
@@ -402,10 +417,7 @@ def bench_hosttier(args, dev, world):
         hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    t = torch.tensor([e0.elapsed_time(e1) / steps], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
     # host-to-device peak of this machine: copy engine, pinned source, 256 MiB
     src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
     dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -418,7 +430,7 @@ def bench_hosttier(args, dev, world):
         torch.cuda.synchronize(dev)
         best = max(best, src.numel() / (a.elapsed_time(b) / 1e3) / 1e9)
     achieved = link / (ms / 1e3) / 1e9
-    return {"metric": "host-tier prefill tokens/s", "value": world * w.B * w.T / (ms / 1e3),
+    return {"metric": "host-tier prefill tokens/s", "value": whole_job_rate(w.B * w.T, world, ms),
             "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
             "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
                        "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
@@ -497,13 +509,9 @@ def main():
         dist.barrier()
     total_ms = evs[0][0].elapsed_time(evs[-1][3])
     stage_ms = [statistics.mean(e[a].elapsed_time(e[a + 1]) for e in evs) for a in range(3)]
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_per_step = total_ms / args.steps
-    tokens = w.B * w.T * world * args.steps
-    value = tokens / (total_ms / 1e3)
+    value = whole_job_rate(w.B * w.T * args.steps, world, total_ms)
 
     # end to end through the public one-call API, host buffers, copies inside
     e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 20))
@@ -529,10 +537,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = (w.B * w.T * world * e2e_steps / (float(te.item()) / 1e3)) if e2e_steps else None
+    te = max_over_ranks(e0.elapsed_time(e1), dev, world)
+    e2e_value = whole_job_rate(w.B * w.T * e2e_steps, world, te) if e2e_steps else None
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hpos))
     d2h = hout.numel() * hout.element_size()
 
