@@ -8,31 +8,33 @@
 // The pages check decode against a full recompute (Table 7); the tests here
 // do the same against the oracle.
 //
-// Two kernels per step, both HBM-bound.  The visible set splits into a part
+// Three kernels per step, all HBM-bound.  The visible set splits into a part
 // routing does not touch (sinks, recent chunks, the current chunk) and the
-// routed groups, so the first kernel attends over the fixed part while it
-// routes, and the second only has to add the routed groups.
-//   k_decode_a  grid (max(scan splits, fixed splits), KV heads, sequences);
-//               each CTA takes one slice of both jobs, so the whole grid is
-//               resident at once (one wave):
-//     fixed keys  CTA s < 4 attends the KV head's G query heads over a slice
-//                 of the fixed keys (the new token's key and value straight
-//                 from the step's inputs, everything else from the cache) and
-//                 writes partial softmax sums;
-//     scan        CTA s < scan splits: split 0 appends the token (rotated key,
-//                 value, position, raw key of the open chunk) and, when the
-//                 token closes its chunk, writes that chunk's summaries.  Each
-//                 scores its 256 middle chunks, one summary row per thread
-//                 (fp64 dot products), and keeps its top K_c keys; the last one
-//                 to finish (atomic counter) merges them, scores the groups of
-//                 the chosen chunks and keeps the top K_g.
+// routed groups, so the fixed part is attended on a second stream while the
+// step routes, and only the routed groups wait for the routing.
+//   k_decode_a  grid (scan splits, KV heads, sequences): split 0 appends the
+//               token (rotated key, value, position, raw key of the open
+//               chunk) and, when the token closes its chunk, writes that
+//               chunk's summaries.  Each CTA scores its 256 middle chunks, one
+//               summary row per thread (fp64 dot products), and keeps its top
+//               K_c keys; the last one to finish (atomic counter) merges them,
+//               scores the groups of the chosen chunks and keeps the top K_g.
+//   k_decode_fixed  grid (4, KV heads, sequences), on a second stream forked
+//               before and joined after the step, beside k_decode_a: attends
+//               the KV head's G query heads over a slice of the fixed keys
+//               (the new token's key and value straight from the step's
+//               inputs, everything else from the cache) and writes partial
+//               softmax sums.
 //   k_decode_b  grid (routed splits, KV heads, sequences), launched as a
 //               programmatic dependent of k_decode_a: it rotates the queries,
-//               then waits for k_decode_a, attends over a slice of the routed
-//               groups, and the last CTA per (sequence, KV head) combines all
-//               partials; the last of those per sequence increments lens.
+//               then waits for k_decode_a and attends over a slice of the
+//               routed groups.
+// The last of the 8 slice CTAs (fixed or routed) of a (sequence, KV head)
+// combines all partials; the last of those per sequence increments lens.
 // Counters live in the workspace; each last CTA resets its counter, so the
 // workspace only has to be zeroed before its first use.
+#include <mutex>
+
 #include "hga_internal.cuh"
 #include "route_common.cuh"
 #include "vec.cuh"
@@ -303,8 +305,105 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
     }
 }
 
-// Shared memory of k_decode_a: a CTA runs its fixed-key attention first and
-// its scan afterwards, so the two jobs' buffers share one pool.
+// Every slice CTA (fixed or routed) ends here: the last of the kParts
+// slices of (b, h) to finish combines all partial softmax sums into the
+// output, and the last (b, h) of a sequence increments its lens.
+template <typename T, int D>
+__device__ void finish_slice(const DecodeArgs &A, int b, int h, int t, int *s_last) {
+    constexpr int DL = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int done = atomicAdd(&A.att_done[b * A.Hkv + h], 1);
+        *s_last = done == kParts - 1;
+    }
+    __syncthreads();
+    if (!*s_last) return;
+    __threadfence();
+    const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
+    for (int g = warp; g < A.G; g += nw) {
+        const float *src = part_b + (int64_t)g * kParts * (D + 2);
+        // every partial's (m, l, o slice) in one round trip to L2
+        float ms[kParts], ls[kParts], vs[kParts][DL];
+#pragma unroll
+        for (int sp = 0; sp < kParts; ++sp) {
+            ms[sp] = __ldcg(src + sp * (D + 2));
+            ls[sp] = __ldcg(src + sp * (D + 2) + 1);
+#pragma unroll
+            for (int e = 0; e < DL; ++e) vs[sp][e] = __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, ms[sp]);
+        float L = 0.f, acc[DL];
+#pragma unroll
+        for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < kParts; ++sp) {
+            const float w = ms[sp] == -INFINITY ? 0.f : exp2f(ms[sp] - M);
+            L += w * ls[sp];
+#pragma unroll
+            for (int e = 0; e < DL; ++e) acc[e] += w * vs[sp][e];
+        }
+        const float inv = 1.f / L;
+        T *o = static_cast<T *>(A.out) + ((int64_t)b * A.Hq + (int64_t)h * A.G + g) * D;
+#pragma unroll
+        for (int e = 0; e < DL; ++e) o[lane * DL + e] = from_f<T>(acc[e] * inv);
+        if (A.lse && lane == 0)
+            A.lse[(int64_t)b * A.Hq + (int64_t)h * A.G + g] = (M + __log2f(L)) * 0.6931471805599453f;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        A.att_done[b * A.Hkv + h] = 0;
+        __threadfence();
+        const int done = atomicAdd(&A.seq_done[b], 1);
+        if (done == A.Hkv - 1) {
+            A.seq_done[b] = 0;
+            A.lens[b] = t + 1;
+        }
+    }
+}
+
+// The fixed keys of the token's visible set (sinks, recent chunks, the
+// current chunk up to the token; the new key and value straight from the
+// step's inputs, everything else from the cache), split in kFixSplits
+// slices.  Runs beside k_decode_a on a second stream: it needs no routing.
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A) {
+    __shared__ __align__(16) float qs[kMaxG * D];
+    __shared__ __align__(16) T knew[D];
+    __shared__ float sc[kMaxG * kThreads];
+    __shared__ int kt_s[kThreads];
+    __shared__ int s_last;
+    extern __shared__ __align__(16) unsigned char dyn[];
+    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
+    const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t = A.lens[b];
+    if (t < 0 || t >= A.Tc) {
+        if (threadIdx.x == 0) atomicExch(&g_decode_error, (int)HGA_ERR_BOUNDS);
+        return;   // every CTA of this sequence sees the same lens and skips
+    }
+    const int c = t / A.C;
+    const int32_t pnew = A.pos_new[b];
+    const int nsink = min(A.F, c);
+    const int rec_lo = max(c - max(A.L, 1), nsink);
+    const int n1 = nsink * A.C, n2 = n1 + (c - rec_lo) * A.C;
+    const int nfix = n2 + (t - c * A.C + 1);
+    const int per = (nfix + kFixSplits - 1) / kFixSplits;
+    const int k0 = min(nfix, f * per), nk = min(nfix, k0 + per) - k0;
+    load_queries<T, D>(A, b, h, pnew, qs);
+    rotate_new_key<T, D>(A, b, h, pnew, knew);
+    __syncthreads();
+    auto key_of = [&](int k) {
+        const int i = k0 + k;
+        return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
+    };
+    attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
+    finish_slice<T, D>(A, b, h, t, &s_last);
+}
+
+// Shared memory of k_decode_a (chunk scan and routing).
 template <typename T, int D>
 struct ScanSmem {
     double qr[D];
@@ -312,34 +411,17 @@ struct ScanSmem {
     unsigned long long lists[kThreads];
     RouteScratch rs;
 };
-template <typename T, int D>
-struct AttSmem {
-    float qs[kMaxG * D];
-    T knew[D];
-    float sc[kMaxG * kThreads];
-    int kt_s[kThreads];
-};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     constexpr int H = D / 2;
-    constexpr size_t kPool = sizeof(ScanSmem<T, D>) > sizeof(AttSmem<T, D>)
-                                 ? sizeof(ScanSmem<T, D>) : sizeof(AttSmem<T, D>);
-    __shared__ __align__(16) unsigned char pool[kPool];
+    __shared__ ScanSmem<T, D> ss;
     __shared__ int s_last;
-    extern __shared__ __align__(16) unsigned char dyn[];
-    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
-    ScanSmem<T, D> &ss = *reinterpret_cast<ScanSmem<T, D> *>(pool);
-    AttSmem<T, D> &as = *reinterpret_cast<AttSmem<T, D> *>(pool);
     double *qr = ss.qr;
     unsigned long long *cand = ss.cand;
     unsigned long long *lists = ss.lists;
     RouteScratch &rs = ss.rs;
     int *sel_c = rs.sel_c, *sel_g = rs.sel_g;
-    float *qs = as.qs;
-    T *knew = as.knew;
-    float *sc = as.sc;
-    int *kt_s = as.kt_s;
 
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
@@ -349,31 +431,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     }
     const int c = t / A.C;
     const int32_t pnew = A.pos_new[b];
-
-    if (s < kFixSplits) {
-        // ------------------------------------------- fixed-key attention --
-        const int f = s;
-        const int nsink = min(A.F, c);
-        const int rec_lo = max(c - max(A.L, 1), nsink);
-        const int n1 = nsink * A.C, n2 = n1 + (c - rec_lo) * A.C;
-        const int nfix = n2 + (t - c * A.C + 1);
-        const int per = (nfix + kFixSplits - 1) / kFixSplits;
-        const int k0 = min(nfix, f * per), nk = min(nfix, k0 + per) - k0;
-        load_queries<T, D>(A, b, h, pnew, qs);
-        rotate_new_key<T, D>(A, b, h, pnew, knew);
-        __syncthreads();
-        auto key_of = [&](int k) {
-            const int i = k0 + k;
-            return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
-        };
-        attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
-        __syncthreads();          // the scan below reuses the shared pool
-    }
-    if (s >= A.ns_scan) {
-        // no chunk rows for this CTA: the routed-keys kernel may start launching
-        asm volatile("griddepcontrol.launch_dependents;");
-        return;
-    }
 
     // ------------------------------------------------------------- scan --
     if (s == 0) {
@@ -487,7 +544,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
-    constexpr int DL = D / 32;
     __shared__ __align__(16) float qs[kMaxG * D];
     __shared__ __align__(16) T knew[D];
     __shared__ float sc[kMaxG * kThreads];
@@ -498,7 +554,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
 
     const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int t = A.lens[b];          // written only by the previous step
     const int32_t pnew = A.pos_new[b];
     if (t >= 0 && t < A.Tc) load_queries<T, D>(A, b, h, pnew, qs);
@@ -519,58 +574,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     };
     attend_part<T, D>(A, b, h, t, nk, key_of, kFixSplits + r, qs, knew, sc, kt_s, Vs);
 
-    // the last CTA of (b, h) combines the fixed and routed partials
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int done = atomicAdd(&A.att_done[b * A.Hkv + h], 1);
-        s_last = done == kRouteSplits - 1;
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
-    for (int g = warp; g < A.G; g += nw) {
-        const float *src = part_b + (int64_t)g * kParts * (D + 2);
-        // every partial's (m, l, o slice) in one round trip to L2
-        float ms[kParts], ls[kParts], vs[kParts][DL];
-#pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) {
-            ms[sp] = __ldcg(src + sp * (D + 2));
-            ls[sp] = __ldcg(src + sp * (D + 2) + 1);
-#pragma unroll
-            for (int e = 0; e < DL; ++e) vs[sp][e] = __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
-        }
-        float M = -INFINITY;
-#pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, ms[sp]);
-        float L = 0.f, acc[DL];
-#pragma unroll
-        for (int e = 0; e < DL; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) {
-            const float w = ms[sp] == -INFINITY ? 0.f : exp2f(ms[sp] - M);
-            L += w * ls[sp];
-#pragma unroll
-            for (int e = 0; e < DL; ++e) acc[e] += w * vs[sp][e];
-        }
-        const float inv = 1.f / L;
-        T *o = static_cast<T *>(A.out) + ((int64_t)b * A.Hq + (int64_t)h * A.G + g) * D;
-#pragma unroll
-        for (int e = 0; e < DL; ++e) o[lane * DL + e] = from_f<T>(acc[e] * inv);
-        if (A.lse && lane == 0)
-            A.lse[(int64_t)b * A.Hq + (int64_t)h * A.G + g] = (M + __log2f(L)) * 0.6931471805599453f;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        A.att_done[b * A.Hkv + h] = 0;
-        __threadfence();
-        const int done = atomicAdd(&A.seq_done[b], 1);
-        if (done == A.Hkv - 1) {
-            A.seq_done[b] = 0;
-            A.lens[b] = t + 1;
-        }
-    }
+    finish_slice<T, D>(A, b, h, t, &s_last);
 }
 
 struct Ws {
@@ -602,6 +606,31 @@ Ws layout(const Geo &g) {
     o += up256(sizeof(float) * (size_t)g.B * g.Hq * kParts * (g.D + 2));
     w.total = o;
     return w;
+}
+
+// Per-device side stream and fork / join events for the fixed-key slices,
+// created on the first decode step of a device and kept for the process.
+// One mutex keeps a step's enqueue sequence (which reuses the events) whole.
+struct DecodeSide {
+    bool ready = false;
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_dec_mu;
+DecodeSide g_dec_side[64];
+
+cudaError_t decode_side(int dev, DecodeSide **out) {
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    DecodeSide &d = g_dec_side[dev];
+    if (!d.ready) {
+        cudaError_t e = cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
 }
 
 template <typename T, int D>
@@ -648,10 +677,19 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.rope = r;
 
     const size_t vs_bytes = sizeof(T) * (size_t)kThreads * D;
-    cudaError_t e = ensure_smem((const void *)k_decode_a<T, D>, vs_bytes);
+    cudaError_t e = ensure_smem((const void *)k_decode_fixed<T, D>, vs_bytes);
     if (e == cudaSuccess) e = ensure_smem((const void *)k_decode_b<T, D>, vs_bytes);
     if (e != cudaSuccess) return cuda_status(e);
-    k_decode_a<T, D><<<dim3(max(A.ns_scan, kFixSplits), g.Hkv, g.B), kThreads, vs_bytes, st>>>(A);
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_status(e);
+    std::lock_guard<std::mutex> lock(g_dec_mu);
+    DecodeSide *sd = nullptr;
+    if ((e = decode_side(dev, &sd)) != cudaSuccess) return cuda_status(e);
+    // caller's stream: scan and routing, then the routed slices as its
+    // programmatic dependents; side stream (forked before, joined after):
+    // the fixed slices, which need no routing
+    if ((e = cudaEventRecord(sd->fork, st)) != cudaSuccess) return cuda_status(e);
+    k_decode_a<T, D><<<dim3(A.ns_scan, g.Hkv, g.B), kThreads, 0, st>>>(A);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg = {};
@@ -664,8 +702,12 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, k_decode_b<T, D>, A);
-    return cuda_status(e);
+    if ((e = cudaLaunchKernelEx(&cfg, k_decode_b<T, D>, A)) != cudaSuccess) return cuda_status(e);
+    if ((e = cudaStreamWaitEvent(sd->side, sd->fork, 0)) != cudaSuccess) return cuda_status(e);
+    k_decode_fixed<T, D><<<dim3(kFixSplits, g.Hkv, g.B), kThreads, vs_bytes, sd->side>>>(A);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    if ((e = cudaEventRecord(sd->join, sd->side)) != cudaSuccess) return cuda_status(e);
+    return cuda_status(cudaStreamWaitEvent(st, sd->join, 0));
 }
 
 }  // namespace

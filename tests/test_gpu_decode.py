@@ -40,8 +40,11 @@ def _np(t):
     return t.detach().float().cpu().numpy()
 
 
-def run_decode(hga, w, T_hist, steps, cap, seed):
+def run_decode(hga, w, T_hist, steps, cap, seed, pos_mod=None):
     d = make_decode_inputs(w, seed=seed, T=T_hist, steps=steps)
+    if pos_mod:
+        d["pos_hist"] = (d["pos_hist"] % pos_mod).contiguous()
+        d["pos_new"] = (d["pos_new"] % pos_mod).contiguous()
     dev = torch.device("cuda")
     dt = d["k_hist"].dtype
     hp = _hp(hga, w)
@@ -63,10 +66,10 @@ def run_decode(hga, w, T_hist, steps, cap, seed):
     return d, cache, torch.stack(outs), torch.stack(lses), torch.stack(selc), torch.stack(selg)
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_decode_parity(gpu_lib, name):
-    w, T_hist, steps, cap = CASES[name]
-    d, cache, out, lse, selc, selg = run_decode(gpu_lib, w, T_hist, steps, cap, seed=5)
+def check_decode(hga, case, seed=5, pos_mod=None):
+    w, T_hist, steps, cap = case
+    d, cache, out, lse, selc, selg = run_decode(hga, w, T_hist, steps, cap, seed=seed,
+                                                pos_mod=pos_mod)
     Ttot = T_hist + steps
     K = torch.cat([d["k_hist"], d["k_new"].transpose(0, 1)], 1)
     V = torch.cat([d["v_hist"], d["v_new"].transpose(0, 1)], 1)
@@ -102,6 +105,19 @@ def test_decode_parity(gpu_lib, name):
     assert row_rel_err(_np(cache.s_chunk[:, :, :nc]), S_c[:, :, :nc]) < 2e-6
     assert row_rel_err(_np(cache.s_group[:, :, :nc * (64 // w.g_s)]),
                        S_g[:, :, :nc * (64 // w.g_s)]) < 2e-6
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_decode_parity(gpu_lib, name):
+    check_decode(gpu_lib, CASES[name])
+
+
+def test_decode_wrapped_positions(gpu_lib):
+    """Positions modulo a period shorter than the sequence (the pages'
+    position-mod-65536 variant at a small period): the steps cross a wrap
+    and a chunk boundary; rotation uses the given positions, causality the
+    token index."""
+    check_decode(gpu_lib, CASES["bf16_qwen_like"], seed=8, pos_mod=677)
 
 
 def test_decode_full_budget_is_dense(gpu_lib):

@@ -48,8 +48,10 @@ def _np(t):
     return t.detach().float().cpu().numpy()
 
 
-def run_and_check(hga, w, seed, units=None, sample_rows=None):
+def run_and_check(hga, w, seed, units=None, sample_rows=None, pos_mod=None):
     q, k, v, pos, _ = make_prefill_inputs(w, seed=seed)
+    if pos_mod:
+        pos = (pos % pos_mod).contiguous()
     dev = torch.device("cuda")
     qd, kd, vd, pd = (x.to(dev) for x in (q, k, v, pos))
     hp = _hp(w)
@@ -149,3 +151,12 @@ def test_exact_token_chunk_variant(gpu_lib):
             chunks = sc[0, blk, h][sc[0, blk, h] >= 0]
             groups = sg[0, blk, h][sg[0, blk, h] >= 0]
             assert sorted(groups.tolist()) == sorted((chunks[:, None] * gpc + np.arange(gpc)).ravel().tolist())
+
+
+@pytest.mark.parametrize("name,mod", [("f32_ragged_1000", 300), ("bf16_qwen_ragged", 1000)])
+def test_prefill_wrapped_positions(gpu_lib, name, mod):
+    """Positions taken modulo a period shorter than the sequence (the pages'
+    position-mod-65536 variant, at a period the oracle can check quickly):
+    RoPE and the summaries' mean positions use the given positions, while
+    causality and the chunk structure follow the token index."""
+    run_and_check(gpu_lib, CASES[name], seed=17, pos_mod=mod)
