@@ -413,7 +413,7 @@ struct ScanSmem {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
+__global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
     constexpr int H = D / 2;
     __shared__ ScanSmem<T, D> ss;
     __shared__ int s_last;
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
     if (threadIdx.x < n)
         cand[threadIdx.x] = pack_key(
-            (float)thread_dot_row<D>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
+            (float)thread_dot_row<D, 8>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
             first + threadIdx.x);
     __syncthreads();
     unsigned long long *mine = A.cand + (((int64_t)b * A.Hkv + h) * A.ns_scan + s) * A.K_c;
@@ -525,9 +525,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_a(const DecodeArgs A) {
     for (int r = threadIdx.x; r < A.K_c; r += blockDim.x) oc[r] = sel_c[r];
     const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
     const int ng = kc * A.gpc;
-    for (int r = threadIdx.x; r < ng; r += blockDim.x) {
-        const int gid = sel_c[r / A.gpc] * A.gpc + r % A.gpc;
-        cand[r] = pack_key((float)thread_dot_row<D>(qr, Sg + (int64_t)gid * D), gid);
+    // four lanes per group row (all of a row's loads in one round trip)
+    for (int x = threadIdx.x; x < ((ng + 63) / 64) * 256; x += blockDim.x) {
+        const int r = x >> 2;
+        const int rr = r < ng ? r : 0;            // whole quads stay converged
+        const int gid = sel_c[rr / A.gpc] * A.gpc + rr % A.gpc;
+        const double sv = ng > 0 ? quad_dot_row<D>(qr, Sg + (int64_t)gid * D) : 0.0;
+        if (r < ng && (x & 3) == 0) cand[r] = pack_key((float)sv, gid);
     }
     __syncthreads();
     if (A.K_g <= 32) {

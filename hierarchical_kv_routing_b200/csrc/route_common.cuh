@@ -224,13 +224,39 @@ __device__ __forceinline__ int block_topk32(const unsigned long long *cand, int 
 
 namespace hga {
 
+// fp64 dot product of q (shared, fp64) with one fp32 row by a quad of
+// adjacent lanes (each a quarter of the row, all its loads in flight), the
+// partial sums combined across the quad; every lane of the quad returns it.
+template <int D>
+__device__ __forceinline__ double quad_dot_row(const double *qr, const float *__restrict__ row) {
+    constexpr int kPer = D / 16;                  // float4 loads per lane
+    const int part = threadIdx.x & 3;
+    const float4 *r4 = reinterpret_cast<const float4 *>(row) + part * kPer;
+    const double2 *q2 = reinterpret_cast<const double2 *>(qr) + part * kPer * 2;
+    float4 v[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) v[e] = __ldg(r4 + e);
+    double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+        const double2 a = q2[2 * e], b = q2[2 * e + 1];
+        s0 = fma(a.x, (double)v[e].x, s0);
+        s1 = fma(a.y, (double)v[e].y, s1);
+        s0 = fma(b.x, (double)v[e].z, s0);
+        s1 = fma(b.y, (double)v[e].w, s1);
+    }
+    double s = s0 + s1;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    return s;
+}
+
 // fp64 dot product of q (shared, fp64) with one fp32 row, by one thread
 // (the whole row streams through this thread's 16-byte loads).
-template <int D>
+template <int D, int kBatch = 8>
 __device__ __forceinline__ double thread_dot_row(const double *qr, const float *__restrict__ row) {
-    // 8 loads in flight per batch: several rows per thread and CTAs per SM
-    // cover the latency, and the routers stay within 80 registers
-    constexpr int kBatch = 8;
+    // kBatch 16-byte loads in flight per batch (8 by default: several rows per
+    // thread and CTAs per SM cover the latency, within few registers)
     const float4 *r4 = reinterpret_cast<const float4 *>(row);
     const double2 *q2 = reinterpret_cast<const double2 *>(qr);
     double s0 = 0.0, s1 = 0.0;
