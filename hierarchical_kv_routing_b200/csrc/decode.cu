@@ -19,17 +19,19 @@
 //               summary row per thread (fp64 dot products), and keeps its top
 //               K_c keys; the last one to finish (atomic counter) merges them,
 //               scores the groups of the chosen chunks and keeps the top K_g.
-//   k_decode_fixed  grid (4, KV heads, sequences), on a second stream forked
+//   k_decode_fixed  grid (nF, KV heads, sequences), on a second stream forked
 //               before and joined after the step, beside k_decode_a: attends
 //               the KV head's G query heads over a slice of the fixed keys
 //               (the new token's key and value straight from the step's
 //               inputs, everything else from the cache) and writes partial
 //               softmax sums.
-//   k_decode_b  grid (routed splits, KV heads, sequences), launched as a
-//               programmatic dependent of k_decode_a: it rotates the queries,
-//               then waits for k_decode_a and attends over a slice of the
-//               routed groups.
-// The last of the 8 slice CTAs (fixed or routed) of a (sequence, KV head)
+//   k_decode_b  grid (nR, KV heads, sequences), launched as a programmatic
+//               dependent of k_decode_a: it rotates the queries, then waits
+//               for k_decode_a and attends over a slice of the routed groups.
+// A slice holds at most slice_keys keys (128 for bf16, D = 128): their key
+// and value rows are staged in shared memory, and Q.K runs register-blocked
+// (each query slice read from shared memory serves four keys).
+// The last of the nF + nR slice CTAs (fixed or routed) of a (sequence, KV head)
 // combines all partials; the last of those per sequence increments lens.
 // Counters live in the workspace; each last CTA resets its counter, so the
 // workspace only has to be zeroed before its first use.
@@ -47,9 +49,14 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kScanChunks = 256;  // middle chunks per scan CTA (one per thread)
-constexpr int kFixSplits = 4;     // CTAs over the fixed keys per (sequence, KV head)
-constexpr int kRouteSplits = 4;   // CTAs over the routed keys
-constexpr int kParts = kFixSplits + kRouteSplits;
+// Keys per attention slice CTA: its key and value rows (32 KB each) are
+// staged in shared memory, which keeps two slice CTAs per SM.
+template <typename T, int D>
+constexpr int slice_keys() {
+    return (32 * 1024) / (D * (int)sizeof(T)) < kThreads ? (32 * 1024) / (D * (int)sizeof(T))
+                                                          : kThreads;
+}
+constexpr int kMinSliceKeys = 64;     // the smallest slice_keys of any type and size
 constexpr int kMaxG = 16;
 constexpr int kMaxCand = 1024;    // merge and group candidate table
 
@@ -66,7 +73,8 @@ struct DecodeArgs {
     float *lse;
     int32_t *sel_c, *sel_g;          // [B, Hkv, K]
     unsigned long long *cand;        // [B, Hkv, ns_scan, K_c]
-    float *part;                     // [B, Hq, kParts, D + 2]
+    float *part;                     // [B, Hq, nparts, D + 2]
+    int nF, nR, nparts;              // fixed and routed slice CTAs per (sequence, KV head)
     int32_t *scan_done, *att_done, *seq_done;
     float scale_log2;
     Rope rope;
@@ -209,67 +217,114 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                  : "memory");
 }
 
-// Partial attention of the G heads over keys key_of(0..nk), nk <= blockDim.
-// The value rows are staged in shared memory (Vs, [nk][D]) with cp.async
-// while the scores are computed, one key per thread with the key row's
-// 16-byte loads all in flight; softmax and P.V then run one warp per head
-// with lanes over dims.  Writes (m, l, o[D]) for part index `pi`.
+// Partial attention of the G heads over keys key_of(0..nk), nk <=
+// slice_keys.  The key and value rows are staged in shared memory with
+// cp.async (the token's own key from knew, its value from the step's
+// inputs).  Q.K: lane s of a key group holds 16-byte slice s of 4 keys and
+// scores them for 8 heads at a time (each q slice read from shared memory
+// serves 4 keys); the group's lanes reduce-scatter the 32 partial sums.
+// Softmax and P.V then run one warp per head with lanes over dims.  Writes
+// (m, l, o[D]) for part index `pi`.
 template <typename T, int D, typename KeyOf>
 __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, KeyOf key_of,
-                            int pi, const float *qs, const T *knew, float *sc, int *kt_s, T *Vs) {
+                            int pi, const float *qs, const T *knew, float *sc, int *kt_s, T *Ks,
+                            T *Vs) {
     constexpr int DL = D / 32;
     constexpr int NV = D * (int)sizeof(T) / 16;     // 16-byte slices per row
     constexpr int EV = 16 / (int)sizeof(T);         // elements per slice
+    constexpr int KPG = 4;                          // keys per Q.K lane
+    constexpr int NVAL = KPG * 8;                   // partial sums per lane
+    constexpr int R = NVAL / NV;                    // sums per lane after the reduce
+    constexpr int KPP = KPG * kThreads / NV;        // keys per Q.K pass
+    static_assert(32 % NV == 0 && NVAL % NV == 0, "Q.K lane groups");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     for (int k = threadIdx.x; k < nk; k += blockDim.x) kt_s[k] = key_of(k);
     __syncthreads();
-    // Every thread handles at most one key (nk * tpk <= blockDim): its key
-    // row's loads go out first, then the value rows' asynchronous copies, and
-    // only then does the thread wait on its key row for the dot products.
-    const int tpk = nk <= (int)blockDim.x / 2 ? 2 : 1;
-    const int gper = (A.G + tpk - 1) / tpk;
-    const int kk = threadIdx.x / tpk, part = threadIdx.x % tpk;
-    const bool has_key = kk < nk;
-    const int kt = has_key ? kt_s[kk] : 0;
-    uint4 kw[NV];
-    if (has_key) {
-        if (kt == t) {
-#pragma unroll
-            for (int e = 0; e < NV; ++e) kw[e] = reinterpret_cast<const uint4 *>(knew)[e];
-        } else {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                static_cast<const T *>(A.k_rot) + (((int64_t)b * A.Tc + kt) * A.Hkv + h) * D);
-#pragma unroll
-            for (int e = 0; e < NV; ++e) kw[e] = __ldg(src + e);
-        }
-    }
+    const T *kbase = static_cast<const T *>(A.k_rot);
     const T *vbase = static_cast<const T *>(A.v);
     const T *vn = static_cast<const T *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
     for (int idx = threadIdx.x; idx < nk * NV; idx += blockDim.x) {
         const int k = idx / NV, pv = idx % NV;
         const int kv = kt_s[k];
-        const T *src = kv == t ? vn : vbase + (((int64_t)b * A.Tc + kv) * A.Hkv + h) * D;
+        const int64_t row = (((int64_t)b * A.Tc + kv) * A.Hkv + h) * D;
+        uint4 *kd = reinterpret_cast<uint4 *>(Ks + (size_t)k * D) + pv;
+        if (kv == t) *kd = reinterpret_cast<const uint4 *>(knew)[pv];
+        else cp_async16(kd, reinterpret_cast<const uint4 *>(kbase + row) + pv);
         cp_async16(reinterpret_cast<uint4 *>(Vs + (size_t)k * D) + pv,
-                   reinterpret_cast<const uint4 *>(src) + pv);
+                   reinterpret_cast<const uint4 *>(kv == t ? vn : vbase + row) + pv);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    if (has_key) {
-        const int g1 = min(A.G, (part + 1) * gper);
-#pragma unroll 1
-        for (int g = part * gper; g < g1; ++g) {
-            const float *qg = qs + g * D;
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int e = 0; e < NV; e += 2) {
-                a0 += dot16<T>(kw[e], qg + e * EV);
-                a1 += dot16<T>(kw[e + 1], qg + (e + 1) * EV);
-            }
-            sc[g * kThreads + kk] = a0 + a1;
-        }
-    }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
+    {
+        const int sl = threadIdx.x % NV, kgp = threadIdx.x / NV;
+        for (int k0 = 0; k0 < nk; k0 += KPP) {
+            float kx[KPG][EV];
+#pragma unroll
+            for (int j = 0; j < KPG; ++j) {
+                const int key = k0 + kgp * KPG + j;
+                uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                if (key < nk) w = reinterpret_cast<const uint4 *>(Ks + (size_t)key * D)[sl];
+                if constexpr (sizeof(T) == 2) {
+                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&w);
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) {
+                        const float2 f = __bfloat1622float2(h2[z]);
+                        kx[j][2 * z] = f.x;
+                        kx[j][2 * z + 1] = f.y;
+                    }
+                } else {
+                    kx[j][0] = __uint_as_float(w.x);
+                    kx[j][1] = __uint_as_float(w.y);
+                    kx[j][2] = __uint_as_float(w.z);
+                    kx[j][3] = __uint_as_float(w.w);
+                }
+            }
+            for (int g0 = 0; g0 < A.G; g0 += 8) {
+                float v[NVAL];
+#pragma unroll
+                for (int x = 0; x < NVAL; ++x) v[x] = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < 8; ++hh) {
+                    if (g0 + hh < A.G) {
+                        const float4 *q4 = reinterpret_cast<const float4 *>(qs + (g0 + hh) * D + sl * EV);
+#pragma unroll
+                        for (int z = 0; z < EV / 4; ++z) {
+                            const float4 qv = q4[z];
+#pragma unroll
+                            for (int j = 0; j < KPG; ++j) {
+                                float a = v[j * 8 + hh];
+                                a = fmaf(qv.x, kx[j][4 * z], a);
+                                a = fmaf(qv.y, kx[j][4 * z + 1], a);
+                                a = fmaf(qv.z, kx[j][4 * z + 2], a);
+                                a = fmaf(qv.w, kx[j][4 * z + 3], a);
+                                v[j * 8 + hh] = a;
+                            }
+                        }
+                    }
+                }
+                // reduce-scatter over the group's lanes: lane s keeps sums
+                // [s R, s R + R) of the group's 4 keys x 8 heads
+#pragma unroll
+                for (int st = NV / 2, n = NVAL; st >= 1; st >>= 1, n >>= 1) {
+                    const bool up = (lane & st) != 0;
+#pragma unroll
+                    for (int x = 0; x < n / 2; ++x) {
+                        const float send = up ? v[x] : v[x + n / 2];
+                        const float keep = up ? v[x + n / 2] : v[x];
+                        v[x] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < R; ++x) {
+                    const int id = sl * R + x, key = k0 + kgp * KPG + id / 8, g = g0 + id % 8;
+                    if (key < nk && g < A.G) sc[g * kThreads + key] = v[x];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * A.nparts * (D + 2);
     for (int g = warp; g < A.G; g += nw) {
         float m = -INFINITY;
         for (int k = lane; k < nk; k += 32) m = fmaxf(m, sc[g * kThreads + k]);
@@ -295,7 +350,7 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
 #pragma unroll
             for (int e = 0; e < DL; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
         }
-        float *dst = part_b + ((int64_t)g * kParts + pi) * (D + 2);
+        float *dst = part_b + ((int64_t)g * A.nparts + pi) * (D + 2);
 #pragma unroll
         for (int e = 0; e < DL; ++e) dst[2 + lane * DL + e] = acc[e];
         if (lane == 0) {
@@ -305,7 +360,7 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
     }
 }
 
-// Every slice CTA (fixed or routed) ends here: the last of the kParts
+// Every slice CTA (fixed or routed) ends here: the last of the nparts
 // slices of (b, h) to finish combines all partial softmax sums into the
 // output, and the last (b, h) of a sequence increments its lens.
 template <typename T, int D>
@@ -316,35 +371,28 @@ __device__ void finish_slice(const DecodeArgs &A, int b, int h, int t, int *s_la
     __syncthreads();
     if (threadIdx.x == 0) {
         const int done = atomicAdd(&A.att_done[b * A.Hkv + h], 1);
-        *s_last = done == kParts - 1;
+        *s_last = done == A.nparts - 1;
     }
     __syncthreads();
     if (!*s_last) return;
     __threadfence();
-    const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * kParts * (D + 2);
+    const float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * A.nparts * (D + 2);
     for (int g = warp; g < A.G; g += nw) {
-        const float *src = part_b + (int64_t)g * kParts * (D + 2);
-        // every partial's (m, l, o slice) in one round trip to L2
-        float ms[kParts], ls[kParts], vs[kParts][DL];
-#pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) {
-            ms[sp] = __ldcg(src + sp * (D + 2));
-            ls[sp] = __ldcg(src + sp * (D + 2) + 1);
-#pragma unroll
-            for (int e = 0; e < DL; ++e) vs[sp][e] = __ldcg(src + sp * (D + 2) + 2 + lane * DL + e);
-        }
+        const float *src = part_b + (int64_t)g * A.nparts * (D + 2);
         float M = -INFINITY;
-#pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) M = fmaxf(M, ms[sp]);
+#pragma unroll 4
+        for (int sp = 0; sp < A.nparts; ++sp) M = fmaxf(M, __ldcg(src + sp * (D + 2)));
         float L = 0.f, acc[DL];
 #pragma unroll
         for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+        for (int sp = 0; sp < A.nparts; ++sp) {
+            const float *ps = src + sp * (D + 2);
+            const float m = __ldcg(ps);
+            const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+            L += w * __ldcg(ps + 1);
 #pragma unroll
-        for (int sp = 0; sp < kParts; ++sp) {
-            const float w = ms[sp] == -INFINITY ? 0.f : exp2f(ms[sp] - M);
-            L += w * ls[sp];
-#pragma unroll
-            for (int e = 0; e < DL; ++e) acc[e] += w * vs[sp][e];
+            for (int e = 0; e < DL; ++e) acc[e] += w * __ldcg(ps + 2 + lane * DL + e);
         }
         const float inv = 1.f / L;
         T *o = static_cast<T *>(A.out) + ((int64_t)b * A.Hq + (int64_t)h * A.G + g) * D;
@@ -367,8 +415,8 @@ __device__ void finish_slice(const DecodeArgs &A, int b, int h, int t, int *s_la
 
 // The fixed keys of the token's visible set (sinks, recent chunks, the
 // current chunk up to the token; the new key and value straight from the
-// step's inputs, everything else from the cache), split in kFixSplits
-// slices.  Runs beside k_decode_a on a second stream: it needs no routing.
+// step's inputs, everything else from the cache), split in nF slices.
+// Runs beside k_decode_a on a second stream: it needs no routing.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A) {
     __shared__ __align__(16) float qs[kMaxG * D];
@@ -377,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A
     __shared__ int kt_s[kThreads];
     __shared__ int s_last;
     extern __shared__ __align__(16) unsigned char dyn[];
-    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
+    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][D]
+    T *Vs = Ks + (size_t)slice_keys<T, D>() * D;                      // [slice_keys][D]
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
     if (t < 0 || t >= A.Tc) {
@@ -390,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A
     const int rec_lo = max(c - max(A.L, 1), nsink);
     const int n1 = nsink * A.C, n2 = n1 + (c - rec_lo) * A.C;
     const int nfix = n2 + (t - c * A.C + 1);
-    const int per = (nfix + kFixSplits - 1) / kFixSplits;
+    const int per = (nfix + A.nF - 1) / A.nF;
     const int k0 = min(nfix, f * per), nk = min(nfix, k0 + per) - k0;
     load_queries<T, D>(A, b, h, pnew, qs);
     rotate_new_key<T, D>(A, b, h, pnew, knew);
@@ -399,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A
         const int i = k0 + k;
         return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
     };
-    attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Vs);
+    attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Ks, Vs);
     finish_slice<T, D>(A, b, h, t, &s_last);
 }
 
@@ -408,8 +457,9 @@ template <typename T, int D>
 struct ScanSmem {
     double qr[D];
     unsigned long long cand[kMaxCand];
+    unsigned long long top[kMaxK];
     unsigned long long lists[kThreads];
-    RouteScratch rs;
+    int sel_c[kMaxK], sel_g[kMaxK];
 };
 
 template <typename T, int D>
@@ -419,9 +469,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
     __shared__ int s_last;
     double *qr = ss.qr;
     unsigned long long *cand = ss.cand;
-    unsigned long long *lists = ss.lists;
-    RouteScratch &rs = ss.rs;
-    int *sel_c = rs.sel_c, *sel_g = rs.sel_g;
+    int *sel_c = ss.sel_c, *sel_g = ss.sel_g;
 
     const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
@@ -485,9 +533,14 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
             (float)thread_dot_row<D, 8>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
             first + threadIdx.x);
     __syncthreads();
+    // this CTA's top K_c keys, descending and 0-padded
     unsigned long long *mine = A.cand + (((int64_t)b * A.Hkv + h) * A.ns_scan + s) * A.K_c;
-    if (A.K_c <= 32) block_topk32_keys(cand, n, A.K_c, mine, lists);
-    else topk_keys(cand, n, A.K_c, mine, rs);
+    if (A.K_c <= 32) {
+        block_topk32_keys(cand, n, A.K_c, mine, ss.lists);
+    } else {
+        rank_topk(cand, n, A.K_c, ss.top);
+        for (int r = threadIdx.x; r < A.K_c; r += blockDim.x) mine[r] = ss.top[r];
+    }
 
     // the last scan CTA of (b, h) merges and routes the groups
     __threadfence();
@@ -504,23 +557,9 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
     const int ntot = A.ns_scan * A.K_c;
     for (int r = threadIdx.x; r < ntot; r += blockDim.x) cand[r] = __ldcg(all + r);
     __syncthreads();
-    int kc;
-    if (A.K_c <= 32) {
-        block_topk32(cand, ntot, A.K_c, sel_c, lists);    // padding keys (0) never win
-        kc = 0;
-        for (int r = 0; r < A.K_c; ++r) kc += sel_c[r] >= 0;
-    } else {
-        if (threadIdx.x == 0) {               // drop the padding, keep the order
-            int w = 0;
-            for (int r = 0; r < ntot; ++r)
-                if (cand[r]) cand[w++] = cand[r];
-            s_last = w;
-        }
-        __syncthreads();
-        kc = topk_select(cand, s_last, A.K_c, sel_c, rs);
-        for (int r = kc + threadIdx.x; r < A.K_c; r += blockDim.x) sel_c[r] = -1;
-        __syncthreads();
-    }
+    // the scan CTAs' lists are descending: ranks by binary search
+    rank_topk_lists(cand, A.ns_scan, A.K_c, A.K_c, ss.top);
+    const int kc = ids_ascending(ss.top, A.K_c, sel_c);
     int32_t *oc = A.sel_c + ((int64_t)b * A.Hkv + h) * A.K_c;
     for (int r = threadIdx.x; r < A.K_c; r += blockDim.x) oc[r] = sel_c[r];
     const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
@@ -534,13 +573,8 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
         if (r < ng && (x & 3) == 0) cand[r] = pack_key((float)sv, gid);
     }
     __syncthreads();
-    if (A.K_g <= 32) {
-        block_topk32(cand, ng, A.K_g, sel_g, lists);
-    } else {
-        const int kg = topk_select(cand, ng, A.K_g, sel_g, rs);
-        for (int r = kg + threadIdx.x; r < A.K_g; r += blockDim.x) sel_g[r] = -1;
-        __syncthreads();
-    }
+    rank_topk(cand, ng, A.K_g, ss.top);
+    ids_ascending(ss.top, A.K_g, sel_g);
     int32_t *og = A.sel_g + ((int64_t)b * A.Hkv + h) * A.K_g;
     for (int r = threadIdx.x; r < A.K_g; r += blockDim.x) og[r] = sel_g[r];
     if (threadIdx.x == 0) A.scan_done[b * A.Hkv + h] = 0;
@@ -555,7 +589,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     __shared__ int sel[kMaxK];
     __shared__ int s_last;
     extern __shared__ __align__(16) unsigned char dyn[];
-    T *Vs = reinterpret_cast<T *>(dyn);                       // [kThreads][D]
+    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][D]
+    T *Vs = Ks + (size_t)slice_keys<T, D>() * D;                      // [slice_keys][D]
 
     const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];          // written only by the previous step
@@ -570,13 +605,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
     int kg = 0;
     for (int j = 0; j < A.K_g; ++j) kg += sel[j] >= 0;
     const int nrt = kg * A.g_s;
-    const int per = (nrt + kRouteSplits - 1) / kRouteSplits;
+    const int per = (nrt + A.nR - 1) / A.nR;
     const int k0 = min(nrt, r * per), nk = min(nrt, k0 + per) - k0;
     auto key_of = [&](int k) {
         const int i = k0 + k;
         return sel[i / A.g_s] * A.g_s + i % A.g_s;
     };
-    attend_part<T, D>(A, b, h, t, nk, key_of, kFixSplits + r, qs, knew, sc, kt_s, Vs);
+    attend_part<T, D>(A, b, h, t, nk, key_of, A.nF + r, qs, knew, sc, kt_s, Ks, Vs);
 
     finish_slice<T, D>(A, b, h, t, &s_last);
 }
@@ -594,8 +629,21 @@ int scan_splits(const Geo &g) {
 
 inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Fixed and routed slice CTAs per (sequence, KV head) for a slice size.
+struct Slices {
+    int nF, nR;
+};
+Slices slices(const Geo &g, int keys) {
+    Slices s;
+    s.nF = ((g.F + max(g.L, 1) + 1) * g.C + keys - 1) / keys;
+    const long long routed = min((long long)g.K_g * g.g_s, (long long)g.T);
+    s.nR = max(1, (int)((routed + keys - 1) / keys));
+    return s;
+}
+
 Ws layout(const Geo &g) {
     const int ns = scan_splits(g);
+    const Slices sl = slices(g, kMinSliceKeys);      // the most partials of any type
     Ws w;
     size_t o = 0;
     w.counters = o;
@@ -607,7 +655,7 @@ Ws layout(const Geo &g) {
     w.sel_g = o;
     o += up256(sizeof(int32_t) * (size_t)g.B * g.Hkv * g.K_g);
     w.part = o;
-    o += up256(sizeof(float) * (size_t)g.B * g.Hq * kParts * (g.D + 2));
+    o += up256(sizeof(float) * (size_t)g.B * g.Hq * (sl.nF + sl.nR) * (g.D + 2));
     w.total = o;
     return w;
 }
@@ -680,7 +728,11 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     A.rope = r;
 
-    const size_t vs_bytes = sizeof(T) * (size_t)kThreads * D;
+    const Slices sl = slices(g, slice_keys<T, D>());
+    A.nF = sl.nF;
+    A.nR = sl.nR;
+    A.nparts = sl.nF + sl.nR;
+    const size_t vs_bytes = 2 * sizeof(T) * (size_t)slice_keys<T, D>() * D;
     cudaError_t e = ensure_smem((const void *)k_decode_fixed<T, D>, vs_bytes);
     if (e == cudaSuccess) e = ensure_smem((const void *)k_decode_b<T, D>, vs_bytes);
     if (e != cudaSuccess) return cuda_status(e);
@@ -697,7 +749,7 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kRouteSplits, g.Hkv, g.B);
+    cfg.gridDim = dim3(A.nR, g.Hkv, g.B);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = vs_bytes;
     cfg.stream = st;
@@ -708,7 +760,7 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     cfg.numAttrs = 1;
     if ((e = cudaLaunchKernelEx(&cfg, k_decode_b<T, D>, A)) != cudaSuccess) return cuda_status(e);
     if ((e = cudaStreamWaitEvent(sd->side, sd->fork, 0)) != cudaSuccess) return cuda_status(e);
-    k_decode_fixed<T, D><<<dim3(kFixSplits, g.Hkv, g.B), kThreads, vs_bytes, sd->side>>>(A);
+    k_decode_fixed<T, D><<<dim3(A.nF, g.Hkv, g.B), kThreads, vs_bytes, sd->side>>>(A);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     if ((e = cudaEventRecord(sd->join, sd->side)) != cudaSuccess) return cuda_status(e);
     return cuda_status(cudaStreamWaitEvent(st, sd->join, 0));
@@ -716,14 +768,11 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
 
 }  // namespace
 
-// Shapes the fixed-size tables hold: per CTA at most kThreads keys, the
-// merge and group candidates fit kMaxCand.
+// Shapes the fixed-size tables hold: the merge and group candidates fit
+// kMaxCand, the query heads of a KV head kMaxG.
 bool decode_supported(const Geo &g) {
     const long long ns = scan_splits(g);
-    const long long routed = min((long long)g.K_g * g.g_s, (long long)g.T);
-    return g.G <= kMaxG && ns * g.K_c <= kMaxCand && (long long)g.K_c * g.gpc <= kMaxCand &&
-           routed <= (long long)kRouteSplits * kThreads &&
-           (long long)(g.F + max(g.L, 1) + 1) * g.C <= (long long)kFixSplits * kThreads;
+    return g.G <= kMaxG && ns * g.K_c <= kMaxCand && (long long)g.K_c * g.gpc <= kMaxCand;
 }
 
 size_t decode_workspace_bytes(const Geo &g) { return layout(g).total; }

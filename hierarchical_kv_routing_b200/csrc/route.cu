@@ -18,7 +18,8 @@
 // scores it against all the run's routing queries (fp64 dot products, the
 // query broadcast from shared memory), which cuts the chunk table's L2
 // traffic by the run length; one warp per block then takes its top K_c
-// (warp bitonic sort and merge of packed (fp32 score, id) keys), scores the
+// (keys below a threshold that cannot reach the top K_c dropped first, then
+// warp bitonic sort and merge of packed (fp32 score, id) keys), scores the
 // groups of its chunks and takes the top K_g.  K above 32 falls back to
 // CTA-wide selection rounds, one block at a time.
 #include "hga_internal.cuh"
@@ -132,36 +133,52 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
     const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
     const int n_rows = max(0, middle_hi(c0 + nb - 1, A.L) - A.F + 1);
-    for (int r = threadIdx.x; r < n_rows; r += kThreads) {
-        const float4 *r4 = reinterpret_cast<const float4 *>(Sc + (int64_t)(A.F + r) * D);
-        double acc[kBlk];
+    // two rows per thread (r and r + kThreads): each query value read from
+    // shared memory (as a pair of dims) serves both rows
+    for (int r = threadIdx.x; r < n_rows; r += 2 * kThreads) {
+        const int r2 = r + kThreads;
+        const bool two = r2 < n_rows;
+        const float4 *ra = reinterpret_cast<const float4 *>(Sc + (int64_t)(A.F + r) * D);
+        const float4 *rb = reinterpret_cast<const float4 *>(Sc + (int64_t)(A.F + (two ? r2 : r)) * D);
+        double acc[kBlk], acc2[kBlk];
 #pragma unroll
-        for (int k = 0; k < kBlk; ++k) acc[k] = 0.0;
+        for (int k = 0; k < kBlk; ++k) acc[k] = acc2[k] = 0.0;
 #pragma unroll 1
-        for (int base = 0; base < D / 4; base += 8) {
-            float4 v[8];
+        for (int base = 0; base < D / 4; base += 4) {
+            float4 va[4], vb[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = __ldg(r4 + base + e);
+            for (int e = 0; e < 4; ++e) {
+                va[e] = __ldg(ra + base + e);
+                vb[e] = __ldg(rb + base + e);
+            }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < 4; ++e) {
                 const int d = 4 * (base + e);
 #pragma unroll
                 for (int k = 0; k < kBlk; ++k) {
                     if (k < nb) {
-                        const double *qk = qr + k * D + d;
-                        acc[k] = fma(qk[0], (double)v[e].x, acc[k]);
-                        acc[k] = fma(qk[1], (double)v[e].y, acc[k]);
-                        acc[k] = fma(qk[2], (double)v[e].z, acc[k]);
-                        acc[k] = fma(qk[3], (double)v[e].w, acc[k]);
+                        const double2 q01 = *reinterpret_cast<const double2 *>(qr + k * D + d);
+                        const double2 q23 = *reinterpret_cast<const double2 *>(qr + k * D + d + 2);
+                        acc[k] = fma(q01.x, (double)va[e].x, acc[k]);
+                        acc2[k] = fma(q01.x, (double)vb[e].x, acc2[k]);
+                        acc[k] = fma(q01.y, (double)va[e].y, acc[k]);
+                        acc2[k] = fma(q01.y, (double)vb[e].y, acc2[k]);
+                        acc[k] = fma(q23.x, (double)va[e].z, acc[k]);
+                        acc2[k] = fma(q23.x, (double)vb[e].z, acc2[k]);
+                        acc[k] = fma(q23.y, (double)va[e].w, acc[k]);
+                        acc2[k] = fma(q23.y, (double)vb[e].w, acc2[k]);
                     }
                 }
             }
         }
 #pragma unroll
         for (int k = 0; k < kBlk; ++k)
-            if (k < nb)
-                cand[k * A.ncap + r] = A.F + r <= middle_hi(c0 + k, A.L)
-                                           ? pack_key((float)acc[k], A.F + r) : 0ull;
+            if (k < nb) {
+                const int mh = middle_hi(c0 + k, A.L);
+                cand[k * A.ncap + r] = A.F + r <= mh ? pack_key((float)acc[k], A.F + r) : 0ull;
+                if (two)
+                    cand[k * A.ncap + r2] = A.F + r2 <= mh ? pack_key((float)acc2[k], A.F + r2) : 0ull;
+            }
     }
     __syncthreads();
 
@@ -170,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
         for (int k = warp; k < nb; k += kThreads / 32) {
             const int c = c0 + k;
             const int n_mid = max(0, middle_hi(c, A.L) - A.F + 1);
-            const unsigned long long top = warp_top32(cand + k * A.ncap, n_mid, 0, 1);
+            const unsigned long long top = warp_topk_filtered(cand + k * A.ncap, n_mid, A.K_c);
             const bool take = lane < A.K_c && top != 0ull;
             const int id = warp_sort_asc_int(take ? key_id(top) : 0x7fffffff);
             const int kc = min(A.K_c, n_mid);
@@ -194,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
         for (int k = warp; k < nb; k += kThreads / 32) {
             const int c = c0 + k;
             const int ng = kc_s[k] * A.gpc;
-            const unsigned long long top = warp_top32(cand + k * A.ncap, ng, 0, 1);
+            const unsigned long long top = warp_topk_filtered(cand + k * A.ncap, ng, A.K_g);
             const bool take = lane < A.K_g && top != 0ull;
             const int id = warp_sort_asc_int(take ? key_id(top) : 0x7fffffff);
             const int kg = min(A.K_g, ng);

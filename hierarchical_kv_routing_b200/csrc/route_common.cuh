@@ -199,6 +199,32 @@ __device__ __forceinline__ unsigned long long warp_top32(const unsigned long lon
     return acc;
 }
 
+// The warp's top 32 of n keys in shared memory, descending, where only the
+// top K (K <= 32) will be used.  At least K lanes hold a key as large as the
+// K-th largest of the lanes' maxima (tau), so every top-K key is >= tau:
+// the keys below tau are dropped first (cand is compacted in place), which
+// leaves the sort-and-merge rounds a few dozen keys instead of n.
+__device__ __forceinline__ unsigned long long warp_topk_filtered(unsigned long long *cand, int n,
+                                                                 int K) {
+    const int lane = threadIdx.x & 31;
+    if (n <= 64) return warp_top32(cand, n, 0, 1);
+    unsigned long long m = 0ull;
+    for (int i = lane; i < n; i += 32) m = cand[i] > m ? cand[i] : m;
+    const unsigned long long tau = __shfl_sync(0xffffffffu, warp_sort_desc(m), K - 1);
+    int w = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        const unsigned long long x = i < n ? cand[i] : 0ull;
+        const bool keep = x != 0ull && x >= tau;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        // writes land below base + 32: never on keys not read yet
+        if (keep) cand[w + __popc(bal & ((1u << lane) - 1u))] = x;
+        w += __popc(bal);
+        __syncwarp();
+    }
+    return warp_top32(cand, w, 0, 1);
+}
+
 // Top-K (K <= 32) of n candidate keys with the whole CTA: every warp reduces
 // its share to a sorted top 32, warp 0 merges them.  Writes the chosen ids
 // ascending to out (K entries, the unused ones -1); returns min(K, n).
@@ -292,6 +318,93 @@ __device__ __forceinline__ void block_topk32_keys(const unsigned long long *cand
         if (lane < K) out[lane] = acc;
     }
     __syncthreads();
+}
+
+}  // namespace hga
+
+namespace hga {
+
+// ---- selection by counting ranks (no dependent shuffle chains)
+
+// The K largest of n distinct candidate keys (0 = padding, never chosen) by
+// rank: a key is chosen when fewer than K keys exceed it.  top[0..K)
+// (shared) receives them descending, 0-padded.  Whole CTA.
+__device__ __forceinline__ void rank_topk(const unsigned long long *cand, int n, int K,
+                                          unsigned long long *top) {
+    for (int r = threadIdx.x; r < K; r += blockDim.x) top[r] = 0ull;
+    __syncthreads();
+    // four lanes per candidate, each counting a quarter of the others
+    const int part = threadIdx.x & 3;
+    for (int base = 0; base < n; base += (int)blockDim.x / 4) {
+        const int i = base + (int)threadIdx.x / 4;
+        const unsigned long long k = i < n ? cand[i] : 0ull;
+        int r = 0;
+        if (k) {
+            int j = part;
+            for (; j + 28 < n; j += 32) {      // eight loads in flight
+                unsigned long long c[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) c[u] = cand[j + 4 * u];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) r += c[u] > k;
+            }
+            for (; j < n; j += 4) r += cand[j] > k;
+        }
+        r += __shfl_xor_sync(0xffffffffu, r, 1);
+        r += __shfl_xor_sync(0xffffffffu, r, 2);
+        if (part == 0 && k && r < K) top[r] = k;
+    }
+    __syncthreads();
+}
+
+// The same over nl descending, 0-padded lists of len keys each (lists[b *
+// len + p]): a key's rank is the number of keys above it in every list,
+// found by binary search.  Whole CTA.
+__device__ __forceinline__ void rank_topk_lists(const unsigned long long *lists, int nl, int len,
+                                                int K, unsigned long long *top) {
+    for (int r = threadIdx.x; r < K; r += blockDim.x) top[r] = 0ull;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nl * len; i += blockDim.x) {
+        const unsigned long long x = lists[i];
+        if (!x) continue;
+        int r = 0;
+        for (int b = 0; b < nl; ++b) {
+            const unsigned long long *Lb = lists + b * len;
+            int lo = 0, hi = len;                 // first index whose key is not above x
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (Lb[mid] > x) lo = mid + 1;
+                else hi = mid;
+            }
+            r += lo;
+        }
+        if (r < K) top[r] = x;
+    }
+    __syncthreads();
+}
+
+// Ids of top[0..K) (descending keys, 0-padded) in ascending order into
+// out[0..K), the unused entries -1; returns how many were chosen.  Whole CTA.
+__device__ __forceinline__ int ids_ascending(const unsigned long long *top, int K, int *out) {
+    for (int i = threadIdx.x; i < K; i += blockDim.x) {
+        const unsigned long long k = top[i];
+        if (!k) {
+            out[i] = -1;
+            continue;
+        }
+        const int id = key_id(k);
+        int r = 0;
+#pragma unroll 8
+        for (int j = 0; j < K; ++j) {
+            const unsigned long long kj = top[j];
+            r += kj != 0ull && key_id(kj) < id;
+        }
+        out[r] = id;
+    }
+    __syncthreads();
+    int n = 0;
+    for (int i = 0; i < K; ++i) n += top[i] != 0ull;
+    return n;
 }
 
 }  // namespace hga
