@@ -365,7 +365,7 @@ def bench_decode(args, dev, world):
                        "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
                        "graph": f"{S} steps captured in one CUDA graph, lens reset between "
                                 "replays outside the timed events"},
-            "gpu_launches_per_step": 2,
+            "gpu_launches_per_step": 3,   # scan, fixed-key and routed slices
             "roofline": {"bound": "hbm", "achieved": achieved,
                          "peak": pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]), "unit": "GB/s",
                          "frac": achieved / pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]),
