@@ -191,19 +191,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
     }
     __syncthreads();
-    // cos/sin of every (token, pair) of this CTA's rows, shared by the G
-    // query heads of a token (each angle formed once instead of G times)
     const int tok0 = t0 + row0 / A.G;
     float2 *cs_tab = reinterpret_cast<float2 *>(smem + C::oCS);
-    if (A.cs_tokens > 0) {
-        // rows padded to H + 1 entries: the 4 tokens a warp reads differ in bank
-        constexpr int H = D / 2;
-        for (int e = threadIdx.x; e < A.cs_tokens * H; e += kThreads) {
-            const int tj = e / H;
-            if (tok0 + tj < A.T) cs_tab[tj * (H + 1) + e % H] = rope_cs_int(A.rope, ctl.s_pos[tj], e % H);
-        }
-        __syncthreads();
-    }
     tc_fence_after();
     // Registers: the producer / MMA warpgroup needs few, the two softmax
     // warpgroups hold a 128-column S row each.  128 x 56 + 256 x 224 equals
@@ -330,6 +319,19 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     } else {
         regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------- softmax --
+        // cos/sin of every (token, pair) of this CTA's rows, shared by the G
+        // query heads of a token (each angle formed once instead of G times);
+        // built by the softmax warps alone while the producers already load
+        // the first key and value tiles
+        if (A.cs_tokens > 0) {
+            // rows padded to H + 1 entries: the 4 tokens a warp reads differ in bank
+            constexpr int H = D / 2;
+            for (int e = threadIdx.x - 128; e < A.cs_tokens * H; e += kThreads - 128) {
+                const int tj = e / H;
+                if (tok0 + tj < A.T) cs_tab[tj * (H + 1) + e % H] = rope_cs_int(A.rope, ctl.s_pos[tj], e % H);
+            }
+            named_bar(1, kThreads - 128);
+        }
         const int mt = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
