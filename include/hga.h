@@ -177,7 +177,11 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   summaries of chunk t/C if t closes it (page section 3, store operation
  *   "append closed chunk"), routes with the token's own query (summed over the
  *   KV head's query heads), attends over the visible set of token t and
- *   increments lens[b].  Requires lens[b] < dims.T.
+ *   increments lens[b].  Requires lens[b] < dims.T.  The attention over the
+ *   keys routing does not choose (sinks, recent and current chunks) runs on
+ *   a library-owned side stream (one per device, created on the first decode
+ *   call) forked from and joined back into `stream` inside the call, so the
+ *   caller sees ordinary stream order and can capture steps in a CUDA graph.
  * HGA_PREFILL_HOSTKV: the prefill of HGA_PREFILL with the token K/V history
  *   in host RAM (page section 3, the three-tier K/V store: the summaries stay
  *   on the GPU and only routed groups are fetched).  io.k and io.v are HOST
