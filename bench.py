@@ -376,11 +376,11 @@ def bench_decode(args, dev, world):
 HOSTTIER_WORKLOAD = "qwen3_30b_a3b_bf16_hosttier_prefill_64k"
 
 
-def hosttier_link_bytes(w, sel_group):
-    """Algorithmic bytes over the host link for one host-tier prefill: raw K
-    once (summaries), K and V of every token once (sinks and fixed windows;
-    window chunks shared by consecutive waves move on the device), and K and
-    V of every routed group of every (block, KV head)."""
+def hosttier_link_bytes_uncached(w, sel_group):
+    """Bytes over the host link for one host-tier prefill without the warm
+    cache: raw K once (summaries), K and V of every token once (sinks and
+    fixed windows; window chunks shared by consecutive waves move on the
+    device), and K and V of every routed group of every (block, KV head)."""
     row = w.Hkv * w.D * 2
     routed = int((sel_group >= 0).sum().item()) * w.g_s * w.D * 2 * 2
     return w.B * w.T * row + 2 * w.B * w.T * row + routed
@@ -404,10 +404,11 @@ def bench_hosttier(args, dev, world):
     ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     res = hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, want_sel=True, workspace=ws)
-    link = hosttier_link_bytes(w, res["sel_group"])
+    uncached = hosttier_link_bytes_uncached(w, res["sel_group"])
     for _ in range(max(2, min(args.warmup, 3))):
         hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
     torch.cuda.synchronize(dev)
+    hga.hga_hostkv_link_bytes(clear=True)
     if world > 1:
         dist.barrier()
     steps = 5
@@ -418,6 +419,9 @@ def bench_hosttier(args, dev, world):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
+    # bytes read over the link per call: the gathers' own count (sinks,
+    # windows, warm-cache misses) plus stage 1's single pass over raw K
+    link = hga.hga_hostkv_link_bytes(clear=True) / steps + w.B * w.T * w.Hkv * w.D * 2
     # host-to-device peak of this machine: copy engine, pinned source, 256 MiB
     src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
     dst = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -434,10 +438,12 @@ def bench_hosttier(args, dev, world):
             "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
             "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
                        "D": w.D, "K_c": w.K_c, "K_g": w.K_g,
-                       "tier": "raw K and V in pinned host RAM; summaries, Q, O and two "
-                               "32-block staging buffers in HBM"},
+                       "tier": "raw K and V in pinned host RAM; summaries, Q, O, two "
+                               "32-block staging buffers and a warm cache of routed groups "
+                               "in HBM"},
             "roofline": {"bound": "host link", "achieved": achieved, "peak": best,
                          "unit": "GB/s", "frac": achieved / best, "bytes_per_step": link,
+                         "bytes_per_step_without_cache": uncached,
                          "peak_source": "measured in this run: pinned host -> device copy "
                                         "of 256 MiB, best of 5"}}
 

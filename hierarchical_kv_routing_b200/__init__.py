@@ -24,7 +24,7 @@ __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "h
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
            "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
            "decode_workspace", "hga_forward_prefill_hostkv", "HGAError", "PREFILL",
-           "DECODE", "PREFILL_HOSTKV", "hga_device_status"]
+           "DECODE", "PREFILL_HOSTKV", "hga_device_status", "hga_hostkv_link_bytes"]
 
 PREFILL, DECODE, PREFILL_HOSTKV = 0, 1, 2
 _F32, _BF16 = 0, 1
@@ -113,6 +113,8 @@ def load():
         lib.hga_last_cuda_error.restype = ctypes.c_int
         lib.hga_device_status.argtypes = [P, ctypes.c_int]
         lib.hga_device_status.restype = ctypes.c_int
+        lib.hga_hostkv_link_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
+        lib.hga_hostkv_link_bytes.restype = ctypes.c_int
         for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -245,6 +247,17 @@ def hga_device_status(clear: bool = True, stream=None) -> int:
     access).  Waits for the work queued on `stream`."""
     lib = load()
     return int(lib.hga_device_status(_stream(stream), 1 if clear else 0))
+
+
+def hga_hostkv_link_bytes(clear: bool = True, stream=None) -> int:
+    """Bytes the host tier's stage 3 has read over the host link since the
+    last reset (sinks, windows and the routed groups its warm cache missed).
+    Waits for the work queued on `stream`."""
+    lib = load()
+    v = ctypes.c_ulonglong(0)
+    _check(lib.hga_hostkv_link_bytes(_stream(stream), ctypes.byref(v), 1 if clear else 0),
+           "hga_hostkv_link_bytes")
+    return int(v.value)
 
 
 def hga_workspace_size(mode: int, B: int, T: int, Hq: int, Hkv: int, D: int, dtype,

@@ -283,12 +283,18 @@ int hga_last_cuda_error(void) { return g_last_cuda_error; }
 hga_status hga_device_status(void *stream, int clear) {
     const cudaStream_t st = (cudaStream_t)stream;
     hga_status first = HGA_OK;
-    const hga_status parts[3] = {summaries_error_take(st, clear != 0),
+    const hga_status parts[4] = {summaries_error_take(st, clear != 0),
                                  attend_tc_error_take(st, clear != 0),
-                                 decode_error_take(st, clear != 0)};
+                                 decode_error_take(st, clear != 0),
+                                 tier_error_take(st, clear != 0)};
     for (hga_status p : parts)
         if (p != HGA_OK && first == HGA_OK) first = p;
     return first;
+}
+
+hga_status hga_hostkv_link_bytes(void *stream, unsigned long long *bytes, int clear) {
+    if (!bytes) return HGA_ERR_INVALID_ARG;
+    return tier_link_bytes_take((cudaStream_t)stream, bytes, clear != 0);
 }
 
 }  // extern "C"

@@ -75,11 +75,12 @@ struct TcArgs {
     int rows_per_unit, ctas_per_unit, tokM;
     int cs_tokens;            // > 0: the CTA's (token, pair) cos/sin table is in smem
     int c0;                   // first query block of this launch
-    // Host-resident tier: K/V rows come from a wave's staging buffer, not from
-    // the token layout.  Tokens below sink_rows sit at row = token; other
-    // tokens at row = win_row0 + token - win_tok0; group slot j of block c at
-    // rows rt_row0 + ((c - c0) * K_g + j) * g_s.
-    int tier, sink_rows, win_tok0, win_row0, rt_row0;
+    // Host-resident tier: K/V rows come from the tier's buffers, not from the
+    // token layout.  Tokens below sink_rows sit at row buf_row0 + token, other
+    // fixed tokens at buf_row0 + win_row0 + token - win_tok0; routed group
+    // slot j of (block c, head h, sequence b) at the row rt_map gives.
+    int tier, sink_rows, win_tok0, win_row0, buf_row0, rt_W;
+    const int32_t *rt_map;
     const int32_t *sel_group;
     const int32_t *pos;
     __nv_bfloat16 *out;
@@ -165,7 +166,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int n_fixed = 8 * (nsink + (c - rec_lo));
         // load row of a token: itself, or its place in the tier's window
         auto row_of = [&](int tok) {
-            return (!A.tier || tok < A.sink_rows) ? tok : A.win_row0 + tok - A.win_tok0;
+            return !A.tier ? tok
+                           : A.buf_row0 + (tok < A.sink_rows ? tok : A.win_row0 + tok - A.win_tok0);
         };
         for (int s = lane; s < n_fixed; s += 32)
             ctl.seg_tok[s] = row_of(s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8);
@@ -177,7 +179,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             kg += __popc(__ballot_sync(0xffffffffu, v >= 0));
         }
         for (int j = lane; j < kg; j += 32) {
-            const int r0 = A.tier ? A.rt_row0 + ((c - A.c0) * A.K_g + j) * A.g_s : sel[j] * A.g_s;
+            const int r0 = A.tier ? A.rt_map[(((int64_t)b * A.rt_W + (c - A.c0)) * A.Hkv + h) * A.K_g + j]
+                                  : sel[j] * A.g_s;
             for (int e = 0; e < gseg; ++e) ctl.seg_tok[n_fixed + j * gseg + e] = r0 + e * 8;
         }
         const int n_route = n_fixed + kg * gseg;
@@ -542,7 +545,9 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     a.sink_rows = tw ? tw->sink_rows : 0;
     a.win_tok0 = tw ? tw->win_tok0 : 0;
     a.win_row0 = tw ? tw->win_row0 : 0;
-    a.rt_row0 = tw ? tw->rt_row0 : 0;
+    a.buf_row0 = tw ? tw->buf_row0 : 0;
+    a.rt_W = tw ? tw->rt_W : 0;
+    a.rt_map = tw ? tw->rt_map : nullptr;
     const int nblk = tw ? tw->c1 - tw->c0 : g.NB;
     a.T = g.T;
     a.Hq = g.Hq;

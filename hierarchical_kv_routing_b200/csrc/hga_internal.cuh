@@ -150,8 +150,14 @@ bool attend_tc_supported(const Geo &g, int dtype);
 // tokens below sink_rows at row = token, other fixed-window and current
 // tokens at row = win_row0 + token - win_tok0, and group slot j of block c at
 // rows rt_row0 + ((c - c0) * K_g + j) * g_s (slot j holds the j-th routed id).
+// One wave of the host tier: blocks [c0, c1); sinks and the recent/current
+// window sit in a staging buffer starting at row buf_row0 (token tok < sink_rows
+// at buf_row0 + tok, others at buf_row0 + win_row0 + tok - win_tok0); routed
+// group slot j of (block c, KV head h, sequence b) starts at row
+// rt_map[((b * rt_W + c - c0) * Hkv + h) * K_g + j] (the group cache).
 struct TierWave {
-    int c0, c1, sink_rows, win_tok0, win_row0, rt_row0;
+    int c0, c1, sink_rows, win_tok0, win_row0, buf_row0, rt_W;
+    const int32_t *rt_map;
 };
 
 // tw == nullptr: every query block, keys at their token rows.
@@ -170,6 +176,8 @@ hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, 
 hga_status attend_tc_error_take(cudaStream_t st, bool clear);
 hga_status decode_error_take(cudaStream_t st, bool clear);
 hga_status summaries_error_take(cudaStream_t st, bool clear);
+hga_status tier_error_take(cudaStream_t st, bool clear);
+hga_status tier_link_bytes_take(cudaStream_t st, unsigned long long *bytes, bool clear);
 
 // Decode step (append, close-chunk summaries, route, split attention).
 size_t decode_workspace_bytes(const Geo &g);

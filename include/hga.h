@@ -191,12 +191,17 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   pointers; io.cache must be empty.  bf16 only, shapes the tensor-core
  *   attention takes (g_s a multiple of 8, Hq/Hkv a power of two <= 16).
  *   Stage 1 reads K over the host link once; stage 3 runs in waves of 32
- *   query blocks whose sink, recent, current and routed K/V rows are fetched
- *   by the GPU over the link into two HBM staging buffers in the workspace,
- *   on a library-owned side stream (one per device, created on the first
- *   such call), the next wave's fetch overlapping this wave's attention; the
- *   call joins that stream back into `stream` before returning, so the
- *   caller sees ordinary stream order.  Host memory that is not pinned and
+ *   query blocks whose sink, recent and current K/V rows are fetched by the
+ *   GPU over the link into two HBM staging buffers in the workspace, and
+ *   whose routed groups go through a warm tier: a cache of routed groups in
+ *   the workspace (page section 3's warm VRAM tier; CLOCK replacement, two
+ *   waves' worth of groups per sequence and KV head, or all of them when
+ *   fewer) from which hits are read and into which misses are fetched.
+ *   This runs on a library-owned side stream (one per device, created on
+ *   the first such call), the next wave's fetch overlapping this wave's
+ *   attention; the call joins that stream back into `stream` before
+ *   returning, so the caller sees ordinary stream order.  The cache lives
+ *   for one call.  Host memory that is not pinned and
  *   mapped returns HGA_ERR_INVALID_ARG.  The outputs equal HGA_PREFILL's.
  * workspace: hga_workspace_size(mode) bytes of device memory, 256-byte
  * aligned.  For HGA_DECODE it must be zero-filled before its first use; the
@@ -243,6 +248,13 @@ hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hga_params *p
  * clear != 0 resets them.  Returns HGA_OK when none is set, the first set
  * status otherwise, or HGA_ERR_CUDA if the copies fail. */
 hga_status hga_device_status(void *stream, int clear);
+
+/* Bytes the host tier (HGA_PREFILL_HOSTKV) has read over the host link for
+ * stage 3 since the last reset: the K and V rows of sinks, windows and the
+ * routed groups its warm cache did not hold (stage 1's single pass over K is
+ * not counted).  Waits for the work queued on `stream`; clear != 0 resets the
+ * count.  *bytes must be a host pointer (HGA_ERR_INVALID_ARG if NULL). */
+hga_status hga_hostkv_link_bytes(void *stream, unsigned long long *bytes, int clear);
 
 /* Static description of a status code. */
 const char *hga_status_string(hga_status s);

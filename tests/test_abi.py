@@ -101,9 +101,12 @@ def test_hostkv_mode_host_checks(lib):
     p = hga.HGAParams(F=2, L=8, K_c=16, K_g=32, rope_theta=1e6).c()
     d = _dims(T=4096, Hq=32, Hkv=4, D=128, dtype=1)
     n = lib.hga_workspace_size(2, ctypes.byref(d), ctypes.byref(p))
-    # two staging buffers of K and V for a 32-block wave dominate
-    rows = 2 * 64 + (32 + 8) * 64 + 32 * 32 * 16
-    assert n >= 4 * rows * 4 * 128 * 2
+    # the K and V row spaces dominate: two staging buffers (sinks and the
+    # window of a 32-block wave) and the group cache (every group of the
+    # 64 chunks here, fewer than two waves' worth of routed groups)
+    groups = min(64 * (64 // 16), 2 * 32 * 32)
+    rows = 2 * (2 * 64 + (32 + 8) * 64) + groups * 16
+    assert n >= 2 * rows * 4 * 128 * 2
     io = hga._IO()
     fake = ctypes.c_void_p(1 << 20)
     st = lib.hga_forward(2, ctypes.byref(d), ctypes.byref(p), ctypes.byref(io), fake, n, None)

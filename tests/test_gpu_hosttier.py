@@ -6,7 +6,9 @@ The tier runs the same arithmetic as the in-HBM prefill (keys are rotated
 with the same rounding when they are fetched), so its routed sets and
 outputs must equal that path's bit for bit; outputs are also checked against
 the CPU oracle on the routed sets.  Cases span several waves (32 blocks
-each), a ragged last block, F = 0 / L = 0, MHA with D = 64 and B > 1.
+each), a ragged last block, F = 0 / L = 0, MHA with D = 64, B > 1 and a warm
+cache smaller than the sequence's groups; the bytes the tier reads over the
+link are checked against bounds that follow from the routed sets.
 """
 import numpy as np
 import pytest
@@ -28,6 +30,9 @@ CASES = {
     "qwen_F0_L0": QWEN.replace(T=64 * 40, F=0, L=0, K_c=5, K_g=9),
     "smalllm_B2_D64": SMALLLM.replace(B=2, T=64 * 66),
     "qwen_L1_F3": QWEN.replace(T=64 * 33 + 5, F=3, L=1, K_c=4, K_g=7),
+    # 800 groups per KV head against a warm cache of two waves' worth
+    # (2 x 32 x 3 = 192 slots): slots are evicted and reused across 7 waves
+    "qwen_cache_evicts": QWEN.replace(T=64 * 200, K_c=2, K_g=3),
 }
 
 
@@ -129,3 +134,52 @@ def test_hosttier_64k_full_size(gpu_lib):
     (q, k, v, pos), ref, tier = _run_pair(gpu_lib, w, seed=13)
     assert torch.equal(tier["sel_group"], ref["sel_group"])
     assert torch.equal(_bits(tier["out"]), _bits(ref["out"]))
+
+
+def _fixed_link_bytes(w, T):
+    """Bytes of sinks and windows the gathers read from host memory: the sink
+    chunks for each of the first two waves, and each wave's window minus the
+    tokens the previous wave's buffer already holds (same wave plan as the
+    library: 32-block waves, window from max(c0 - max(L, 1), F) to c1)."""
+    C, NB, Lw = w.C, (T + w.C - 1) // w.C, max(w.L, 1)
+    row = w.Hkv * w.D * 2 * 2                     # K and V of one token, all heads
+    tokens, prev = 0, (0, 0)
+    for wave, c0 in enumerate(range(0, NB, 32)):
+        c1 = min(c0 + 32, NB)
+        if wave < 2:
+            tokens += min(w.F * C, T)
+        nsink = min(c0, w.F)
+        wlo = max(max(c0 - Lw, nsink), w.F)
+        t0, t1 = wlo * C, max(min(c1 * C, T), wlo * C)
+        held = max(0, min(t1, prev[1]) - max(t0, prev[0])) if wave > 0 else 0
+        tokens += (t1 - t0) - held
+        prev = (t0, t1)
+    return w.B * tokens * row
+
+
+def test_hosttier_warm_cache_link_bytes(gpu_lib):
+    """The warm cache's traffic: every distinct routed group crosses the link
+    at least once, and no group twice within a wave (at most the sum over
+    waves of the wave's distinct groups); hits across waves make it less."""
+    w = QWEN.replace(T=64 * 200, K_c=2, K_g=3)
+    (q, k, v, pos), ref, tier = _run_pair(gpu_lib, w, seed=11)
+    assert torch.equal(_bits(tier["out"]), _bits(ref["out"]))
+    dev = torch.device("cuda")
+    gpu_lib.hga_hostkv_link_bytes(clear=True)
+    gpu_lib.hga_forward_prefill_hostkv(q.to(dev), k.pin_memory(), v.pin_memory(), pos.to(dev),
+                                       _hp(w))
+    got = gpu_lib.hga_hostkv_link_bytes(clear=True)
+    assert gpu_lib.hga_device_status(clear=True) == 0
+    sg = tier["sel_group"].cpu().numpy()          # [B, NB, Hkv, K_g]
+    group = w.g_s * w.D * 2 * 2                   # K and V rows of one group, one head
+    lower = upper = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            ids = sg[b, :, h, :]
+            lower += np.unique(ids[ids >= 0]).size
+            for c0 in range(0, ids.shape[0], 32):
+                wv = ids[c0:c0 + 32]
+                upper += np.unique(wv[wv >= 0]).size
+    routed = got - _fixed_link_bytes(w, w.T)
+    assert lower * group <= routed <= upper * group, (lower, routed / group, upper)
+    assert routed < upper * group          # some groups are served from the cache
