@@ -79,7 +79,7 @@ struct TcArgs {
     // token layout.  Tokens below sink_rows sit at row buf_row0 + token, other
     // fixed tokens at buf_row0 + win_row0 + token - win_tok0; routed group
     // slot j of (block c, head h, sequence b) at the row rt_map gives.
-    int tier, sink_rows, win_tok0, win_row0, buf_row0, rt_W;
+    int sink_rows, win_tok0, win_row0, buf_row0, rt_W;
     const int32_t *rt_map;
     const int32_t *sel_group;
     const int32_t *pos;
@@ -99,7 +99,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int D>
+// kTier: keys come from the host tier's buffers and group cache (TcArgs tier
+// fields) instead of the token layout; a separate instantiation, so the
+// in-HBM prefill's code is not touched by it.
+template <int D, bool kTier>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
@@ -166,8 +169,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int n_fixed = 8 * (nsink + (c - rec_lo));
         // load row of a token: itself, or its place in the tier's window
         auto row_of = [&](int tok) {
-            return !A.tier ? tok
-                           : A.buf_row0 + (tok < A.sink_rows ? tok : A.win_row0 + tok - A.win_tok0);
+            if constexpr (kTier)
+                return A.buf_row0 + (tok < A.sink_rows ? tok : A.win_row0 + tok - A.win_tok0);
+            else
+                return tok;
         };
         for (int s = lane; s < n_fixed; s += 32)
             ctl.seg_tok[s] = row_of(s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8);
@@ -179,8 +184,11 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             kg += __popc(__ballot_sync(0xffffffffu, v >= 0));
         }
         for (int j = lane; j < kg; j += 32) {
-            const int r0 = A.tier ? A.rt_map[(((int64_t)b * A.rt_W + (c - A.c0)) * A.Hkv + h) * A.K_g + j]
-                                  : sel[j] * A.g_s;
+            int r0;
+            if constexpr (kTier)
+                r0 = A.rt_map[(((int64_t)b * A.rt_W + (c - A.c0)) * A.Hkv + h) * A.K_g + j];
+            else
+                r0 = sel[j] * A.g_s;
             for (int e = 0; e < gseg; ++e) ctl.seg_tok[n_fixed + j * gseg + e] = r0 + e * 8;
         }
         const int n_route = n_fixed + kg * gseg;
@@ -541,7 +549,6 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
                cudaStream_t st, const TierWave *tw) {
     TcArgs a;
     a.c0 = tw ? tw->c0 : 0;
-    a.tier = tw != nullptr;
     a.sink_rows = tw ? tw->sink_rows : 0;
     a.win_tok0 = tw ? tw->win_tok0 : 0;
     a.win_row0 = tw ? tw->win_row0 : 0;
@@ -585,7 +592,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         !make_map(&mv64, v, D, g.Hkv, (long long)g.B * v_T, 1, 64))
         return HGA_ERR_CUDA;
     const size_t smem = Cfg<D>::oEnd + 1024 + (size_t)a.cs_tokens * (D / 2 + 1) * sizeof(float2);
-    auto kern = k_attend_tc<D>;
+    auto kern = tw ? k_attend_tc<D, true> : k_attend_tc<D, false>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(nblk * a.ctas_per_unit, g.Hkv, g.B);
