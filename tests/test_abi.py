@@ -117,3 +117,10 @@ def test_hostkv_mode_host_checks(lib):
     n32 = lib.hga_workspace_size(2, ctypes.byref(d32), ctypes.byref(p))
     st = lib.hga_forward(2, ctypes.byref(d32), ctypes.byref(p), ctypes.byref(io), fake, n32, None)
     assert st == 2
+
+
+def test_hostkv_link_bytes_checks_its_pointer(lib):
+    """hga_hostkv_link_bytes refuses a null result pointer before any CUDA call."""
+    lib.hga_hostkv_link_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    lib.hga_hostkv_link_bytes.restype = ctypes.c_int
+    assert lib.hga_hostkv_link_bytes(None, None, 0) == 1     # HGA_ERR_INVALID_ARG
