@@ -183,3 +183,57 @@ def test_hosttier_warm_cache_link_bytes(gpu_lib):
     routed = got - _fixed_link_bytes(w, w.T)
     assert lower * group <= routed <= upper * group, (lower, routed / group, upper)
     assert routed < upper * group          # some groups are served from the cache
+
+
+def _clock_misses(sel_group, W, NS):
+    """Misses of the warm tier's policy, replayed in plain Python: per wave the
+    distinct routed groups, ascending; hits keep their slot; misses, ascending,
+    take the first slots from the hand on that are free or were last used
+    before the previous wave; the hand moves past the last slot taken."""
+    B, NB, Hkv, _ = sel_group.shape
+    misses = 0
+    for b in range(B):
+        for h in range(Hkv):
+            slot_of, gid_of, stamp, hand = {}, [-1] * NS, [0] * NS, 0
+            for wave, c0 in enumerate(range(0, NB, W)):
+                ids = sel_group[b, c0:c0 + W, h, :].ravel()
+                uniq = sorted(set(int(x) for x in ids if x >= 0))
+                miss = []
+                for g in uniq:
+                    if g in slot_of:
+                        stamp[slot_of[g]] = wave
+                    else:
+                        miss.append(g)
+                victims = []
+                for k in range(NS):
+                    if len(victims) == len(miss):
+                        break
+                    s = (hand + k) % NS
+                    if gid_of[s] < 0 or stamp[s] < wave - 1:
+                        victims.append(s)
+                assert len(victims) == len(miss)
+                for s in victims:
+                    if gid_of[s] >= 0:
+                        del slot_of[gid_of[s]]
+                for s, g in zip(victims, miss):
+                    slot_of[g], gid_of[s], stamp[s] = s, g, wave
+                if victims:
+                    hand = (victims[-1] + 1) % NS
+                misses += len(miss)
+    return misses
+
+
+def test_hosttier_warm_cache_follows_clock(gpu_lib):
+    """The link bytes equal the sinks and windows plus exactly the misses the
+    CLOCK policy has on these routed sets (a cache of 192 slots per KV head
+    for 800 groups, so slots are evicted)."""
+    w = QWEN.replace(T=64 * 200, K_c=2, K_g=3)
+    (q, k, v, pos), ref, tier = _run_pair(gpu_lib, w, seed=17)
+    dev = torch.device("cuda")
+    gpu_lib.hga_hostkv_link_bytes(clear=True)
+    gpu_lib.hga_forward_prefill_hostkv(q.to(dev), k.pin_memory(), v.pin_memory(), pos.to(dev),
+                                       _hp(w))
+    got = gpu_lib.hga_hostkv_link_bytes(clear=True)
+    ns = min((w.T // w.C) * (w.C // w.g_s), 2 * 32 * w.K_g)
+    misses = _clock_misses(tier["sel_group"].cpu().numpy(), 32, ns)
+    assert got == _fixed_link_bytes(w, w.T) + misses * w.g_s * w.D * 2 * 2
