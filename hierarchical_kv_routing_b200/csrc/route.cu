@@ -22,6 +22,11 @@
 // warp bitonic sort and merge of packed (fp32 score, id) keys), scores the
 // groups of its chunks and takes the top K_g.  K above 32 falls back to
 // CTA-wide selection rounds, one block at a time.
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <utility>
+
 #include "hga_internal.cuh"
 #include "route_common.cuh"
 
@@ -247,6 +252,51 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     }
 }
 
+// Run length for the grid: CTAs = ceil(NB / n) runs x Hkv x B.  When the
+// grid fits in one wave of resident CTAs, take the n that minimises the
+// query blocks of the busiest SM (its CTA count times n), ties to the longer
+// run (fewer reads of the chunk table); otherwise the longest run.  Every
+// block's routing is computed the same way whatever run it falls in, so n
+// changes the schedule, never a result.
+int pick_run(int NB, int units, int nmax, int sms, int per_sm) {
+    const long long slots = (long long)sms * per_sm;
+    int best = nmax;
+    long long best_cost = -1;
+    for (int n = nmax; n >= 1; --n) {
+        const long long ctas = (long long)((NB + n - 1) / n) * units;
+        if (ctas > slots) break;                      // shorter runs only add CTAs
+        const long long cost = (long long)n * ((ctas + sms - 1) / sms);
+        if (best_cost < 0 || cost < best_cost) {
+            best = n;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// SM count and resident CTAs per SM of `kern` at `smem` bytes on the current
+// device (looked up once per kernel, size and device).
+cudaError_t residency(const void *kern, size_t smem, int *sms, int *per_sm) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, size_t, int>, std::pair<int, int>> seen;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(kern, smem, dev);
+    auto it = seen.find(key);
+    if (it == seen.end()) {
+        int n = 0, k = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&k, kern, kThreads, smem);
+        if (e != cudaSuccess) return e;
+        it = seen.emplace(key, std::make_pair(n, k)).first;
+    }
+    *sms = it->second.first;
+    *per_sm = it->second.second;
+    return cudaSuccess;
+}
+
 template <typename T, int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                const float *s_chunk, const float *s_group, int nc_cap, int32_t *sel_chunk,
@@ -269,16 +319,22 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     a.ncap = (int)max(max((long long)g.NC, 1ll), (long long)min(g.K_c, g.NC) * g.gpc);
     const size_t row_bytes = sizeof(unsigned long long) * (size_t)a.ncap;
     if (row_bytes > kCandBytes) return HGA_ERR_UNSUPPORTED;   // must fit on chip
-    a.nblk = (int)min((size_t)kBlk, kCandBytes / row_bytes);
+    const int nmax = (int)min((size_t)kBlk, kCandBytes / row_bytes);
     a.s_chunk = s_chunk;
     a.s_group = s_group;
     a.sel_chunk = sel_chunk;
     a.sel_group = sel_group;
     a.rope = r;
-    const size_t smem = sizeof(double) * kBlk * D + row_bytes * a.nblk;
+    // shared memory sized for the longest run, so the residency does not
+    // depend on the run length picked below
+    const size_t smem = sizeof(double) * kBlk * D + row_bytes * nmax;
     auto kern = k_route<T, D>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
+    int sms = 0, per_sm = 0;
+    e = residency((const void *)kern, smem, &sms, &per_sm);
+    if (e != cudaSuccess) return cuda_status(e);
+    a.nblk = per_sm > 0 ? pick_run(g.NB, g.Hkv * g.B, nmax, sms, per_sm) : nmax;
     dim3 grid((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
     kern<<<grid, kThreads, smem, st>>>(a);
     return cuda_status(cudaGetLastError());
