@@ -3,8 +3,9 @@
 // enqueued on the caller's stream.
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
-#include <unordered_map>
+#include <utility>
 
 #include "hga_internal.cuh"
 #include "route_common.cuh"
@@ -19,11 +20,16 @@ hga_status cuda_status(cudaError_t e) {
     return HGA_ERR_CUDA;
 }
 
+// The opt-in belongs to the kernel as loaded on one device, so the record of
+// what was granted is kept per (kernel, device).
 cudaError_t ensure_smem(const void *kernel, size_t bytes) {
     static std::mutex mu;
-    static std::unordered_map<const void *, size_t> granted;
+    static std::map<std::pair<const void *, int>, size_t> granted;
+    int dev = 0;
+    const cudaError_t de = cudaGetDevice(&dev);
+    if (de != cudaSuccess) return de;
     std::lock_guard<std::mutex> lock(mu);
-    size_t &have = granted[kernel];
+    size_t &have = granted[std::make_pair(kernel, dev)];
     if (bytes <= have) return cudaSuccess;
     const cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);

@@ -678,7 +678,14 @@ cudaError_t decode_side(int dev, DecodeSide **out) {
         cudaError_t e = cudaStreamCreateWithFlags(&d.side, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) {
+            // release what was made, so a later call starts from nothing
+            if (d.join) cudaEventDestroy(d.join);
+            if (d.fork) cudaEventDestroy(d.fork);
+            if (d.side) cudaStreamDestroy(d.side);
+            d = DecodeSide();
+            return e;
+        }
         d.ready = true;
     }
     *out = &d;

@@ -366,7 +366,17 @@ cudaError_t side_resources(int dev, SideRes **out) {
             e = cudaEventCreateWithFlags(&s.ready_ev[i], cudaEventDisableTiming);
             if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.free_ev[i], cudaEventDisableTiming);
         }
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) {
+            // release what was made, so a later call starts from nothing
+            for (int i = 0; i < 2; ++i) {
+                if (s.free_ev[i]) cudaEventDestroy(s.free_ev[i]);
+                if (s.ready_ev[i]) cudaEventDestroy(s.ready_ev[i]);
+            }
+            if (s.start) cudaEventDestroy(s.start);
+            if (s.side) cudaStreamDestroy(s.side);
+            s = SideRes();
+            return e;
+        }
         s.ready = true;
     }
     *out = &s;
