@@ -46,6 +46,28 @@ struct RouteArgs {
     Rope rope;
 };
 
+// Run and (KV head, sequence) unit of the CTA at linear index lin, for R
+// runs per unit and U units.  Chunk-scoring work grows with the run index
+// (a later run has more middle chunks), and CTAs start about in linear order,
+// two to an SM.  So the lightest run is paired with the heaviest, the next
+// lightest with the next heaviest, and so on; the two members of pair i sit
+// at linear indices i and i + N/2, and which of them takes the heavy run
+// alternates with i, so that CTAs adjacent in linear order and CTAs N/2
+// apart both hold complementary work.  With N odd the median CTA comes last.
+__host__ __device__ __forceinline__ void pair_slot(int lin, int R, int U, int *run, int *unit) {
+    const int N = R * U, P = N / 2;
+    int j;                                     // position in run-major order
+    if (lin >= 2 * P) {
+        j = P;
+    } else {
+        const int i = lin < P ? lin : lin - P;
+        const bool heavy = ((i & 1) == 0) == (lin < P);
+        j = heavy ? N - 1 - i : i;
+    }
+    *run = j / U;
+    *unit = j % U;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     constexpr int H = D / 2;
@@ -62,8 +84,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     __shared__ unsigned long long lists[kThreads];
     __shared__ RouteScratch rs;
 
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int c0 = blockIdx.x * A.nblk;
+    int run, unit;
+    pair_slot((int)((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x), (int)gridDim.x,
+              (int)(gridDim.y * gridDim.z), &run, &unit);
+    const int h = unit % (int)gridDim.y, b = unit / (int)gridDim.y;
+    const int c0 = run * A.nblk;
     const int nb = min(A.nblk, A.NB - c0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const T *q = static_cast<const T *>(A.q);
