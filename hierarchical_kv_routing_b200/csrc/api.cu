@@ -1,6 +1,7 @@
 // The C ABI of include/hga.h: host-side argument checks, workspace layout and
 // kernel dispatch.  Nothing here allocates device memory; every kernel is
 // enqueued on the caller's stream.
+#include <climits>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -56,6 +57,8 @@ namespace {
 
 inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+constexpr int kMaxGridYZ = 65535;
+
 hga_status check_common(const hga_dims *d, const hga_params *p) {
     if (!d || !p) return HGA_ERR_INVALID_ARG;
     if (d->B < 1 || d->T < 0 || d->Hq < 1 || d->Hkv < 1 || d->Hq % d->Hkv) return HGA_ERR_INVALID_ARG;
@@ -65,6 +68,10 @@ hga_status check_common(const hga_dims *d, const hga_params *p) {
     if (!(p->rope_theta > 1.0) || !std::isfinite(p->rope_theta) || std::isnan(p->hf_wavelength))
         return HGA_ERR_INVALID_ARG;
     if (d->D != 64 && d->D != 128) return HGA_ERR_UNSUPPORTED;
+    // B and Hkv index grid axes (65535 at most); token rows b * T + t are
+    // 32-bit tensor-map coordinates
+    if (d->B > kMaxGridYZ || d->Hkv > kMaxGridYZ || (long long)d->B * d->T > (long long)INT32_MAX)
+        return HGA_ERR_UNSUPPORTED;
     if (p->C != kChunk) return HGA_ERR_UNSUPPORTED;
     if (p->K_c > kMaxK || p->K_g > kMaxK) return HGA_ERR_UNSUPPORTED;
     return HGA_OK;
@@ -219,6 +226,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
             return HGA_ERR_INVALID_ARG;
         if (!fill_only && !ws_ok) return HGA_ERR_WORKSPACE;   // fill only needs none
         if (fill) {
+            if ((long long)dims->B * cc.capacity > (long long)INT32_MAX) return HGA_ERR_UNSUPPORTED;
             if (cc.capacity < dims->T || cc.capacity % prm->C || !cc.v || !cc.pos || !cc.k_open ||
                 !cc.s_chunk || !cc.s_group || !cc.lens)
                 return HGA_ERR_INVALID_ARG;

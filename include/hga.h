@@ -37,6 +37,8 @@
  *    wider.
  *  - Errors: arguments are checked on the host first; a failing check
  *    returns HGA_ERR_INVALID_ARG or HGA_ERR_UNSUPPORTED and launches nothing.
+ *    Size limits of this build (HGA_ERR_UNSUPPORTED beyond them): B <= 65535,
+ *    Hkv <= 65535, and B * T (B * capacity for a K/V cache) below 2^31.
  *    A launch failure returns HGA_ERR_CUDA (the CUDA error is not cleared by
  *    the library; hga_last_cuda_error() gives its code).
  */

@@ -52,7 +52,8 @@ def test_workspace_size_host_only(lib):
 
 
 @pytest.mark.parametrize("bad,code", [
-    (dict(D=96), 2), (dict(Hq=3, Hkv=2), 1), (dict(dtype=7), 1), (dict(B=0), 1)])
+    (dict(D=96), 2), (dict(Hq=3, Hkv=2), 1), (dict(dtype=7), 1), (dict(B=0), 1),
+    (dict(B=65536, T=64), 2), (dict(Hq=65536, Hkv=65536), 2), (dict(B=2, T=1 << 30), 2)])
 def test_bad_dims_rejected_before_launch(lib, bad, code):
     p = hga.HGAParams(rope_theta=1e4).c()
     d = _dims(**bad)
