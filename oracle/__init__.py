@@ -11,7 +11,9 @@ rotation and its relative-position property; the high/low pair split against
 its closed form; summaries against the g_s=1 and identical-key special cases
 and linearity; top-K against brute-force enumeration; the visible set against
 the policy's invariants; full-budget HGA against dense eq. (1); dense eq. (1)
-against a library softmax attention.  Parity unpinned: the readings R1-R3 of
+against a library softmax attention; the backward against automatic
+differentiation of dense attention (full budget), central differences of the
+forward (routed sets), its sum rules and position-shift invariance.  Parity unpinned: the readings R1-R3 of
 ``hga_oracle.c`` (pair convention, high/low threshold, p_mid) beyond those
 special cases are readings of the page, not facts it prints.
 """
@@ -93,6 +95,9 @@ def _load():
             lib.or_hga.restype = i32
             lib.or_dense.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, dbl, P, P]
             lib.or_dense.restype = i32
+            lib.or_hga_backward.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, P, P, i32,
+                                            P, P, P]
+            lib.or_hga_backward.restype = i32
             _lib = lib
     return _lib
 
@@ -279,3 +284,31 @@ def dense(Q, K, V, pos, theta: float):
     if rc != 0:
         raise ValueError("oracle: malformed arguments")
     return O, LSE
+
+
+def hga_backward(Q, K, V, pos, dO, params: Params, sel_g, nthreads: int | None = None):
+    """Gradients of the HGA prefill attention with the routed groups held
+    fixed: sel_g [B, NB, Hkv, K_g] are the groups the forward attended (the
+    routing is a discrete choice).  dO [B,T,Hq,D] is the gradient of the loss
+    with respect to O.  Returns (dQ, dK, dV) with respect to the raw
+    (pre-RoPE) q and k, and v, as fp64 arrays."""
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    dO = _f64(dO)
+    pos = _i32(pos)
+    B, T, Hq, D = Q.shape
+    Hkv = K.shape[2]
+    NB = (T + params.C - 1) // params.C
+    sg = np.ascontiguousarray(_i32(sel_g).reshape(B, NB, Hkv, params.K_g))
+    dQ = np.empty_like(Q)
+    dK = np.empty_like(K)
+    dV = np.empty_like(V)
+    if nthreads is None:
+        nthreads = len(os.sched_getaffinity(0))
+    pc = params.c()
+    rc = _load().or_hga_backward(_p(Q), _p(K), _p(V), _p(pos), _p(dO), B, T, Hq, Hkv, D,
+                                 ctypes.byref(pc), _p(sg), int(nthreads), _p(dQ), _p(dK), _p(dV))
+    if rc != 0:
+        raise ValueError("oracle: malformed arguments")
+    return dQ, dK, dV

@@ -14,6 +14,11 @@
  *     selection equation M_sel = topK_c, G_sel = topK_g -> or_route, or_visible_mark
  *   - "精确 Token 输出注意力" exact softmax over the routed set -> or_attend_row
  *   - eq. (2) token cost model (used only by the bench's byte/flop counts)
+ *   - training through the routed attention (Tab. 8 "Training and Prefill
+ *     Speed"; Sec. 5.9 "Fine-tuning Stability", QK fine-tuning in
+ *     exact-token mode): the gradient of eq. (1) restricted to each query's
+ *     visible set, with the routed groups held fixed -> or_hga_backward.
+ *     The page prints no formula for it; it is the textbook derivative.
  *
  * Readings where the page is silent (all stated again in the design notes):
  *   R1 RoPE pairs are rotate-half: pair i couples dims (i, i+D/2) with
@@ -489,5 +494,173 @@ int or_dense(const double *Q, const double *K, const double *V, const int32_t *p
     free(qrot);
     free(Krot);
     free(mark);
+    return 0;
+}
+
+/* ---------------------------------------------------------- backward -- */
+
+/* x = R_p^T(y), the adjoint of R1's rotation (rotation by -p); x may not
+ * alias y. */
+static void rope_adjoint(const double *y, double p, int D, const double *omega, double *x)
+{
+    int h = D / 2;
+    for (int i = 0; i < h; ++i) {
+        double a = p * omega[i];
+        double c = cos(a), s = sin(a);
+        x[i] = y[i] * c + y[i + h] * s;
+        x[i + h] = y[i + h] * c - y[i] * s;
+    }
+}
+
+typedef struct {
+    const double *Q, *K, *V, *dO;
+    const int32_t *pos, *sel_g;
+    int B, T, Hq, Hkv, D, NB;
+    const or_params *p;
+    double *dQ, *dK, *dV;
+    const double *omega;
+    int nthreads, tid;
+} or_bwd_job;
+
+/* One (sequence b, KV head h): every query row of h's query heads, in
+ * order; dK and dV rows of (b, h) and dQ rows of those heads belong to this
+ * item alone. */
+static void bwd_item(const or_bwd_job *J, int b, int h)
+{
+    const or_params *p = J->p;
+    int T = J->T, D = J->D, G = J->Hq / J->Hkv;
+    int64_t ks = (int64_t)J->Hkv * D; /* key row stride */
+    double scale = 1.0 / sqrt((double)D);
+    double *krot = (double *)malloc(sizeof(double) * (size_t)((int64_t)(T > 0 ? T : 1) * D));
+    double *dkrot = (double *)calloc((size_t)((int64_t)(T > 0 ? T : 1) * D), sizeof(double));
+    double *pr = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    uint8_t *mark = (uint8_t *)malloc((size_t)T + 1);
+    double *qrot = (double *)malloc(sizeof(double) * (size_t)D);
+    double *o = (double *)malloc(sizeof(double) * (size_t)D);
+    double *dqrot = (double *)malloc(sizeof(double) * (size_t)D);
+    const double *Kb = J->K + ((int64_t)b * T * J->Hkv + h) * D;
+    const double *Vb = J->V + ((int64_t)b * T * J->Hkv + h) * D;
+    double *dKb = J->dK + ((int64_t)b * T * J->Hkv + h) * D;
+    double *dVb = J->dV + ((int64_t)b * T * J->Hkv + h) * D;
+    for (int j = 0; j < T; ++j) {
+        rope(Kb + (int64_t)j * ks, (double)J->pos[(int64_t)b * T + j], D, J->omega,
+             krot + (int64_t)j * D);
+        for (int d = 0; d < D; ++d)
+            dVb[(int64_t)j * ks + d] = 0.0;
+    }
+    for (int i = 0; i < T; ++i) {
+        int c = i / p->C;
+        or_visible_mark(c, i, T, J->sel_g + (((int64_t)b * J->NB + c) * J->Hkv + h) * p->K_g, p,
+                        mark);
+        double pi = (double)J->pos[(int64_t)b * T + i];
+        for (int hh = h * G; hh < (h + 1) * G; ++hh) {
+            int64_t row = ((int64_t)b * T + i) * J->Hq + hh;
+            const double *dO = J->dO + row * D;
+            rope(J->Q + row * D, pi, D, J->omega, qrot);
+            /* forward again: P_j and O_i */
+            double mx = -INFINITY;
+            for (int j = 0; j < T; ++j) {
+                if (!mark[j]) continue;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += qrot[d] * krot[(int64_t)j * D + d];
+                pr[j] = dot * scale;
+                if (pr[j] > mx) mx = pr[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j < T; ++j)
+                if (mark[j]) {
+                    pr[j] = exp(pr[j] - mx);
+                    l += pr[j];
+                }
+            for (int d = 0; d < D; ++d)
+                o[d] = 0.0;
+            for (int j = 0; j < T; ++j) {
+                if (!mark[j]) continue;
+                pr[j] /= l;
+                for (int d = 0; d < D; ++d)
+                    o[d] += pr[j] * Vb[(int64_t)j * ks + d];
+            }
+            /* D_i = dO_i . O_i, then the gradients through P */
+            double di = 0.0;
+            for (int d = 0; d < D; ++d)
+                di += dO[d] * o[d];
+            for (int d = 0; d < D; ++d)
+                dqrot[d] = 0.0;
+            for (int j = 0; j < T; ++j) {
+                if (!mark[j]) continue;
+                double dp = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dp += dO[d] * Vb[(int64_t)j * ks + d];
+                double ds = pr[j] * (dp - di);
+                for (int d = 0; d < D; ++d) {
+                    dVb[(int64_t)j * ks + d] += pr[j] * dO[d];
+                    dqrot[d] += ds * scale * krot[(int64_t)j * D + d];
+                    dkrot[(int64_t)j * D + d] += ds * scale * qrot[d];
+                }
+            }
+            rope_adjoint(dqrot, pi, D, J->omega, J->dQ + row * D);
+        }
+    }
+    for (int j = 0; j < T; ++j)
+        rope_adjoint(dkrot + (int64_t)j * D, (double)J->pos[(int64_t)b * T + j], D, J->omega,
+                     dKb + (int64_t)j * ks);
+    free(krot);
+    free(dkrot);
+    free(pr);
+    free(mark);
+    free(qrot);
+    free(o);
+    free(dqrot);
+}
+
+static void *bwd_worker(void *arg)
+{
+    or_bwd_job *J = (or_bwd_job *)arg;
+    for (int it = J->tid; it < J->B * J->Hkv; it += J->nthreads)
+        bwd_item(J, it / J->Hkv, it % J->Hkv);
+    return NULL;
+}
+
+/* Backward of the exact attention of HGA prefill (eq. (1) restricted to each
+ * query token's visible set, blocks of C query tokens).  Routing is a
+ * discrete choice, so no gradient reaches the summaries: the routed groups
+ * are an input, sel_g [B, NB, Hkv, K_g] (NB = ceil(T / C)), the ones the
+ * forward attended.  Given dO [B,T,Hq,D], writes the gradients of the loss
+ * with respect to the RAW (pre-RoPE) q and k and to v:
+ *   S_ij = R_{p_i}(q_i) . R_{p_j}(k_j) / sqrt(D), P_ij = softmax_j S_ij over
+ *   j in V(i), O_i = sum_j P_ij v_j,
+ *   dv_j = sum_i P_ij dO_i,
+ *   dS_ij = P_ij (dO_i . v_j - dO_i . O_i),
+ *   dq_i = R_{p_i}^T sum_j dS_ij R_{p_j}(k_j) / sqrt(D),
+ *   dk_j = R_{p_j}^T sum_i dS_ij R_{p_i}(q_i) / sqrt(D),
+ * where i runs over the query rows of every query head of k_j's KV head.
+ * dQ [B,T,Hq,D], dK and dV [B,T,Hkv,D].  Returns 0, or -1 on a malformed
+ * argument. */
+int or_hga_backward(const double *Q, const double *K, const double *V, const int32_t *pos,
+                    const double *dO, int B, int T, int Hq, int Hkv, int D, const or_params *p,
+                    const int32_t *sel_g, int nthreads, double *dQ, double *dK, double *dV)
+{
+    if (Hq % Hkv || D % 2 || p->C % p->g_s || p->C < 1 || T < 0 || B < 1) return -1;
+    int NB = (T + p->C - 1) / p->C;
+    double *omega = (double *)malloc(sizeof(double) * (size_t)(D / 2));
+    or_omega(D, p->theta, omega);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B * Hkv) nthreads = B * Hkv;
+    or_bwd_job *jobs = (or_bwd_job *)malloc(sizeof(or_bwd_job) * (size_t)nthreads);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 0; t < nthreads; ++t) {
+        or_bwd_job J = {Q, K, V, dO, pos, sel_g, B, T, Hq, Hkv, D, NB, p, dQ, dK, dV, omega,
+                        nthreads, t};
+        jobs[t] = J;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        pthread_create(&th[t], NULL, bwd_worker, &jobs[t]);
+    bwd_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        pthread_join(th[t], NULL);
+    free(jobs);
+    free(th);
+    free(omega);
     return 0;
 }
