@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-hosttier", action="store_true")
+    ap.add_argument("--no-cold-l2", action="store_true")
     ap.add_argument("--decode-replays", type=int, default=10)
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling variant: only the decode part")
@@ -91,6 +92,62 @@ def config_of(w, n):
             "cosine 0.5 to one earlier middle chunk per block",
             "l2": "inputs larger than L2: Q and O stream 537 MB per step",
             "parallelism": "single GPU" if n == 1 else f"{n} independent replicas"}
+
+
+def stage_bytes(w):
+    """Compulsory HBM bytes of one summaries launch and one routing launch:
+    every input read once and every output written once.  Summaries: K and
+    positions in, rotated K and the chunk and group summary tables out.
+    Routing: Q and positions in, the two summary tables read once, the chunk
+    and group selections out."""
+    e = 2 if w.dtype == "bf16" else 4
+    NC = w.T // w.C
+    NB = (w.T + w.C - 1) // w.C
+    tables = w.B * w.Hkv * NC * (1 + w.C // w.g_s) * w.D * 4
+    kv = w.B * w.T * w.Hkv * w.D * e
+    summaries = 2 * kv + w.B * w.T * 4 + tables
+    route = (w.B * w.T * w.Hq * w.D * e + w.B * w.T * 4 + tables
+             + w.B * NB * w.Hkv * (w.K_c + w.K_g) * 4)
+    return summaries, route
+
+
+def cold_l2_times(fns, stream, dev, iters=20):
+    """Mean CUDA-event time of each call in fns with a cold L2: before every
+    timed call a scratch buffer of twice the L2 size is written on the same
+    stream, outside the events."""
+    import torch
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or 126 * 10**6)
+    scratch = torch.empty(2 * l2 // 4 + 1024, dtype=torch.int32, device=dev)
+    marks = []
+    for it in range(iters + 2):                    # the first two are warm-up
+        for n, fn in enumerate(fns):
+            scratch.fill_(it)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            if it >= 2:
+                marks.append((n, a, b))
+    torch.cuda.synchronize(dev)
+    out = [statistics.mean(a.elapsed_time(b) for m, a, b in marks if m == n)
+           for n in range(len(fns))]
+    del scratch
+    return out
+
+
+def cold_l2_report(cold, w, pk, src):
+    """The line's cold_l2 entry: per stage its mean time, compulsory bytes,
+    rate and fraction of the measured HBM copy peak; or the error text when
+    the timing failed."""
+    if not (isinstance(cold, list) and len(cold) == 2 and all(t > 0 for t in cold)):
+        return {"error": str(cold)}
+    hbm = pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    out = {"flush": "a scratch write of twice the L2 size before each timed call"}
+    for name, t, nb in zip(("summaries", "route"), cold, stage_bytes(w)):
+        out[name] = {"ms": t, "bytes": nb, "gbs": nb / t / 1e6, "frac": nb / t / 1e6 / hbm}
+    out["peak_gbs"] = hbm
+    out["peak_source"] = f"{src} hbm_gbs (copy)"
+    return out
 
 
 def attention_flops(w, sel_group):
@@ -519,6 +576,19 @@ def main():
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(w.B * w.T * args.steps, world, total_ms)
 
+    # summaries and routing again, each after a 2x-L2 scratch write (cold L2);
+    # a failure here is reported in the line and never costs the bench line
+    cold = None
+    if not (args.no_cold_l2 or args.seq or args.no_e2e):   # full bench line only
+        try:
+            cold = cold_l2_times(
+                [lambda: hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c,
+                                                 s_group=s_g),
+                 lambda: hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)],
+                stream, dev)
+        except Exception as exc:               # noqa: BLE001 - reported, not raised
+            cold = f"{type(exc).__name__}: {exc}"
+
     # end to end through the public one-call API, host buffers, every step's
     # copies inside the timed region; consecutive steps overlap as a serving
     # loop would run them: inputs in on one stream, the prefill on a second,
@@ -610,6 +680,8 @@ def main():
             "gpu_launches": 3 * args.steps,
             "stage_ms": {"summaries": stage_ms[0], "route": stage_ms[1], "attend": stage_ms[2]},
             "roofline": roof}
+    if cold is not None:
+        line["cold_l2"] = cold_l2_report(cold, w, pk, src)
     if dec is not None:
         line["decode"] = dec
     if tier is not None:
