@@ -203,7 +203,10 @@ def test_decode_64k_full_size_graph(gpu_lib):
                 ok, _ = check_unit_selection(ref, 0, h, t, t + 1, t // 64, sc[t - w.T, h],
                                              sg[t - w.T, h], rr["sel_c"][i, h], rr["sel_g"][i, h])
                 assert ok, f"routing mismatch b={b} t={t} h={h}"
-        sample = [0, 1, 63, 64, 127, 128, 200, S - 1]
+        # 32 steps per sequence, 64 (sequence, step) outputs in all
+        edges = [0, 1, 63, 64, 127, 128, 200, S - 1]
+        sample = sorted(edges + [s for s in range(2, S - 1, 10) if s not in edges][:32 - len(edges)])
+        assert len(sample) == 32
         u2 = [(0, w.T + s) for s in sample]
         force = np.stack([sg[s] for s in sample])
         orc = oracle.hga(Q, K, V, pos, p, route_block=1, units=u2, sel_g_force=force)

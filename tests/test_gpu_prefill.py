@@ -130,7 +130,8 @@ def test_qwen_32k_full_size(gpu_lib):
     through the middle and the last)."""
     w = QWEN
     NB = w.T // 64
-    blocks = list(range(0, w.F + w.L + 2)) + list(range(40, NB, 61)) + [NB - 1]
+    blocks = list(range(0, w.F + w.L + 2)) + list(range(w.F + w.L + 3, NB - 1, 9)) + [NB - 1]
+    assert len(blocks) >= 64
     run_and_check(gpu_lib, w, seed=11, units=[(0, u) for u in blocks])
 
 
