@@ -22,6 +22,7 @@
 // warp bitonic sort and merge of packed (fp32 score, id) keys), scores the
 // groups of its chunks and takes the top K_g.  K above 32 falls back to
 // CTA-wide selection rounds, one block at a time.
+#include <climits>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -46,7 +47,6 @@ struct RouteArgs {
     int32_t *sel_chunk, *sel_group;
     Rope rope;
 };
-
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
@@ -257,7 +257,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     }
 }
 
-
 // SM count and resident CTAs per SM of `kern` at `smem` bytes on the current
 // device (looked up once per kernel, size and device).
 cudaError_t residency(const void *kern, size_t smem, int *sms, int *per_sm) {
@@ -319,6 +318,9 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     e = residency((const void *)kern, smem, &sms, &per_sm);
     if (e != cudaSuccess) return cuda_status(e);
     a.nblk = per_sm > 0 ? pick_run(g.NB, g.Hkv * g.B, nmax, sms, per_sm) : nmax;
+    // the kernel forms a 32-bit linear CTA index
+    if ((long long)((g.NB + a.nblk - 1) / a.nblk) * g.Hkv * g.B > (long long)INT32_MAX)
+        return HGA_ERR_UNSUPPORTED;
     dim3 grid((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
     kern<<<grid, kThreads, smem, st>>>(a);
     return cuda_status(cudaGetLastError());
