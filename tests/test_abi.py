@@ -125,3 +125,31 @@ def test_hostkv_link_bytes_checks_its_pointer(lib):
     lib.hga_hostkv_link_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.hga_hostkv_link_bytes.restype = ctypes.c_int
     assert lib.hga_hostkv_link_bytes(None, None, 0) == 1     # HGA_ERR_INVALID_ARG
+
+
+def test_decode_mode_host_checks(lib):
+    """HGA_DECODE: the workspace, the step's inputs and every cache buffer are
+    checked on the host; a cache whose capacity is not dims.T and a
+    misaligned row are refused before anything is launched (the fake pointers
+    below are never dereferenced, and no call here is valid enough to launch)."""
+    by = ctypes.byref
+    p = hga.HGAParams(F=2, L=8, K_c=16, K_g=32, rope_theta=1e6).c()
+    d = _dims(B=2, T=4096, Hq=32, Hkv=4, D=128, dtype=1)
+    n = lib.hga_workspace_size(1, by(d), by(p))
+    assert n > 0
+    ws = ctypes.c_void_p(1 << 20)
+    io = hga._IO()
+    assert lib.hga_forward(1, by(d), by(p), by(io), None, 0, None) == 6       # no workspace
+    assert lib.hga_forward(1, by(d), by(p), by(io), ws, n - 1, None) == 6     # too small
+    assert lib.hga_forward(1, by(d), by(p), by(io), ws, n, None) == 1         # no inputs
+    A = 1 << 24
+    for f in ("q_new", "k_new", "v_new", "pos_new", "out"):
+        setattr(io, f, A)
+    assert lib.hga_forward(1, by(d), by(p), by(io), ws, n, None) == 1         # no cache
+    io.cache.capacity = 4096 - 64
+    for f in ("k_rot", "v", "pos", "k_open", "s_chunk", "s_group", "lens"):
+        setattr(io.cache, f, A)
+    assert lib.hga_forward(1, by(d), by(p), by(io), ws, n, None) == 1         # capacity != T
+    io.cache.capacity = 4096
+    io.out = A + 8
+    assert lib.hga_forward(1, by(d), by(p), by(io), ws, n, None) == 1         # misaligned out
