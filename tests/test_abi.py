@@ -153,3 +153,36 @@ def test_decode_mode_host_checks(lib):
     io.cache.capacity = 4096
     io.out = A + 8
     assert lib.hga_forward(1, by(d), by(p), by(io), ws, n, None) == 1         # misaligned out
+
+
+def test_prefill_cache_fill_host_checks(lib):
+    """HGA_PREFILL filling a decode cache: a capacity below T or not a whole
+    number of chunks, and a cache beyond the 32-bit row limit, are refused
+    before any launch (fake pointers, never dereferenced)."""
+    by = ctypes.byref
+    p = hga.HGAParams(F=2, L=8, K_c=16, K_g=32, rope_theta=1e6).c()
+    d = _dims(B=2, T=4096, Hq=32, Hkv=4, D=128, dtype=1)
+    A = 1 << 24
+    io = hga._IO()
+    for f in ("k", "v", "pos"):                 # cache fill only: no q, no out
+        setattr(io, f, A)
+    for f in ("k_rot", "v", "pos", "k_open", "s_chunk", "s_group", "lens"):
+        setattr(io.cache, f, A)
+    io.cache.capacity = 4096 - 64
+    assert lib.hga_forward(0, by(d), by(p), by(io), None, 0, None) == 1       # below T
+    io.cache.capacity = 4096 + 32
+    assert lib.hga_forward(0, by(d), by(p), by(io), None, 0, None) == 1       # not whole chunks
+    io.cache.capacity = 1 << 30
+    assert lib.hga_forward(0, by(d), by(p), by(io), None, 0, None) == 2       # B*capacity >= 2^31
+
+
+def test_noalloc_rejects_oversized_shapes_on_the_host(lib):
+    """The no-allocation prefill refuses a shape whose scratch exceeds its
+    fixed 16 MiB before any CUDA call (fake pointers, never dereferenced)."""
+    by = ctypes.byref
+    p = hga.HGAParams(F=2, L=8, K_c=16, K_g=32, rope_theta=1e6).c()
+    big = _dims(B=1, T=32768, Hq=32, Hkv=4, D=128, dtype=1)
+    assert lib.hga_workspace_size(0, by(big), by(p)) > 16 << 20
+    A = ctypes.c_void_p(1 << 24)
+    st = lib.hga_forward_prefill_noalloc(by(big), by(p), A, A, A, A, A, None, None)
+    assert st == 6
