@@ -42,3 +42,21 @@ def test_cold_l2_report():
     assert bench.cold_l2_report("RuntimeError: out of memory", w, {}, "fallback") == {
         "error": "RuntimeError: out of memory"}
     assert "error" in bench.cold_l2_report([0.0, 0.1], w, {}, "fallback")
+
+
+def test_reference_arm_line_on_cpu(monkeypatch, capsys):
+    # the reference arm is the oracle on host cores: one JSON line with the
+    # same metric and workload as the library's line, its CPU baseline, and
+    # an e2e entry that moves no bytes
+    import argparse
+    import json
+    monkeypatch.setenv("RANK", "0")
+    bench.run_reference(argparse.Namespace(gpus=1, steps=1, warmup=0, seed=0))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["config"]["workload"] == bench.WORKLOAD
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    e = line["e2e"]
+    assert e["value"] == line["value"] and e["h2d_bytes_per_step"] == e["d2h_bytes_per_step"] == 0
