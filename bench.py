@@ -14,6 +14,7 @@ cross-sequence exchange); value = all ranks' tokens / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import math
@@ -30,7 +31,10 @@ WORKLOAD = "qwen3_30b_a3b_bf16_prefill_32k"
 METRIC = "HGA routed-attn prefill tokens/s & decode steps/s at 32K/64K; % HBM roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attend_tc_qwen32k_traffic.txt")
-ATTEND_SRC = os.path.join(ROOT, "hierarchical_kv_routing_b200", "csrc", "attend_tc.cu")
+CSRC = os.path.join(ROOT, "hierarchical_kv_routing_b200", "csrc")
+ATTEND_SRC = os.path.join(CSRC, "attend_tc.cu")
+DECODE_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_qwen64k_traffic.txt")
+DECODE_SRC = os.path.join(CSRC, "decode.cu")
 
 
 def parse():
@@ -45,6 +49,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-hosttier", action="store_true")
     ap.add_argument("--no-cold-l2", action="store_true")
+    ap.add_argument("--no-smalllm", action="store_true")
     ap.add_argument("--decode-replays", type=int, default=10)
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling variant: only the decode part")
@@ -171,16 +176,20 @@ def attention_flops(w, sel_group):
 
 
 class ClockSampler:
-    """Samples SM clock, max clock and active clock-event reasons via NVML
-    while the timed region runs (reading only; nothing is changed)."""
+    """Samples SM clock, max clock and active clock-event reasons via NVML on
+    a background thread (reading only; nothing is changed), every `period`
+    seconds.  `leg(name)` brackets a timed region so the result can give each
+    region's own sample count and median clock."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
+    def __init__(self, device_index, period=0.0005):
+        self.samples, self.max_mhz = [], None      # (time, MHz, reason bits)
+        self.period = period
+        self.legs = {}
         self._stop = threading.Event()
         self._ok = False
         try:
@@ -208,14 +217,12 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
                 r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
+                self.samples.append((time.perf_counter(), mhz, r))
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(self.period)
 
     def __enter__(self):
         if self._ok:
@@ -228,21 +235,62 @@ class ClockSampler:
         if self._ok:
             self.t.join()
 
+    class _Leg:
+        def __init__(self, owner, name):
+            self.owner, self.name = owner, name
+
+        def __enter__(self):
+            self.t0 = time.perf_counter()
+
+        def __exit__(self, *a):
+            self.owner.legs.setdefault(self.name, []).append((self.t0, time.perf_counter()))
+
+    def leg(self, name):
+        return self._Leg(self, name)
+
+    def _summary(self, samples):
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, _, r in samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for _, m, _ in samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons - {"gpu_idle"}),
+                "samples": len(samples)}
+
     def result(self):
-        if not self._ok or not self.samples:
+        """Median clock and reasons over every bracketed leg (all samples when
+        no leg was bracketed), plus each leg's own."""
+        if not self._ok:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        spans = [sp for v in self.legs.values() for sp in v]
+        inside = [x for x in self.samples if any(a <= x[0] <= b for a, b in spans)] \
+            if spans else list(self.samples)
+        out = self._summary(inside)
+        out["period_ms"] = self.period * 1e3
+        out["legs"] = {}
+        for name, sp in self.legs.items():
+            leg = self._summary([x for x in self.samples if any(a <= x[0] <= b for a, b in sp)])
+            out["legs"][name] = {"samples": leg["samples"], "sm_mhz": leg["sm_mhz"],
+                                 "reasons": leg["reasons"],
+                                 "seconds": round(sum(b - a for a, b in sp), 4)}
+        return out
 
 
-def traffic_for_current_kernel():
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu
-    summary, only if that summary was taken on the current kernel source."""
-    if not os.path.exists(TRAFFIC_FILE):
+def traffic_for_current_kernel(traffic_file=TRAFFIC_FILE, sources=(ATTEND_SRC,)):
+    """Per-launch (or per-step) DRAM bytes from a committed ncu summary, only
+    if that summary was taken on the current kernel source (the hash of the
+    listed source files, in order, must match the one recorded)."""
+    if not os.path.exists(traffic_file):
         return None
-    src_hash = hashlib.sha256(open(ATTEND_SRC, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in sources:
+        h.update(open(f, "rb").read())
+    src_hash = h.hexdigest()[:16]
     vals = {}
-    for line in open(TRAFFIC_FILE):
+    for line in open(traffic_file):
         if "=" in line and not line.startswith("#"):
             k, v = line.split("=", 1)
             vals[k.strip()] = v.strip()
@@ -294,8 +342,13 @@ def cpu_baseline(w, seed, budget_s=20.0, per_call=16):
                       f"pass + mean block time x {NB}"}
 
 
-def run_reference(args, per_step=2):
-    """The CPU oracle on the same workload (rank 0 only)."""
+def run_reference(args):
+    """The CPU oracle on the same workload (rank 0 only).  Each step is a
+    bounded sample: the full-sequence rotation and summary pass plus enough
+    query blocks (all KV heads each) to give every host thread one (block,
+    KV head) unit.  ms_per_step is the measured time of such a sampled step;
+    value extrapolates it to the whole workload (that pass + mean block time
+    x blocks)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -303,28 +356,36 @@ def run_reference(args, per_step=2):
     w = WORKLOADS[WORKLOAD]
     inputs = _oracle_inputs(w, args.seed)
     nthreads = len(os.sched_getaffinity(0))
+    per_step = max(1, -(-nthreads // w.Hkv))
     t_pre = _oracle_sample(w, inputs, [], nthreads)
     NB = w.T // w.C
-    step_est = []
+    step_est, step_meas = [], []
     for s in range(args.warmup + args.steps):
         blocks = [(s * 97 * per_step + j * 211 + 11) % NB for j in range(per_step)]
         dt = _oracle_sample(w, inputs, blocks, nthreads)
         if s >= args.warmup:
+            step_meas.append(dt)
             step_est.append(t_pre + max(dt - t_pre, 0.0) / per_step * NB)
     est = statistics.median(step_est)
     value = w.B * w.T / est
     cores = min(nthreads, per_step * w.Hkv)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": statistics.mean(step_meas) * 1e3,
+            "ms_per_step_is": "the measured time of one sampled step (see cpu_baseline.sample); "
+                              "value is the whole workload's tokens over the extrapolated "
+                              "whole-workload time",
+            "whole_workload_ms_estimate": est * 1e3,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, 1),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle",
-                             "sample": f"each step: {per_step} of {NB} query blocks (all KV "
-                                       f"heads) after a {t_pre:.2f} s full-sequence pass; step "
-                                       f"value = that pass + mean block time x {NB}; median "
-                                       f"over steps"},
+                             "sample": f"each step: {per_step} of {NB} query blocks (all "
+                                       f"{w.Hkv} KV heads, one (block, KV head) unit per "
+                                       f"thread on {cores} threads) after a {t_pre:.2f} s "
+                                       f"full-sequence pass; whole-workload time = that pass "
+                                       f"+ mean block time x {NB}; median over steps"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -355,7 +416,7 @@ def decode_bytes_per_step(w, T0, steps):
     return total / steps
 
 
-def bench_decode(args, dev, world):
+def bench_decode(args, dev, world, clk=None):
     """16 sequences with a 64K-token cache, 256 decode steps captured in one
     CUDA graph; steps/s and the HBM roofline of a step."""
     import torch
@@ -404,10 +465,11 @@ def bench_decode(args, dev, world):
     for _ in range(args.decode_replays):
         cache.lens.fill_(w.T)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        graph.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
+        with (clk.leg("decode") if clk else contextlib.nullcontext()):
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
         times.append(e0.elapsed_time(e1))
     assert int(cache.lens[0].item()) == cap
     ms_step = max_over_ranks(sum(times), dev, world) / (len(times) * S)
@@ -426,7 +488,9 @@ def bench_decode(args, dev, world):
             "roofline": {"bound": "hbm", "achieved": achieved,
                          "peak": pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]), "unit": "GB/s",
                          "frac": achieved / pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]),
-                         "traffic": None, "bytes_per_step": bps,
+                         "traffic": traffic_for_current_kernel(DECODE_TRAFFIC_FILE,
+                                                               (DECODE_SRC,)),
+                         "bytes_per_step": bps,
                          "peak_source": f"{src} hbm_gbs (copy)"}}
 
 
@@ -443,7 +507,7 @@ def hosttier_link_bytes_uncached(w, sel_group):
     return w.B * w.T * row + 2 * w.B * w.T * row + routed
 
 
-def bench_hosttier(args, dev, world):
+def bench_hosttier(args, dev, world, clk=None):
     """The 64K prefill with K/V in pinned host RAM; tokens/s and the fraction
     of the host-to-device copy bandwidth measured in the same run."""
     import torch
@@ -470,11 +534,12 @@ def bench_hosttier(args, dev, world):
         dist.barrier()
     steps = 5
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    with (clk.leg("hosttier") if clk else contextlib.nullcontext()):
+        e0.record(stream)
+        for _ in range(steps):
+            hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
     # bytes read over the link per call: the gathers' own count (sinks,
     # windows, warm-cache misses) plus stage 1's single pass over raw K
@@ -505,6 +570,85 @@ def bench_hosttier(args, dev, world):
                                         "of 256 MiB, best of 5"}}
 
 
+SMALLLM_WORKLOAD = "smalllm40m_bf16_prefill_4k"
+
+
+def smalllm_bytes(w):
+    """Compulsory HBM bytes of one prefill step of a workload: Q, K, V and O
+    once each, and the rotated keys written once (the summary tables and the
+    routed ids are under 2% more and are left out)."""
+    e = 2 if w.dtype == "bf16" else 4
+    return w.B * w.T * (2 * w.Hq + 3 * w.Hkv) * w.D * e
+
+
+def bench_smalllm(args, dev, world, clk):
+    """The SmallLM-40M-shaped prefill (8 sequences x 4096 tokens, 8 heads,
+    D=64, MHA): the same three stages as the main step, timed with CUDA
+    events; tokens/s and the HBM roofline of the step's compulsory bytes."""
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_kv_routing_b200 as hga
+    from workloads import WORKLOADS, make_prefill_inputs
+    w = WORKLOADS[SMALLLM_WORKLOAD]
+    hp = params_of(w)
+    rank = int(os.environ.get("RANK", "0"))
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=args.seed + 500 + rank, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    k_rot, s_c, s_g = hga.hga_build_summaries(k, pos, hp)
+    sel_c, sel_g = hga.hga_route(q, pos, s_c, s_g, hp)
+    out = torch.empty_like(q)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c, s_group=s_g)
+        if ev:
+            ev[1].record(stream)
+        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)
+        if ev:
+            ev[2].record(stream)
+        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    flops = attention_flops(w, sel_g)
+    steps = max(args.steps, 20)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with clk.leg("smalllm"):
+        for i in range(steps):
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[-1][3]), dev, world)
+    stage_ms = [statistics.mean(e[a].elapsed_time(e[a + 1]) for e in evs) for a in range(3)]
+    ms = total_ms / steps
+    pk, src = peaks()
+    hbm = pk.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    nb = smalllm_bytes(w)
+    achieved = nb / (ms / 1e3) / 1e9
+    tc = flops / (stage_ms[2] / 1e3) / 1e12
+    tpk = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    return {"metric": "prefill tokens/s", "value": whole_job_rate(w.B * w.T * steps, world, total_ms),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+                       "D": w.D, "F": w.F, "L": w.L, "K_c": w.K_c, "K_g": w.K_g,
+                       "recipe": "chunk-topic keys (sigma 0.5); Q, V N(0,1)",
+                       "l2": "Q, K, V, O and K_rot: 168 MB per step, above the 126 MB L2"},
+            "stage_ms": {"summaries": stage_ms[0], "route": stage_ms[1], "attend": stage_ms[2]},
+            "gpu_launches": 3 * steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "bytes_per_step": nb, "traffic": None,
+                         "peak_source": f"{src} hbm_gbs (copy)",
+                         "attention_tflops": tc, "attention_frac_of_bf16": tc / tpk,
+                         "attention_flops_per_launch": flops}}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -526,7 +670,9 @@ def main():
     dev = torch.device("cuda", local)
     hga.load()
     if args.decode_only:
-        dec = bench_decode(args, dev, world)
+        with ClockSampler(local) as clk:
+            dec = bench_decode(args, dev, world, clk)
+        dec["clocks"] = clk.result()
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
@@ -564,7 +710,8 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+    clk = ClockSampler(local).__enter__()     # runs until every leg is timed
+    with clk.leg("prefill"):
         for i in range(args.steps):
             step(evs[i])
         torch.cuda.synchronize(dev)
@@ -581,11 +728,12 @@ def main():
     cold = None
     if not (args.no_cold_l2 or args.seq or args.no_e2e):   # full bench line only
         try:
-            cold = cold_l2_times(
-                [lambda: hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c,
-                                                 s_group=s_g),
-                 lambda: hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)],
-                stream, dev)
+            with clk.leg("cold_l2"):
+                cold = cold_l2_times(
+                    [lambda: hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c,
+                                                     s_group=s_g),
+                     lambda: hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)],
+                    stream, dev)
         except Exception as exc:               # noqa: BLE001 - reported, not raised
             cold = f"{type(exc).__name__}: {exc}"
 
@@ -638,21 +786,24 @@ def main():
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for s_ in (s_in, s_comp, s_out):
-        s_.wait_stream(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    join()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    with clk.leg("e2e"):
+        e0.record(stream)
+        for s_ in (s_in, s_comp, s_out):
+            s_.wait_stream(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        join()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
     te = max_over_ranks(e0.elapsed_time(e1), dev, world)
     e2e_value = whole_job_rate(w.B * w.T * e2e_steps, world, te) if e2e_steps else None
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hpos))
     d2h = houts[0].numel() * houts[0].element_size()
 
-    dec = None if args.no_decode else bench_decode(args, dev, world)
-    tier = None if args.no_hosttier else bench_hosttier(args, dev, world)
+    dec = None if args.no_decode else bench_decode(args, dev, world, clk)
+    tier = None if args.no_hosttier else bench_hosttier(args, dev, world, clk)
+    small = None if (args.no_smalllm or args.seq) else bench_smalllm(args, dev, world, clk)
+    clk.__exit__(None, None, None)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -686,6 +837,8 @@ def main():
         line["decode"] = dec
     if tier is not None:
         line["hosttier"] = tier
+    if small is not None:
+        line["smalllm"] = small
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.seed)
     if args.seq or args.no_e2e:

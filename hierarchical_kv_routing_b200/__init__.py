@@ -135,10 +135,20 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device=None) -> ctypes.c_void_p:
+    """The stream a call is enqueued on: the given one, or the current stream
+    of the call's device.  A given stream must belong to that device."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise HGAError(f"stream is on {stream.device}, the call's tensors are on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(device):
+    """Make the call's device current while the library runs (the library
+    launches on the current device and looks up per-device state there)."""
+    return torch.cuda.device(device)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -149,11 +159,13 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise HGAError(f"unsupported dtype {t.dtype}: float32 or bfloat16")
 
 
-def _need(t: torch.Tensor, name: str, shape=None, dtype=None):
+def _need(t: torch.Tensor, name: str, shape=None, dtype=None, device=None):
     if not isinstance(t, torch.Tensor):
         raise HGAError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise HGAError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise HGAError(f"{name} is on {t.device}, the call's tensors are on {device}")
     if not t.is_contiguous():
         raise HGAError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -176,9 +188,9 @@ def hga_build_summaries(k_raw: torch.Tensor, pos: torch.Tensor, params: HGAParam
     lib = load()
     _need(k_raw, "k_raw")
     B, T, Hkv, D = k_raw.shape
-    _need(pos, "pos", (B, T), torch.int32)
-    NC = T // params.C
     dev = k_raw.device
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    NC = T // params.C
     if k_rot is None and want_k_rot:
         k_rot = torch.empty_like(k_raw)
     if s_chunk is None:
@@ -186,10 +198,16 @@ def hga_build_summaries(k_raw: torch.Tensor, pos: torch.Tensor, params: HGAParam
     if s_group is None:
         s_group = torch.empty(B, Hkv, NC * (params.C // params.g_s), D, device=dev,
                               dtype=torch.float32)
+    if k_rot is not None:
+        _need(k_rot, "k_rot", (B, T, Hkv, D), k_raw.dtype, dev)
+    _need(s_chunk, "s_chunk", (B, Hkv, NC, D), torch.float32, dev)
+    _need(s_group, "s_group", (B, Hkv, NC * (params.C // params.g_s), D), torch.float32, dev)
     dims = _dims(B, T, Hkv, Hkv, D, _dtype_code(k_raw))
     pc = params.c()
-    st = lib.hga_build_summaries(ctypes.byref(dims), ctypes.byref(pc), _ptr(k_raw), _ptr(pos),
-                                 _ptr(k_rot), _ptr(s_chunk), _ptr(s_group), _stream(stream))
+    with _on(dev):
+        st = lib.hga_build_summaries(ctypes.byref(dims), ctypes.byref(pc), _ptr(k_raw), _ptr(pos),
+                                     _ptr(k_rot), _ptr(s_chunk), _ptr(s_group),
+                                     _stream(stream, dev))
     _check(st, "hga_build_summaries")
     return k_rot, s_chunk, s_group
 
@@ -200,19 +218,24 @@ def hga_route(q: torch.Tensor, pos: torch.Tensor, s_chunk: torch.Tensor, s_group
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
+    dev = q.device
     Hkv = s_chunk.shape[1]
-    _need(pos, "pos", (B, T), torch.int32)
-    _need(s_chunk, "s_chunk", dtype=torch.float32)
-    _need(s_group, "s_group", dtype=torch.float32)
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    _need(s_chunk, "s_chunk", (B, Hkv, T // params.C, D), torch.float32, dev)
+    _need(s_group, "s_group", (B, Hkv, (T // params.C) * (params.C // params.g_s), D),
+          torch.float32, dev)
     NB = (T + params.C - 1) // params.C
     if sel_chunk is None:
         sel_chunk = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
     if sel_group is None:
         sel_group = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+    _need(sel_chunk, "sel_chunk", (B, NB, Hkv, params.K_c), torch.int32, dev)
+    _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
-    st = lib.hga_route(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(s_chunk),
-                       _ptr(s_group), _ptr(sel_chunk), _ptr(sel_group), _stream(stream))
+    with _on(dev):
+        st = lib.hga_route(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(s_chunk),
+                           _ptr(s_group), _ptr(sel_chunk), _ptr(sel_group), _stream(stream, dev))
     _check(st, "hga_route")
     return sel_chunk, sel_group
 
@@ -224,19 +247,25 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
+    dev = q.device
     Hkv = k_rot.shape[2]
-    _need(k_rot, "k_rot", (B, T, Hkv, D), q.dtype)
-    _need(v, "v", (B, T, Hkv, D), q.dtype)
-    _need(pos, "pos", (B, T), torch.int32)
-    _need(sel_group, "sel_group", dtype=torch.int32)
+    NB = (T + params.C - 1) // params.C
+    _need(k_rot, "k_rot", (B, T, Hkv, D), q.dtype, dev)
+    _need(v, "v", (B, T, Hkv, D), q.dtype, dev)
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+    _need(out, "out", (B, T, Hq, D), q.dtype, dev)
+    if lse is not None:
+        _need(lse, "lse", (B, Hq, T), torch.float32, dev)
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
-    st = lib.hga_attend(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(k_rot),
-                        _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream))
+    with _on(dev):
+        st = lib.hga_attend(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(k_rot),
+                            _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream, dev))
     _check(st, "hga_attend")
     return (out, lse) if want_lse or lse is not None else out
 
@@ -288,6 +317,13 @@ class KVCache:
         self.s_group = torch.zeros(B, Hkv, capacity // params.g_s, D, dtype=torch.float32, **z)
         self.lens = torch.zeros(B, dtype=torch.int32, **z)
 
+    def check_device(self, device):
+        """Raise unless every cache buffer lies on `device`."""
+        for name in ("k_rot", "v", "pos", "k_open", "s_chunk", "s_group", "lens"):
+            t = getattr(self, name)
+            if t.device != device:
+                raise HGAError(f"cache.{name} is on {t.device}, the call's tensors are on {device}")
+
     def c(self) -> _Cache:
         return _Cache(self.capacity, self.k_rot.data_ptr(), self.v.data_ptr(), self.pos.data_ptr(),
                       self.k_open.data_ptr(), self.s_chunk.data_ptr(), self.s_group.data_ptr(),
@@ -295,16 +331,38 @@ class KVCache:
 
 
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor], zero: bool):
+    """(tensor kept alive for the call, 256-byte aligned base address, bytes
+    usable from that base).  A caller's workspace must lie on the call's
+    device and hold nbytes from its first 256-byte boundary on: the base is
+    rounded up, so a buffer of exactly nbytes that does not start on such a
+    boundary is refused rather than overrun."""
     if nbytes == 0:
-        return None
+        return None, None, 0
     if workspace is not None:
-        if workspace.numel() * workspace.element_size() < nbytes:
-            raise HGAError(f"workspace too small: need {nbytes} bytes")
-        return workspace
-    w = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
-    if zero:
-        w.zero_()
-    return w
+        if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+            raise HGAError("workspace must be a CUDA tensor")
+        if workspace.device != device:
+            raise HGAError(f"workspace is on {workspace.device}, the call's tensors are on {device}")
+        if not workspace.is_contiguous():
+            raise HGAError("workspace must be contiguous")
+        w = workspace
+    else:
+        w = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        if zero:
+            w.zero_()
+    base, avail = _aligned_span(w.data_ptr(), w.numel() * w.element_size(), nbytes)
+    return w, base, avail
+
+
+def _aligned_span(start: int, size: int, nbytes: int):
+    """(base, avail): the first 256-byte boundary at or after `start` and the
+    bytes of [start, start + size) from there on; raises unless avail >= nbytes."""
+    base = (start + 255) // 256 * 256
+    avail = start + size - base
+    if avail < nbytes:
+        raise HGAError(f"workspace too small: need {nbytes} bytes from its first 256-byte "
+                       f"boundary, have {max(avail, 0)}")
+    return base, avail
 
 
 def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCache] = None,
@@ -313,32 +371,36 @@ def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCa
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
+    dev = q.device
     Hkv = k.shape[2]
-    _need(k, "k", (B, T, Hkv, D), q.dtype)
-    _need(v, "v", (B, T, Hkv, D), q.dtype)
-    _need(pos, "pos", (B, T), torch.int32)
+    _need(k, "k", (B, T, Hkv, D), q.dtype, dev)
+    _need(v, "v", (B, T, Hkv, D), q.dtype, dev)
+    _need(pos, "pos", (B, T), torch.int32, dev)
     NB = (T + params.C - 1) // params.C
     res = {"out": torch.empty_like(q) if out is None else out}
+    _need(res["out"], "out", (B, T, Hq, D), q.dtype, dev)
     io = _IO()
     io.q, io.k, io.v, io.pos = q.data_ptr(), k.data_ptr(), v.data_ptr(), pos.data_ptr()
     io.out = res["out"].data_ptr()
     if want_lse:
-        res["lse"] = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+        res["lse"] = torch.empty(B, Hq, T, device=dev, dtype=torch.float32)
         io.lse = res["lse"].data_ptr()
     if want_sel:
-        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
-        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=dev, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=dev, dtype=torch.int32)
         io.sel_chunk = res["sel_chunk"].data_ptr()
         io.sel_group = res["sel_group"].data_ptr()
     if cache is not None:
+        cache.check_device(dev)
         io.cache = cache.c()
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
     nbytes = int(lib.hga_workspace_size(PREFILL, ctypes.byref(dims), ctypes.byref(pc)))
-    ws = _workspace(nbytes, q.device, workspace, zero=False)
-    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
-    st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
-                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    ws, base, avail = _workspace(nbytes, dev, workspace, zero=False)
+    with _on(dev):
+        st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                             None if base is None else ctypes.c_void_p(base), avail,
+                             _stream(stream, dev))
     _check(st, "hga_forward(prefill)")
     return res
 
@@ -352,33 +414,36 @@ def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
+    dev = q.device
     Hkv = k_host.shape[2]
     for t, name in ((k_host, "k_host"), (v_host, "v_host")):
         if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
             raise HGAError(f"{name} must be a pinned CPU tensor")
         if not t.is_contiguous() or tuple(t.shape) != (B, T, Hkv, D) or t.dtype != q.dtype:
             raise HGAError(f"{name} must be contiguous {(B, T, Hkv, D)} {q.dtype}")
-    _need(pos, "pos", (B, T), torch.int32)
+    _need(pos, "pos", (B, T), torch.int32, dev)
     NB = (T + params.C - 1) // params.C
     res = {"out": torch.empty_like(q) if out is None else out}
+    _need(res["out"], "out", (B, T, Hq, D), q.dtype, dev)
     io = _IO()
     io.q, io.k, io.v, io.pos = q.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), pos.data_ptr()
     io.out = res["out"].data_ptr()
     if want_lse:
-        res["lse"] = torch.empty(B, Hq, T, device=q.device, dtype=torch.float32)
+        res["lse"] = torch.empty(B, Hq, T, device=dev, dtype=torch.float32)
         io.lse = res["lse"].data_ptr()
     if want_sel:
-        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=q.device, dtype=torch.int32)
-        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
+        res["sel_chunk"] = torch.empty(B, NB, Hkv, params.K_c, device=dev, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, NB, Hkv, params.K_g, device=dev, dtype=torch.int32)
         io.sel_chunk = res["sel_chunk"].data_ptr()
         io.sel_group = res["sel_group"].data_ptr()
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
     nbytes = int(lib.hga_workspace_size(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc)))
-    ws = _workspace(nbytes, q.device, workspace, zero=False)
-    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
-    st = lib.hga_forward(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
-                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    ws, base, avail = _workspace(nbytes, dev, workspace, zero=False)
+    with _on(dev):
+        st = lib.hga_forward(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc),
+                             ctypes.byref(io), None if base is None else ctypes.c_void_p(base),
+                             avail, _stream(stream, dev))
     _check(st, "hga_forward(prefill, host K/V)")
     return res
 
@@ -389,15 +454,18 @@ def hga_fill_cache(k, v, pos, cache: "KVCache", params: HGAParams, *, stream=Non
     lib = load()
     _need(k, "k")
     B, T, Hkv, D = k.shape
-    _need(v, "v", (B, T, Hkv, D), k.dtype)
-    _need(pos, "pos", (B, T), torch.int32)
+    dev = k.device
+    _need(v, "v", (B, T, Hkv, D), k.dtype, dev)
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    cache.check_device(dev)
     io = _IO()
     io.k, io.v, io.pos = k.data_ptr(), v.data_ptr(), pos.data_ptr()
     io.cache = cache.c()
     dims = _dims(B, T, Hkv, Hkv, D, _dtype_code(k))
     pc = params.c()
-    st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io), None, 0,
-                         _stream(stream))
+    with _on(dev):
+        st = lib.hga_forward(PREFILL, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                             None, 0, _stream(stream, dev))
     _check(st, "hga_forward(prefill, cache fill)")
     return cache
 
@@ -412,18 +480,20 @@ def hga_forward_prefill_noalloc(q, k, v, pos, params: HGAParams, out: torch.Tens
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
+    dev = q.device
     Hkv = k.shape[2]
-    _need(k, "k", (B, T, Hkv, D), q.dtype)
-    _need(v, "v", (B, T, Hkv, D), q.dtype)
-    _need(pos, "pos", (B, T), torch.int32)
-    _need(out, "out", (B, T, Hq, D), q.dtype)
+    _need(k, "k", (B, T, Hkv, D), q.dtype, dev)
+    _need(v, "v", (B, T, Hkv, D), q.dtype, dev)
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    _need(out, "out", (B, T, Hq, D), q.dtype, dev)
     if lse is not None:
-        _need(lse, "lse", (B, Hq, T), torch.float32)
+        _need(lse, "lse", (B, Hq, T), torch.float32, dev)
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
-    st = lib.hga_forward_prefill_noalloc(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(k),
-                                         _ptr(v), _ptr(pos), _ptr(out), _ptr(lse),
-                                         _stream(stream))
+    with _on(dev):
+        st = lib.hga_forward_prefill_noalloc(ctypes.byref(dims), ctypes.byref(pc), _ptr(q),
+                                             _ptr(k), _ptr(v), _ptr(pos), _ptr(out), _ptr(lse),
+                                             _stream(stream, dev))
     _check(st, "hga_forward_prefill_noalloc")
     return out
 
@@ -436,31 +506,35 @@ def hga_forward_decode(q_new, k_new, v_new, pos_new, cache: KVCache, params: HGA
     lib = load()
     _need(q_new, "q_new")
     B, Hq, D = q_new.shape
+    dev = q_new.device
     Hkv = k_new.shape[1]
-    _need(k_new, "k_new", (B, Hkv, D), q_new.dtype)
-    _need(v_new, "v_new", (B, Hkv, D), q_new.dtype)
-    _need(pos_new, "pos_new", (B,), torch.int32)
+    _need(k_new, "k_new", (B, Hkv, D), q_new.dtype, dev)
+    _need(v_new, "v_new", (B, Hkv, D), q_new.dtype, dev)
+    _need(pos_new, "pos_new", (B,), torch.int32, dev)
+    cache.check_device(dev)
     res = {"out": torch.empty_like(q_new) if out is None else out}
+    _need(res["out"], "out", (B, Hq, D), q_new.dtype, dev)
     io = _IO()
     io.q_new, io.k_new, io.v_new = q_new.data_ptr(), k_new.data_ptr(), v_new.data_ptr()
     io.pos_new = pos_new.data_ptr()
     io.out = res["out"].data_ptr()
     if want_lse:
-        res["lse"] = torch.empty(B, Hq, device=q_new.device, dtype=torch.float32)
+        res["lse"] = torch.empty(B, Hq, device=dev, dtype=torch.float32)
         io.lse = res["lse"].data_ptr()
     if want_sel:
-        res["sel_chunk"] = torch.empty(B, Hkv, params.K_c, device=q_new.device, dtype=torch.int32)
-        res["sel_group"] = torch.empty(B, Hkv, params.K_g, device=q_new.device, dtype=torch.int32)
+        res["sel_chunk"] = torch.empty(B, Hkv, params.K_c, device=dev, dtype=torch.int32)
+        res["sel_group"] = torch.empty(B, Hkv, params.K_g, device=dev, dtype=torch.int32)
         io.sel_chunk = res["sel_chunk"].data_ptr()
         io.sel_group = res["sel_group"].data_ptr()
     io.cache = cache.c()
     dims = _dims(B, cache.capacity, Hq, Hkv, D, _dtype_code(q_new))
     pc = params.c()
     nbytes = int(lib.hga_workspace_size(DECODE, ctypes.byref(dims), ctypes.byref(pc)))
-    ws = _workspace(nbytes, q_new.device, workspace, zero=True)
-    base = None if ws is None else (ws.data_ptr() + 255) // 256 * 256
-    st = lib.hga_forward(DECODE, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
-                         None if base is None else ctypes.c_void_p(base), nbytes, _stream(stream))
+    ws, base, avail = _workspace(nbytes, dev, workspace, zero=True)
+    with _on(dev):
+        st = lib.hga_forward(DECODE, ctypes.byref(dims), ctypes.byref(pc), ctypes.byref(io),
+                             None if base is None else ctypes.c_void_p(base), avail,
+                             _stream(stream, dev))
     _check(st, "hga_forward(decode)")
     return res
 

@@ -157,7 +157,12 @@ hga_status hga_route(const hga_dims *dims, const hga_params *prm,
  * query token i of block b attends, with scale 1/sqrt(D), to the union of
  * sink chunks 0..F-1, recent chunks b-L..b-1, chunk b-1, the tokens of
  * sel_group, and tokens b*C..i of its own chunk.  q is raw (pre-RoPE) and is
- * rotated inside; k_rot comes from hga_build_summaries.  lse may be NULL. */
+ * rotated inside; k_rot comes from hga_build_summaries.  lse may be NULL.
+ * Which kernel runs: bf16 with Hq/Hkv a power of two <= 16, g_s a multiple
+ * of 8 and a visible set of at most 2048 8-token segments runs on the tensor
+ * cores (tcgen05); fp32, and bf16 outside those limits, run on the CUDA cores
+ * in fp32 arithmetic.  Both give the same result within rounding (bf16
+ * outputs are rounded from fp32 accumulators). */
 hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
                       const void *q, const int32_t *pos,
                       const void *k_rot, const void *v,
@@ -232,7 +237,11 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
  *
  * The first call on a device, with that device current, looks up the
  * array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture.  All calls share the one array:
+ * first call before any stream capture.  The cached address belongs to the
+ * device's primary context as it was then: after cudaDeviceReset on that
+ * device the address is stale, so do not call this entry point on a device
+ * after resetting it (load the library in a fresh process instead).  All
+ * calls share the one array:
  * calls that overlap on the GPU (other streams, other threads, without
  * ordering between them) race on it and give wrong results. */
 hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hga_params *prm,

@@ -186,3 +186,22 @@ def test_noalloc_rejects_oversized_shapes_on_the_host(lib):
     A = ctypes.c_void_p(1 << 24)
     st = lib.hga_forward_prefill_noalloc(by(big), by(p), A, A, A, A, A, None, None)
     assert st == 6
+
+
+@pytest.mark.parametrize("start,size,need,ok", [
+    (0x7f0000000000, 4096, 4096, True),          # aligned, exact size
+    (0x7f0000000010, 4096, 4096, False),         # unaligned slice of exactly nbytes
+    (0x7f0000000010, 4096 + 240, 4096, True),    # unaligned, enough after the boundary
+    (0x7f00000000f0, 4096 + 15, 4096, False),    # one byte short after rounding up
+])
+def test_workspace_span_accounts_for_alignment(start, size, need, ok):
+    """A caller's workspace is used from its first 256-byte boundary, and the
+    bytes passed to the library are those left from there, so a buffer that
+    starts off a boundary is refused unless the rest still holds nbytes."""
+    if ok:
+        base, avail = hga._aligned_span(start, size, need)
+        assert base % 256 == 0 and base >= start and avail >= need
+        assert base + avail == start + size
+    else:
+        with pytest.raises(hga.HGAError, match="workspace too small"):
+            hga._aligned_span(start, size, need)

@@ -60,3 +60,39 @@ def test_reference_arm_line_on_cpu(monkeypatch, capsys):
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     e = line["e2e"]
     assert e["value"] == line["value"] and e["h2d_bytes_per_step"] == e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_uses_every_host_thread_and_measures_its_step(monkeypatch, capsys):
+    # one (block, KV head) unit per host thread, and ms_per_step is the time
+    # the sampled step took, so steps x ms_per_step fits inside the run
+    import argparse
+    import json
+    import time
+    monkeypatch.setenv("RANK", "0")
+    t0 = time.perf_counter()
+    bench.run_reference(argparse.Namespace(gpus=1, steps=2, warmup=0, seed=0))
+    wall_ms = (time.perf_counter() - t0) * 1e3
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    n = len(os.sched_getaffinity(0))
+    w = WORKLOADS[bench.WORKLOAD]
+    assert line["cpu_baseline"]["cores"] == min(n, -(-n // w.Hkv) * w.Hkv)
+    assert line["steps"] * line["ms_per_step"] <= wall_ms
+    assert line["whole_workload_ms_estimate"] >= line["ms_per_step"]
+
+
+def test_smalllm_bytes():
+    # Q and O (8 heads) and K, V, rotated K (8 KV heads): 168 MB at 8 x 4096
+    w = WORKLOADS["smalllm40m_bf16_prefill_4k"]
+    assert bench.smalllm_bytes(w) == 8 * 4096 * (2 * 8 + 3 * 8) * 64 * 2
+    assert 167e6 < bench.smalllm_bytes(w) < 168e6
+
+
+def test_clock_sampler_legs_without_nvml():
+    # the per-leg summary counts only the samples inside each bracketed leg
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.max_mhz, s.period, s.legs, s._ok = [], 1965, 0.0005, {}, True
+    s.samples = [(0.5, 1900, 0), (1.5, 1965, 0x4), (2.5, 1965, 0), (3.5, 1000, 0x1)]
+    s.legs = {"prefill": [(1.0, 2.0)], "decode": [(2.0, 3.0)]}
+    r = s.result()
+    assert r["samples"] == 2 and r["sm_mhz"] == 1965 and r["reasons"] == ["sw_power_cap"]
+    assert r["legs"]["prefill"]["samples"] == 1 and r["legs"]["decode"]["samples"] == 1

@@ -35,6 +35,10 @@ CASES = {
     "bf16_qwen_2048": QWEN.replace(T=2048),
     "bf16_qwen_ragged": QWEN.replace(T=64 * 20 + 33),
     "bf16_qwen_L0_F0": QWEN.replace(T=1280, F=0, L=0, K_c=5, K_g=9),
+    # bf16 shapes the tensor-core kernel does not take (Hq/Hkv not a power of
+    # two; groups shorter than its 8-token segments) run on the CUDA cores
+    "bf16_G3_cuda_cores": QWEN.replace(T=64 * 12 + 5, Hq=6, Hkv=2, K_c=4, K_g=8),
+    "bf16_gs4_cuda_cores": SMALLLM.replace(B=1, T=900, Hq=4, Hkv=4, g_s=4, K_g=24),
 }
 
 
@@ -161,3 +165,23 @@ def test_prefill_wrapped_positions(gpu_lib, name, mod):
     RoPE and the summaries' mean positions use the given positions, while
     causality and the chunk structure follow the token index."""
     run_and_check(gpu_lib, CASES[name], seed=17, pos_mod=mod)
+
+
+@pytest.mark.slow
+def test_smalllm_4k_full_size(gpu_lib):
+    """The SmallLM-40M-shaped prefill (8 sequences x 4096 tokens, 8 heads,
+    MHA, D=64) exactly as the bench times it: every routed set of every
+    sequence checked; outputs on 64 sampled (sequence, block) pairs that
+    include the first F+L+2 blocks and the last block."""
+    w = SMALLLM
+    NB = w.T // 64
+    first = list(range(0, w.F + w.L + 2))
+    units = [(0, u) for u in first] + [(7, NB - 1)]
+    for b in range(w.B):
+        for u in (w.F + w.L + 2 + 7 * b, 31 + b, 40 + 3 * b, 50 + b, NB - 1 - b, 13 + 5 * b,
+                  22 + 2 * b, 57 - b):
+            if (b, u) not in units:
+                units.append((b, u))
+    units = units[:max(64, len(first) + 1)]
+    assert len(units) >= 64 and (7, NB - 1) in units
+    run_and_check(gpu_lib, w, seed=13, units=units)
