@@ -549,6 +549,20 @@ static void bwd_item(const or_bwd_job *J, int b, int h)
             dVb[(int64_t)j * ks + d] = 0.0;
     }
     for (int i = 0; i < T; ++i) {
+        /* A query row whose dO is zero adds nothing to any gradient (every
+         * term it contributes carries a factor dO_i, including dO_i . O_i)
+         * and its own dq is zero: such rows are skipped. */
+        int live = 0;
+        for (int hh = h * G; hh < (h + 1) * G && !live; ++hh) {
+            const double *dO = J->dO + (((int64_t)b * T + i) * J->Hq + hh) * D;
+            for (int d = 0; d < D; ++d)
+                if (dO[d] != 0.0) { live = 1; break; }
+        }
+        if (!live) {
+            for (int hh = h * G; hh < (h + 1) * G; ++hh)
+                memset(J->dQ + (((int64_t)b * T + i) * J->Hq + hh) * D, 0, sizeof(double) * (size_t)D);
+            continue;
+        }
         int c = i / p->C;
         or_visible_mark(c, i, T, J->sel_g + (((int64_t)b * J->NB + c) * J->Hkv + h) * p->K_g, p,
                         mark);

@@ -185,3 +185,25 @@ def test_backward_is_invariant_to_a_position_shift():
         moved = oracle.hga_backward(q, k, v, pos + delta, dO, p, sel)
         for a, b in zip(base, moved):
             np.testing.assert_allclose(a, b, atol=1e-9 * max(1.0, np.abs(a).max()), rtol=0)
+
+
+def test_backward_with_dO_zero_outside_sampled_blocks_equals_masked_autograd():
+    # dO nonzero on a few query blocks only (how the full-size GPU test
+    # samples): the oracle skips the other rows, and its gradients still equal
+    # automatic differentiation of the whole masked attention with that dO
+    w = WORKLOADS["tiny_f32_prefill_1k"].replace(T=64 * 7 + 9, Hq=4, Hkv=2)
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=15)
+    q, k, v, pos = q.numpy(), k.numpy(), v.numpy(), pos.numpy()
+    p = oracle.Params.of(w)
+    dO = np.random.default_rng(16).standard_normal(q.shape)
+    keep = np.zeros(w.T, bool)
+    for blk in (0, 3, 7):
+        keep[64 * blk:64 * blk + 64] = True
+    dO[:, ~keep] = 0.0
+    dO[:, 64 * 3 + 5, 1] = 0.0           # one zero row inside a kept block
+    sel = _routed(q, k, v, pos, p)
+    got = oracle.hga_backward(q, k, v, pos, dO, p, sel)
+    want = _autograd(q, k, v, pos, p.theta, _routed_mask(sel, w.B, w.T, w.Hq, w.Hkv, p), dO)
+    for g, w_ in zip(got, want):
+        np.testing.assert_allclose(g, w_, atol=1e-10, rtol=0)
+    assert np.abs(got[0][:, ~keep]).max() == 0.0
