@@ -24,9 +24,10 @@ __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "h
            "hga_attend", "hga_forward", "hga_forward_prefill", "hga_forward_decode",
            "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
            "decode_workspace", "hga_forward_prefill_hostkv", "HGAError", "PREFILL",
-           "DECODE", "PREFILL_HOSTKV", "hga_device_status", "hga_hostkv_link_bytes"]
+           "DECODE", "PREFILL_HOSTKV", "ATTEND_BACKWARD", "hga_device_status",
+           "hga_hostkv_link_bytes", "hga_attend_backward"]
 
-PREFILL, DECODE, PREFILL_HOSTKV = 0, 1, 2
+PREFILL, DECODE, PREFILL_HOSTKV, ATTEND_BACKWARD = 0, 1, 2, 3
 _F32, _BF16 = 0, 1
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libhga.so")
@@ -115,7 +116,9 @@ def load():
         lib.hga_device_status.restype = ctypes.c_int
         lib.hga_hostkv_link_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         lib.hga_hostkv_link_bytes.restype = ctypes.c_int
-        for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward"):
+        lib.hga_attend_backward.argtypes = [P] * 14 + [ctypes.c_size_t, P]
+        for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward",
+                  "hga_attend_backward"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -268,6 +271,49 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
                             _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream, dev))
     _check(st, "hga_attend")
     return (out, lse) if want_lse or lse is not None else out
+
+
+def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch.Tensor,
+                        sel_group: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                        d_out: torch.Tensor, params: HGAParams, *, dq=None, dk=None, dv=None,
+                        workspace=None, stream=None):
+    """Backward of stage 3 with the routed groups held fixed.  q, pos, k_rot,
+    v, sel_group as given to hga_attend; out and lse as it returned them;
+    d_out [B,T,Hq,D] the gradient of the loss with respect to out.  Returns
+    (dq [B,T,Hq,D], dk [B,T,Hkv,D], dv [B,T,Hkv,D]) in fp32, dq and dk with
+    respect to the raw (pre-RoPE) q and k."""
+    lib = load()
+    _need(q, "q")
+    B, T, Hq, D = q.shape
+    dev = q.device
+    Hkv = k_rot.shape[2]
+    NB = (T + params.C - 1) // params.C
+    _need(pos, "pos", (B, T), torch.int32, dev)
+    _need(k_rot, "k_rot", (B, T, Hkv, D), q.dtype, dev)
+    _need(v, "v", (B, T, Hkv, D), q.dtype, dev)
+    _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
+    _need(out, "out", (B, T, Hq, D), q.dtype, dev)
+    _need(lse, "lse", (B, Hq, T), torch.float32, dev)
+    _need(d_out, "d_out", (B, T, Hq, D), q.dtype, dev)
+    f32 = dict(device=dev, dtype=torch.float32)
+    dq = torch.empty(B, T, Hq, D, **f32) if dq is None else dq
+    dk = torch.empty(B, T, Hkv, D, **f32) if dk is None else dk
+    dv = torch.empty(B, T, Hkv, D, **f32) if dv is None else dv
+    _need(dq, "dq", (B, T, Hq, D), torch.float32, dev)
+    _need(dk, "dk", (B, T, Hkv, D), torch.float32, dev)
+    _need(dv, "dv", (B, T, Hkv, D), torch.float32, dev)
+    dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
+    pc = params.c()
+    nbytes = int(lib.hga_workspace_size(ATTEND_BACKWARD, ctypes.byref(dims), ctypes.byref(pc)))
+    ws, base, avail = _workspace(nbytes, dev, workspace, zero=False)
+    with _on(dev):
+        st = lib.hga_attend_backward(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos),
+                                     _ptr(k_rot), _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse),
+                                     _ptr(d_out), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     None if base is None else ctypes.c_void_p(base), avail,
+                                     _stream(stream, dev))
+    _check(st, "hga_attend_backward")
+    return dq, dk, dv
 
 
 def hga_device_status(clear: bool = True, stream=None) -> int:

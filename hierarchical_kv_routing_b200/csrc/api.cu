@@ -196,7 +196,32 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
     if (mode == HGA_PREFILL) return prefill_ws(g, dims->dtype).total;
     if (mode == HGA_DECODE) return decode_workspace_bytes(g);
     if (mode == HGA_PREFILL_HOSTKV) return hostkv_workspace_bytes(g);
+    if (mode == HGA_ATTEND_BACKWARD) return backward_workspace_bytes(g, dims->dtype);
     return 0;
+}
+
+hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, const void *q,
+                               const int32_t *pos, const void *k_rot, const void *v,
+                               const int32_t *sel_group, const void *out, const float *lse,
+                               const void *d_out, float *dq, float *dk, float *dv,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    hga_status s = check_common(dims, prm);
+    if (s != HGA_OK) return s;
+    if (dims->T == 0) return HGA_OK;
+    if (!q || !pos || !k_rot || !v || (prm->K_g > 0 && !sel_group) || !out || !lse || !d_out ||
+        !dq || !dk || !dv)
+        return HGA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return HGA_ERR_INVALID_ARG;
+    const Geo g = make_geo(dims, prm);
+    const size_t need = backward_workspace_bytes(g, dims->dtype);
+    if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))
+        return HGA_ERR_WORKSPACE;
+    Rope r;
+    set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
+    return launch_attend_backward(g, r, dims->dtype, q, pos, k_rot, v, sel_group, out, lse, d_out,
+                                  dq, dk, dv, workspace, (cudaStream_t)stream);
 }
 
 hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, const hga_io *io,
@@ -297,10 +322,11 @@ int hga_last_cuda_error(void) { return g_last_cuda_error; }
 hga_status hga_device_status(void *stream, int clear) {
     const cudaStream_t st = (cudaStream_t)stream;
     hga_status first = HGA_OK;
-    const hga_status parts[4] = {summaries_error_take(st, clear != 0),
+    const hga_status parts[5] = {summaries_error_take(st, clear != 0),
                                  attend_tc_error_take(st, clear != 0),
                                  decode_error_take(st, clear != 0),
-                                 tier_error_take(st, clear != 0)};
+                                 tier_error_take(st, clear != 0),
+                                 backward_error_take(st, clear != 0)};
     for (hga_status p : parts)
         if (p != HGA_OK && first == HGA_OK) first = p;
     return first;

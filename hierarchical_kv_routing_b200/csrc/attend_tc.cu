@@ -383,8 +383,10 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                                           : rope_cs_int(A.rope, p, g * 8 + 2 * e);
                         const float2 c1 = A.cs_tokens > 0 ? csr[g * 8 + 2 * e + 1]
                                                           : rope_cs_int(A.rope, p, g * 8 + 2 * e + 1);
-                        pa[e] = __floats2bfloat162_rn(x.x * c0.x - y.x * c0.y, x.y * c1.x - y.y * c1.y);
-                        pb[e] = __floats2bfloat162_rn(y.x * c0.x + x.x * c0.y, y.y * c1.x + x.y * c1.y);
+                        // the same rounding as every other rotation in the library
+                        const float2 r0 = rot_pair(x.x, y.x, c0), r1 = rot_pair(x.y, y.y, c1);
+                        pa[e] = __floats2bfloat162_rn(r0.x, r1.x);
+                        pb[e] = __floats2bfloat162_rn(r0.y, r1.y);
                     }
                     *lo = a;
                     *hi = bb;

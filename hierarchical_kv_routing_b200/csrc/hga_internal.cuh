@@ -171,6 +171,17 @@ size_t hostkv_workspace_bytes(const Geo &g);
 hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, void *ws,
                                  cudaStream_t st);
 
+// Backward of stage 3 (hga_attend_backward): dq [B,T,Hq,D], dk and dv
+// [B,T,Hkv,D], fp32.  Workspace: per query row (LSE in base 2, Delta), and
+// for the tensor-core path the rotated queries in bf16.
+size_t backward_workspace_bytes(const Geo &g, int dtype);
+hga_status launch_attend_backward(const Geo &g, const Rope &r, int dtype, const void *q,
+                                  const int32_t *pos, const void *k_rot, const void *v,
+                                  const int32_t *sel_group, const void *out, const float *lse,
+                                  const void *dout, float *dq, float *dk, float *dv, void *ws,
+                                  cudaStream_t st);
+hga_status backward_error_take(cudaStream_t st, bool clear);
+
 // Device error words (bounded-wait timeouts, bounds checks) of each kernel
 // file: read on a stream after its queued work, optionally reset.
 hga_status attend_tc_error_take(cudaStream_t st, bool clear);

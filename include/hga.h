@@ -64,7 +64,10 @@ typedef enum hga_status {
 
 typedef enum hga_dtype { HGA_F32 = 0, HGA_BF16 = 1 } hga_dtype;
 
-typedef enum hga_mode { HGA_PREFILL = 0, HGA_DECODE = 1, HGA_PREFILL_HOSTKV = 2 } hga_mode;
+typedef enum hga_mode {
+    HGA_PREFILL = 0, HGA_DECODE = 1, HGA_PREFILL_HOSTKV = 2,
+    HGA_ATTEND_BACKWARD = 3     /* hga_workspace_size only: hga_attend_backward */
+} hga_mode;
 
 /* Method parameters (page section 3 and its setup table in section 6). */
 typedef struct hga_params {
@@ -169,7 +172,36 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
                       const int32_t *sel_group, void *out, float *lse,
                       void *stream);
 
-/* Bytes of device workspace hga_forward needs for `mode` (0 if none). */
+/* Backward of stage 3 (training through the routed attention).  Page
+ * section 6, Tab. 8 (a training step through HGA attention) and Sec. 5.9
+ * (QK fine-tuning through it in the exact-token mode).  The page prints no
+ * formula; this is the derivative of eq. (1) restricted to each query's
+ * visible set, the routed groups held fixed (routing is a discrete choice, so
+ * no gradient reaches the summaries):
+ *   P_ij = exp(q~_i . k~_j / sqrt(D) - LSE_i) over j in V(i) (q~, k~ rotated)
+ *   dv_j = sum_i P_ij dO_i
+ *   dS_ij = P_ij (dO_i . v_j - dO_i . O_i)
+ *   dq_i = R_{p_i}^T sum_j dS_ij k~_j / sqrt(D)
+ *   dk_j = R_{p_j}^T sum_i dS_ij q~_i / sqrt(D)
+ * with i over the query rows of every query head of k_j's KV head.
+ * Inputs: q (raw), pos, k_rot, v and sel_group as given to hga_attend; out
+ * and lse as hga_attend returned them (lse is required); d_out [B, T, Hq, D]
+ * in the dtype of q.  Outputs, fp32: dq [B, T, Hq, D] with respect to the raw
+ * q, dk [B, T, Hkv, D] with respect to the RAW k (the rotation undone at each
+ * key's position), dv [B, T, Hkv, D]; every element is written.  workspace:
+ * hga_workspace_size(HGA_ATTEND_BACKWARD) bytes, 256-byte aligned.  bf16 with
+ * the tensor-core forward's shape limits runs on the tensor cores (tcgen05),
+ * everything else on the CUDA cores.  dk and dv are sums over units formed by
+ * atomic additions, so their low bits may differ between runs. */
+hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm,
+                               const void *q, const int32_t *pos, const void *k_rot,
+                               const void *v, const int32_t *sel_group, const void *out,
+                               const float *lse, const void *d_out, float *dq, float *dk,
+                               float *dv, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Bytes of device workspace hga_forward (or, for HGA_ATTEND_BACKWARD,
+ * hga_attend_backward) needs for `mode` (0 if none). */
 size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm);
 
 /* The whole path in one call.
