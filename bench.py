@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-hosttier", action="store_true")
     ap.add_argument("--no-cold-l2", action="store_true")
     ap.add_argument("--no-smalllm", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--decode-replays", type=int, default=10)
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling variant: only the decode part")
@@ -570,6 +571,65 @@ def bench_hosttier(args, dev, world, clk=None):
                                         "of 256 MiB, best of 5"}}
 
 
+def bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp):
+    """The backward of routed attention on the main workload (training
+    through HGA attention): hga_attend_backward after one forward with LSE,
+    timed with CUDA events; the tensor-core roofline of its algorithmic work
+    (five products per visible (row, key): S, dP, dQ, dK, dV, 2 D FLOPs each,
+    i.e. 2.5 times the forward's; the recomputations of S and dP, for Delta
+    and inside the dK/dV kernel, are not counted)."""
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_kv_routing_b200 as hga
+    stream = torch.cuda.current_stream(dev)
+    out, lse = hga.hga_attend(q, pos, k_rot, v, sel_g, hp, want_lse=True)
+    g = torch.Generator(device=dev).manual_seed(args.seed + 9)
+    d_out = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
+    B, T, Hq, D = q.shape
+    Hkv = k_rot.shape[2]
+    f32 = dict(device=dev, dtype=torch.float32)
+    dq = torch.empty(B, T, Hq, D, **f32)
+    dk = torch.empty(B, T, Hkv, D, **f32)
+    dv = torch.empty(B, T, Hkv, D, **f32)
+    n = hga.hga_workspace_size(hga.ATTEND_BACKWARD, B, T, Hq, Hkv, D, q.dtype, hp)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+
+    def call():
+        hga.hga_attend_backward(q, pos, k_rot, v, sel_g, lse, d_out, hp, dq=dq, dk=dk, dv=dv,
+                                workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize(dev)
+    steps = max(5, min(args.steps, 20))
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clk.leg("backward"):
+        e0.record(stream)
+        for _ in range(steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev, world)
+    flops = 2.5 * attention_flops(w, sel_g)
+    pk, src = peaks()
+    peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"metric": "backward tokens/s", "value": whole_job_rate(w.B * w.T, world, ms),
+            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "config": {"workload": w.name, "what": "hga_attend_backward: dq, dk, dv (fp32) from "
+                       "the forward's LSE and a random d_out; routed groups fixed"},
+            "gpu_launches_per_step": 5,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "flops_per_step": flops, "traffic": None,
+                         "kernels": "k_bwd_prep, k_bwd_dq_tc, k_bwd_dkv_tc, k_bwd_finish "
+                                    "(the call's whole time, all four kernels and two memsets)",
+                         "peak_source": f"{src} bf16_tflops (burst)"}}
+
+
 SMALLLM_WORKLOAD = "smalllm40m_bf16_prefill_4k"
 
 
@@ -800,6 +860,12 @@ def main():
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hpos))
     d2h = houts[0].numel() * houts[0].element_size()
 
+    bwd = None
+    if not (args.no_backward or args.seq):
+        try:
+            bwd = bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp)
+        except Exception as exc:               # noqa: BLE001 - reported, not raised
+            bwd = {"error": f"{type(exc).__name__}: {exc}"}
     dec = None if args.no_decode else bench_decode(args, dev, world, clk)
     tier = None if args.no_hosttier else bench_hosttier(args, dev, world, clk)
     small = None if (args.no_smalllm or args.seq) else bench_smalllm(args, dev, world, clk)
@@ -839,6 +905,8 @@ def main():
         line["hosttier"] = tier
     if small is not None:
         line["smalllm"] = small
+    if bwd is not None:
+        line["backward"] = bwd
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.seed)
     if args.seq or args.no_e2e:

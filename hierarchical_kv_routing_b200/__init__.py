@@ -25,7 +25,8 @@ __all__ = ["HGAParams", "KVCache", "load", "lib_path", "hga_build_summaries", "h
            "hga_workspace_size", "hga_forward_prefill_noalloc", "hga_fill_cache",
            "decode_workspace", "hga_forward_prefill_hostkv", "HGAError", "PREFILL",
            "DECODE", "PREFILL_HOSTKV", "ATTEND_BACKWARD", "hga_device_status",
-           "hga_hostkv_link_bytes", "hga_attend_backward"]
+           "hga_hostkv_link_bytes", "hga_attend_backward", "hga_hostkv_plan",
+           "hostkv_workspace_bytes"]
 
 PREFILL, DECODE, PREFILL_HOSTKV, ATTEND_BACKWARD = 0, 1, 2, 3
 _F32, _BF16 = 0, 1
@@ -57,6 +58,12 @@ class _Cache(ctypes.Structure):
                 ("pos", ctypes.c_void_p), ("k_open", ctypes.c_void_p),
                 ("s_chunk", ctypes.c_void_p), ("s_group", ctypes.c_void_p),
                 ("lens", ctypes.c_void_p)]
+
+
+class _HostkvPlan(ctypes.Structure):
+    _fields_ = [("wave_blocks", ctypes.c_int32), ("cache_slots", ctypes.c_int32),
+                ("bytes", ctypes.c_size_t), ("min_bytes", ctypes.c_size_t),
+                ("max_bytes", ctypes.c_size_t)]
 
 
 class _IO(ctypes.Structure):
@@ -116,7 +123,9 @@ def load():
         lib.hga_device_status.restype = ctypes.c_int
         lib.hga_hostkv_link_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         lib.hga_hostkv_link_bytes.restype = ctypes.c_int
-        lib.hga_attend_backward.argtypes = [P] * 14 + [ctypes.c_size_t, P]
+        lib.hga_attend_backward.argtypes = [P] * 13 + [ctypes.c_size_t, P]
+        lib.hga_hostkv_plan_for.argtypes = [P, P, ctypes.c_size_t, P]
+        lib.hga_hostkv_plan_for.restype = ctypes.c_int
         for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward",
                   "hga_attend_backward"):
             getattr(lib, f).restype = ctypes.c_int
@@ -274,12 +283,12 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
 
 
 def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch.Tensor,
-                        sel_group: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
-                        d_out: torch.Tensor, params: HGAParams, *, dq=None, dk=None, dv=None,
-                        workspace=None, stream=None):
+                        sel_group: torch.Tensor, lse: torch.Tensor, d_out: torch.Tensor,
+                        params: HGAParams, *, dq=None, dk=None, dv=None, workspace=None,
+                        stream=None):
     """Backward of stage 3 with the routed groups held fixed.  q, pos, k_rot,
-    v, sel_group as given to hga_attend; out and lse as it returned them;
-    d_out [B,T,Hq,D] the gradient of the loss with respect to out.  Returns
+    v, sel_group as given to hga_attend; lse as it returned it; d_out
+    [B,T,Hq,D] the gradient of the loss with respect to its output.  Returns
     (dq [B,T,Hq,D], dk [B,T,Hkv,D], dv [B,T,Hkv,D]) in fp32, dq and dk with
     respect to the raw (pre-RoPE) q and k."""
     lib = load()
@@ -292,7 +301,6 @@ def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor,
     _need(k_rot, "k_rot", (B, T, Hkv, D), q.dtype, dev)
     _need(v, "v", (B, T, Hkv, D), q.dtype, dev)
     _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
-    _need(out, "out", (B, T, Hq, D), q.dtype, dev)
     _need(lse, "lse", (B, Hq, T), torch.float32, dev)
     _need(d_out, "d_out", (B, T, Hq, D), q.dtype, dev)
     f32 = dict(device=dev, dtype=torch.float32)
@@ -308,7 +316,7 @@ def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor,
     ws, base, avail = _workspace(nbytes, dev, workspace, zero=False)
     with _on(dev):
         st = lib.hga_attend_backward(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos),
-                                     _ptr(k_rot), _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse),
+                                     _ptr(k_rot), _ptr(v), _ptr(sel_group), _ptr(lse),
                                      _ptr(d_out), _ptr(dq), _ptr(dk), _ptr(dv),
                                      None if base is None else ctypes.c_void_p(base), avail,
                                      _stream(stream, dev))
@@ -451,12 +459,48 @@ def hga_forward_prefill(q, k, v, pos, params: HGAParams, *, cache: Optional[KVCa
     return res
 
 
+def hga_hostkv_plan(B: int, T: int, Hq: int, Hkv: int, D: int, params: HGAParams,
+                    workspace_bytes: int = 0) -> dict:
+    """How the host tier uses a workspace of workspace_bytes (0: report the
+    bounds only): dict(wave_blocks, cache_slots, bytes, min_bytes, max_bytes);
+    bytes is 0 when the workspace is below min_bytes."""
+    lib = load()
+    dims = _dims(B, T, Hq, Hkv, D, _BF16)
+    pc = params.c()
+    pl = _HostkvPlan()
+    st = lib.hga_hostkv_plan_for(ctypes.byref(dims), ctypes.byref(pc), int(workspace_bytes),
+                                 ctypes.byref(pl))
+    if st not in (0, 6):
+        _check(st, "hga_hostkv_plan_for")
+    return {f: int(getattr(pl, f)) for f, _ in _HostkvPlan._fields_}
+
+
+def hostkv_workspace_bytes(B, T, Hq, Hkv, D, params: HGAParams, *, cache_bytes=None,
+                           vram_headroom=None, device="cuda") -> int:
+    """Workspace size for the host tier.  cache_bytes: a budget in bytes
+    (clamped to the tier's [min_bytes, max_bytes]).  vram_headroom: leave
+    that many bytes of the device's currently free memory unused, the warm
+    cache taking the rest up to max_bytes and shrinking down to min_bytes.
+    Neither: the default size."""
+    bounds = hga_hostkv_plan(B, T, Hq, Hkv, D, params)
+    if cache_bytes is None and vram_headroom is None:
+        return hga_workspace_size(PREFILL_HOSTKV, B, T, Hq, Hkv, D, torch.bfloat16, params)
+    if cache_bytes is None:
+        free, _ = torch.cuda.mem_get_info(torch.device(device))
+        cache_bytes = free - int(vram_headroom) - 256
+    return int(min(max(int(cache_bytes), bounds["min_bytes"]), bounds["max_bytes"]))
+
+
 def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out=None,
-                               want_lse=False, want_sel=False, workspace=None, stream=None):
+                               want_lse=False, want_sel=False, workspace=None,
+                               cache_bytes=None, vram_headroom=None, stream=None):
     """Prefill with the token K/V history in host RAM (the host-resident
     tier).  q [B,T,Hq,D] and pos [B,T] are CUDA tensors; k_host and v_host
     [B,T,Hkv,D] are pinned CPU tensors (raw keys, values).  Returns the same
-    dict as hga_forward_prefill; the outputs equal that call's."""
+    dict as hga_forward_prefill (the outputs equal that call's) plus "plan",
+    the wave size and warm-cache slots the workspace gave (see
+    hostkv_workspace_bytes for cache_bytes and vram_headroom; a caller's
+    workspace is used at its own size)."""
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
@@ -484,8 +528,13 @@ def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out
         io.sel_group = res["sel_group"].data_ptr()
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
-    nbytes = int(lib.hga_workspace_size(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc)))
+    if workspace is not None:
+        nbytes = hga_hostkv_plan(B, T, Hq, Hkv, D, params)["min_bytes"]
+    else:
+        nbytes = hostkv_workspace_bytes(B, T, Hq, Hkv, D, params, cache_bytes=cache_bytes,
+                                        vram_headroom=vram_headroom, device=dev)
     ws, base, avail = _workspace(nbytes, dev, workspace, zero=False)
+    res["plan"] = hga_hostkv_plan(B, T, Hq, Hkv, D, params, avail)
     with _on(dev):
         st = lib.hga_forward(PREFILL_HOSTKV, ctypes.byref(dims), ctypes.byref(pc),
                              ctypes.byref(io), None if base is None else ctypes.c_void_p(base),

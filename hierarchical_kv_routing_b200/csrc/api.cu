@@ -200,19 +200,27 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
     return 0;
 }
 
+hga_status hga_hostkv_plan_for(const hga_dims *dims, const hga_params *prm,
+                               size_t workspace_bytes, hga_hostkv_plan *plan) {
+    if (!plan) return HGA_ERR_INVALID_ARG;
+    const hga_status s = check_common(dims, prm);
+    if (s != HGA_OK) return s;
+    return hostkv_plan(make_geo(dims, prm), workspace_bytes, plan);
+}
+
 hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, const void *q,
                                const int32_t *pos, const void *k_rot, const void *v,
-                               const int32_t *sel_group, const void *out, const float *lse,
-                               const void *d_out, float *dq, float *dk, float *dv,
-                               void *workspace, size_t workspace_bytes, void *stream) {
+                               const int32_t *sel_group, const float *lse, const void *d_out,
+                               float *dq, float *dk, float *dv, void *workspace,
+                               size_t workspace_bytes, void *stream) {
     hga_status s = check_common(dims, prm);
     if (s != HGA_OK) return s;
     if (dims->T == 0) return HGA_OK;
-    if (!q || !pos || !k_rot || !v || (prm->K_g > 0 && !sel_group) || !out || !lse || !d_out ||
-        !dq || !dk || !dv)
+    if (!q || !pos || !k_rot || !v || (prm->K_g > 0 && !sel_group) || !lse || !d_out || !dq ||
+        !dk || !dv)
         return HGA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(out) ||
-        !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(d_out) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return HGA_ERR_INVALID_ARG;
     const Geo g = make_geo(dims, prm);
     const size_t need = backward_workspace_bytes(g, dims->dtype);
@@ -220,7 +228,7 @@ hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, cons
         return HGA_ERR_WORKSPACE;
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
-    return launch_attend_backward(g, r, dims->dtype, q, pos, k_rot, v, sel_group, out, lse, d_out,
+    return launch_attend_backward(g, r, dims->dtype, q, pos, k_rot, v, sel_group, lse, d_out,
                                   dq, dk, dv, workspace, (cudaStream_t)stream);
 }
 
@@ -233,7 +241,13 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
     const Geo g = make_geo(dims, prm);
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
-    const size_t need = hga_workspace_size(mode, dims, prm);
+    size_t need = hga_workspace_size(mode, dims, prm);
+    if (mode == HGA_PREFILL_HOSTKV) {
+        // any workspace the warm tier's smallest plan fits in
+        hga_hostkv_plan pl;
+        hostkv_plan(g, 0, &pl);
+        need = pl.min_bytes;
+    }
     const bool ws_ok =
         need == 0 || (workspace && workspace_bytes >= need && !((uintptr_t)workspace & 255u));
     char *ws = static_cast<char *>(workspace);
@@ -299,7 +313,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
             return HGA_ERR_INVALID_ARG;
         if (!aligned16(io->q) || !aligned16(io->k) || !aligned16(io->v) || !aligned16(io->out))
             return HGA_ERR_INVALID_ARG;
-        return launch_prefill_hostkv(g, r, *io, workspace, st);
+        return launch_prefill_hostkv(g, r, *io, workspace, workspace_bytes, st);
     }
     return HGA_ERR_INVALID_ARG;
 }

@@ -9,22 +9,29 @@
 // eq. (1) restricted to each query token's visible set V(i):
 //   S_ij = q~_i . k~_j / sqrt(D),  P_ij = exp(S_ij - LSE_i),  j in V(i)
 //   dV_j  = sum_i P_ij dO_i
-//   dS_ij = P_ij (dO_i . v_j - Delta_i),  Delta_i = dO_i . O_i
+//   dS_ij = P_ij (dO_i . v_j - Delta_i),  Delta_i = sum_j P_ij dO_i . v_j
 //   dq_i  = R_{p_i}^T  sum_j dS_ij k~_j / sqrt(D)
 //   dk_j  = R_{p_j}^T  sum_i dS_ij q~_i / sqrt(D)
 // where q~ = R_p(q), k~ = R_p(k) and i runs over the query rows of every
-// query head of k_j's KV head.
+// query head of k_j's KV head.  Delta_i equals dO_i . O_i; it is formed from
+// the kernels' own P and dO . v (a first pass over the keys) rather than from
+// the stored output, so that the difference dO_i . v_j - Delta_i, which
+// cancels heavily on rows whose weight sits on few keys, is taken between
+// values with the same rounding (with a bf16 output the error of dO . O
+// dominated such rows' dq).
 //
 // Kernels (bf16 on the tensor cores; fp32, and bf16 shapes the tensor-core
 // kernels do not take, on the CUDA cores):
 //   k_bwd_prep   per query row: q~ rounded to bf16 exactly as the forward
-//                rounds it, LSE in base 2, Delta = dO . O.
+//                rounds it, and the LSE (in base 2 for the tensor cores).
 //   k_bwd_dq_tc  query-major, like the forward: one CTA per (block, KV head,
 //                256-row half), two 128-row M-tiles ping-ponging; per 64-key
-//                tile S = Q~ K~^T and dP = dO V^T into TMEM, the softmax
-//                warpgroups form dS (bf16, over the S columns) and the tensor
-//                core accumulates dQ~ += dS K~ in TMEM; the epilogue rotates
-//                dQ~ back and stores fp32 rows.
+//                tile S = Q~ K~^T and dP = dO V^T into TMEM.  A first pass
+//                over the tiles sums Delta = P . dP per row (and stores it for
+//                the dK/dV kernel); in the second the softmax warpgroups form
+//                dS (bf16, over the S columns) and the tensor core
+//                accumulates dQ~ += dS K~ in TMEM; the epilogue rotates dQ~
+//                back and stores fp32 rows.
 //   k_bwd_dkv_tc key-major inside a unit: one CTA per (block, KV head) owns
 //                all 64*G query rows; per 128-key tile and 64-row subtile
 //                S^T = K~ Q~^T and dP^T = V dO^T into TMEM (lane = key), the
@@ -72,13 +79,14 @@ __device__ __forceinline__ float2 unrot_pair(float x, float y, float2 cs) {
 // ------------------------------------------------------------------ prep --
 // One warp per query row (b, t, hq).  Writes q~ (bf16, rounded exactly as
 // the forward rounds its rotated queries) when qt is non-null, and
-// rowstat = (LSE * log2(e), Delta) with Delta = dO . O.
+// rowstat.x = LSE, to base 2 (times log2 e) for the tensor-core kernels,
+// which exponentiate with ex2, natural for the CUDA-core kernel.  rowstat.y
+// (Delta) is written by the main kernels' first pass.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-k_bwd_prep(const T *__restrict__ q, const int32_t *__restrict__ pos, const T *__restrict__ out,
-           const T *__restrict__ dout, const float *__restrict__ lse, int Tlen, int Hq,
-           long long rows, __nv_bfloat16 *__restrict__ qt, float2 *__restrict__ rowstat,
-           Rope rope) {
+k_bwd_prep(const T *__restrict__ q, const int32_t *__restrict__ pos,
+           const float *__restrict__ lse, int Tlen, int Hq, long long rows,
+           __nv_bfloat16 *__restrict__ qt, float2 *__restrict__ rowstat, Rope rope) {
     constexpr int H = D / 2, PL = H / 32;     // pairs per lane
     const int lane = threadIdx.x & 31;
     const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -86,17 +94,8 @@ k_bwd_prep(const T *__restrict__ q, const int32_t *__restrict__ pos, const T *__
     const long long bt = r / Hq;              // (b, t)
     const int hq = (int)(r % Hq);
     const long long b = bt / Tlen, t = bt % Tlen;
-    const T *qr = q + r * D, *orow = out + r * D, *gr = dout + r * D;
-    float dl = 0.f;
-#pragma unroll
-    for (int e = 0; e < PL; ++e) {
-        const int i = lane * PL + e;
-        dl = fmaf(to_f(orow[i]), to_f(gr[i]), dl);
-        dl = fmaf(to_f(orow[i + H]), to_f(gr[i + H]), dl);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
     if (qt) {
+        const T *qr = q + r * D;
         const int32_t p = pos[bt];
 #pragma unroll
         for (int e = 0; e < PL; ++e) {
@@ -106,8 +105,10 @@ k_bwd_prep(const T *__restrict__ q, const int32_t *__restrict__ pos, const T *__
             qt[r * D + i + H] = __float2bfloat16_rn(rr.y);
         }
     }
-    if (lane == 0)
-        rowstat[r] = make_float2(lse[(b * Hq + hq) * Tlen + t] * kLog2e, dl);
+    if (lane == 0) {
+        const float l = lse[(b * Hq + hq) * Tlen + t];
+        rowstat[r] = make_float2(qt ? l * kLog2e : l, 0.f);
+    }
 }
 
 // ------------------------------------------------------------- finish --
@@ -146,6 +147,7 @@ k_bwd_simt(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, i
            const float2 *__restrict__ rowstat, const T *__restrict__ dout,
            float *__restrict__ dq, float *__restrict__ dk_acc, float *__restrict__ dv, Rope rope,
            float scale) {
+    // scale = 1/sqrt(D); rowstat.x = natural-log LSE
     constexpr int H = D / 2, PL = H / 32;     // pairs per lane: dims (i, i+H) of i = lane*PL+e
     extern __shared__ int keys[];
     __shared__ RunList rl;
@@ -175,8 +177,27 @@ k_bwd_simt(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, i
             gh[e] = to_f(dout[row * D + i + H]);
             dl[e] = dh[e] = 0.f;
         }
-        const float2 st = rowstat[row];
+        const float lse_i = rowstat[row].x;
         const int nvis = rl.cur_off + (tok - t0 + 1);
+        // first pass: Delta = sum_j P_ij dO_i . v_j with this kernel's own P
+        float delta = 0.f;
+        for (int kk = 0; kk < nvis; ++kk) {
+            const int j = keys[kk];
+            const int64_t kr = (((int64_t)b * Tlen + j) * Hkv + h) * D;
+            float s = 0.f, dp = 0.f;
+#pragma unroll
+            for (int e = 0; e < PL; ++e) {
+                const int i = lane * PL + e;
+                s = fmaf(ql[e], to_f(k_rot[kr + i]), fmaf(qh[e], to_f(k_rot[kr + i + H]), s));
+                dp = fmaf(gl[e], to_f(v[kr + i]), fmaf(gh[e], to_f(v[kr + i + H]), dp));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                dp += __shfl_xor_sync(0xffffffffu, dp, o);
+            }
+            delta = fmaf(expf(fmaf(s, scale, -lse_i)), dp, delta);
+        }
         for (int kk = 0; kk < nvis; ++kk) {
             const int j = keys[kk];
             const int64_t kr = (((int64_t)b * Tlen + j) * Hkv + h) * D;
@@ -196,8 +217,8 @@ k_bwd_simt(const T *__restrict__ q, const int32_t *__restrict__ pos, int Tlen, i
                 s += __shfl_xor_sync(0xffffffffu, s, o);
                 dp += __shfl_xor_sync(0xffffffffu, dp, o);
             }
-            const float pr = exp2f(fmaf(s, scale * kLog2e, -st.x));
-            const float ds = pr * (dp - st.y) * scale;
+            const float pr = expf(fmaf(s, scale, -lse_i));
+            const float ds = pr * (dp - delta) * scale;
 #pragma unroll
             for (int e = 0; e < PL; ++e) {
                 const int i = lane * PL + e;
@@ -231,7 +252,7 @@ struct BwdArgs {
     int rows_per_unit, ctas_per_unit, tokM, tokS;
     const int32_t *sel_group;
     const int32_t *pos;
-    const float2 *rowstat;
+    float2 *rowstat;      // (LSE in base 2, Delta): Delta written by the dQ kernel
     float *dq, *dk, *dv;
     float scale_log2;     // log2(e) / sqrt(D)
     float inv_sqrt_d;
@@ -404,9 +425,10 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             prefetch_tensormap(&tmV16);
             prefetch_tensormap(&tmK64);
             prefetch_tensormap(&tmV64);
-            for (int j = 0; j < ntiles && !ctl.abort; ++j) {
-                const int s = j % C::kStages;
-                if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1)) {
+            // every tile twice: the Delta pass, then the dS / dQ pass
+            for (int t = 0; t < 2 * ntiles && !ctl.abort; ++t) {
+                const int j = t % ntiles, s = t % C::kStages;
+                if (t >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((t / C::kStages) - 1) & 1)) {
                     bwd_fail(ctl);
                     break;
                 }
@@ -424,26 +446,34 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             bool ok = true;
             for (int mt = 0; mt < NT && ok; ++mt) ok = mbar_wait(&ctl.q_full[mt], 0);
             tc_fence_after();
-            for (int j = 0; j <= ntiles && ok; ++j) {
-                const int s = j % C::kStages;
+            // step t < ntiles: the Delta pass over tile t; t >= ntiles: the
+            // dS / dQ pass over tile t - ntiles
+            const int T2 = 2 * ntiles;
+            for (int t = 0; t <= T2 && ok; ++t) {
+                const int s = t % C::kStages;
+                const int j = t % ntiles;
                 for (int mt = 0; mt < NT && ok; ++mt) {
-                    if (j > 0) {
-                        // dQ~ += dS(j-1) K~(j-1): A from TMEM, K~ as an MN-major B
-                        if (!(ok = mbar_wait(&ctl.p_full[mt], (j - 1) & 1))) break;
+                    if (t > 0) {
+                        if (!(ok = mbar_wait(&ctl.p_full[mt], (t - 1) & 1))) break;
                         tc_fence_after();
-                        const int sp = (j - 1) % C::kStages;
-                        const int nsj = min(C::kSegPerTile, nseg - (j - 1) * C::kSegPerTile);
-                        const uint32_t kbase = smem_addr(smem + C::oK + sp * C::kKTile);
-                        for (int ks = 0; ks < nsj / 2; ++ks)
-                            mma_ts(tmem + mt * 256 + 128, tmem + mt * 256 + ks * 8,
-                                   smem_desc_sw128(kbase + ks * 2048, C::kKHalf, 1024), idesc_dq,
-                                   (j > 1 || ks > 0) ? 1u : 0u);
-                        if (j == ntiles) mma_commit(&ctl.o_full[mt]);
-                        else if (mt == NT - 1) mma_commit(&ctl.kv_empty[sp]);
+                        if (t - 1 >= ntiles) {
+                            // dQ~ += dS K~ of the previous tile: A from TMEM,
+                            // K~ as an MN-major B
+                            const int jp = (t - 1) - ntiles;
+                            const int sp = (t - 1) % C::kStages;
+                            const int nsj = min(C::kSegPerTile, nseg - jp * C::kSegPerTile);
+                            const uint32_t kbase = smem_addr(smem + C::oK + sp * C::kKTile);
+                            for (int ks = 0; ks < nsj / 2; ++ks)
+                                mma_ts(tmem + mt * 256 + 128, tmem + mt * 256 + ks * 8,
+                                       smem_desc_sw128(kbase + ks * 2048, C::kKHalf, 1024),
+                                       idesc_dq, (jp > 0 || ks > 0) ? 1u : 0u);
+                            if (t == T2) mma_commit(&ctl.o_full[mt]);
+                            else if (mt == NT - 1) mma_commit(&ctl.kv_empty[sp]);
+                        }
                     }
-                    if (j < ntiles) {
+                    if (t < T2) {
                         if (mt == 0) {
-                            if (!(ok = mbar_wait(&ctl.kv_full[s], (j / C::kStages) & 1))) break;
+                            if (!(ok = mbar_wait(&ctl.kv_full[s], (t / C::kStages) & 1))) break;
                             tc_fence_after();
                         }
                         const int nsj = min(C::kSegPerTile, nseg - j * C::kSegPerTile);
@@ -465,6 +495,8 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                    smem_desc_sw128(vb + ob, 16, 1024), idesc, kk > 0 ? 1u : 0u);
                         }
                         mma_commit(&ctl.s_full[mt]);
+                        // a Delta-pass tile is done with its stage once S and dP are
+                        if (t < ntiles && mt == NT - 1) mma_commit(&ctl.kv_empty[s]);
                     }
                 }
             }
@@ -483,14 +515,15 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const int head = R % A.G;
         const bool valid = mt < NT && (mt * 128 + r) < rows && tok < A.T;
         const int64_t grow = ((int64_t)b * A.T + tok) * A.Hq + (int64_t)h * A.G + head;
-        const float2 st = valid ? A.rowstat[grow] : make_float2(0.f, 0.f);
+        const float lse2 = valid ? A.rowstat[grow].x : 0.f;
         const int nvis = valid ? first_cur * 8 + (tok - t0 + 1) : 0;
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
         const float sc = A.scale_log2, isd = A.inv_sqrt_d;
         bool ok = true;
         if (mt < NT) {
-            for (int j = 0; j < ntiles && ok; ++j) {
-                if (!(ok = mbar_wait(&ctl.s_full[mt], j & 1))) {
+            float delta = 0.f;
+            for (int t = 0; t < 2 * ntiles && ok; ++t) {
+                if (!(ok = mbar_wait(&ctl.s_full[mt], t & 1))) {
                     bwd_fail(ctl);
                     break;
                 }
@@ -501,21 +534,38 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
                 tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
                 tmem_ld_wait();
-                const int gc0 = j * C::kSegPerTile * 8;
+                const int gc0 = (t % ntiles) * C::kSegPerTile * 8;
+                if (t < ntiles) {
+                    // Delta pass: sum of P dP over the row's visible keys
+                    float d8[8];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float ds[2];
+                    for (int u = 0; u < 8; ++u) d8[u] = 0.f;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = 2 * e + u;
+                    for (int col = 0; col < 64; ++col) {
                         const float p = gc0 + col < nvis
-                            ? ex2(fmaf(__uint_as_float(sv[col]), sc, -st.x)) : 0.f;
-                        ds[u] = p > 0.f ? p * (__uint_as_float(dp[col]) - st.y) * isd : 0.f;
+                            ? ex2(fmaf(__uint_as_float(sv[col]), sc, -lse2)) : 0.f;
+                        // columns past the tile's keys hold stale values: only
+                        // visible keys (p > 0) contribute
+                        d8[col & 7] += p > 0.f ? p * __uint_as_float(dp[col]) : 0.f;
                     }
-                    sv[e] = pack_bf16(ds[0], ds[1]);
+                    delta += ((d8[0] + d8[1]) + (d8[2] + d8[3])) + ((d8[4] + d8[5]) + (d8[6] + d8[7]));
+                    if (t == ntiles - 1 && valid) A.rowstat[grow].y = delta;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        float ds[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int col = 2 * e + u;
+                            const float p = gc0 + col < nvis
+                                ? ex2(fmaf(__uint_as_float(sv[col]), sc, -lse2)) : 0.f;
+                            ds[u] = p > 0.f ? p * (__uint_as_float(dp[col]) - delta) * isd : 0.f;
+                        }
+                        sv[e] = pack_bf16(ds[0], ds[1]);
+                    }
+                    tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sv[0]));
+                    tmem_st_wait();
                 }
-                tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sv[0]));
-                tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&ctl.p_full[mt]);
             }
@@ -876,7 +926,7 @@ bool make_map(CUtensorMap *m, const void *base, int D, int heads, long long n_ro
 template <int D>
 hga_status run_tc(const Geo &g, const Rope &r, const __nv_bfloat16 *qt, const int32_t *pos,
                   const void *k_rot, const void *v, const int32_t *sel_group,
-                  const float2 *rowstat, const void *dout, float *dq, float *dk, float *dv,
+                  float2 *rowstat, const void *dout, float *dq, float *dk, float *dv,
                   cudaStream_t st) {
     BwdArgs a;
     a.T = g.T;
@@ -954,7 +1004,7 @@ hga_status run_simt(const Geo &g, const Rope &r, const void *q, const int32_t *p
 
 template <typename T, int D>
 hga_status run_all(const Geo &g, const Rope &r, bool tc, const void *q, const int32_t *pos,
-                   const void *k_rot, const void *v, const int32_t *sel_group, const void *out,
+                   const void *k_rot, const void *v, const int32_t *sel_group,
                    const float *lse, const void *dout, float *dq, float *dk, float *dv, void *ws,
                    cudaStream_t st) {
     const long long qrows = (long long)g.B * g.T * g.Hq, krows = (long long)g.B * g.T * g.Hkv;
@@ -967,8 +1017,7 @@ hga_status run_all(const Geo &g, const Rope &r, bool tc, const void *q, const in
     if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, sizeof(float) * krows * D, st);
     if (e != cudaSuccess) return cuda_status(e);
     k_bwd_prep<T, D><<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
-        static_cast<const T *>(q), pos, static_cast<const T *>(out), static_cast<const T *>(dout),
-        lse, g.T, g.Hq, qrows, qt, rowstat, r);
+        static_cast<const T *>(q), pos, lse, g.T, g.Hq, qrows, qt, rowstat, r);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     hga_status s;
     if constexpr (sizeof(T) == 2) {
@@ -994,19 +1043,19 @@ size_t backward_workspace_bytes(const Geo &g, int dtype) {
 
 hga_status launch_attend_backward(const Geo &g, const Rope &r, int dtype, const void *q,
                                   const int32_t *pos, const void *k_rot, const void *v,
-                                  const int32_t *sel_group, const void *out, const float *lse,
+                                  const int32_t *sel_group, const float *lse,
                                   const void *dout, float *dq, float *dk, float *dv, void *ws,
                                   cudaStream_t st) {
     if (g.NB <= 0) return HGA_OK;
     const bool tc = dtype == HGA_BF16 && attend_tc_supported(g, dtype);
     if (dtype == HGA_BF16)
-        return g.D == 128 ? run_all<__nv_bfloat16, 128>(g, r, tc, q, pos, k_rot, v, sel_group, out,
+        return g.D == 128 ? run_all<__nv_bfloat16, 128>(g, r, tc, q, pos, k_rot, v, sel_group,
                                                         lse, dout, dq, dk, dv, ws, st)
-                          : run_all<__nv_bfloat16, 64>(g, r, tc, q, pos, k_rot, v, sel_group, out,
+                          : run_all<__nv_bfloat16, 64>(g, r, tc, q, pos, k_rot, v, sel_group,
                                                        lse, dout, dq, dk, dv, ws, st);
-    return g.D == 128 ? run_all<float, 128>(g, r, false, q, pos, k_rot, v, sel_group, out, lse,
+    return g.D == 128 ? run_all<float, 128>(g, r, false, q, pos, k_rot, v, sel_group, lse,
                                             dout, dq, dk, dv, ws, st)
-                      : run_all<float, 64>(g, r, false, q, pos, k_rot, v, sel_group, out, lse,
+                      : run_all<float, 64>(g, r, false, q, pos, k_rot, v, sel_group, lse,
                                            dout, dq, dk, dv, ws, st);
 }
 

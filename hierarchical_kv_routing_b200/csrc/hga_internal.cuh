@@ -168,8 +168,9 @@ hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const in
 
 // Prefill with K and V in pinned host memory (hga_forward HGA_PREFILL_HOSTKV).
 size_t hostkv_workspace_bytes(const Geo &g);
+hga_status hostkv_plan(const Geo &g, size_t workspace_bytes, hga_hostkv_plan *plan);
 hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, void *ws,
-                                 cudaStream_t st);
+                                 size_t ws_bytes, cudaStream_t st);
 
 // Backward of stage 3 (hga_attend_backward): dq [B,T,Hq,D], dk and dv
 // [B,T,Hkv,D], fp32.  Workspace: per query row (LSE in base 2, Delta), and
@@ -177,7 +178,7 @@ hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, 
 size_t backward_workspace_bytes(const Geo &g, int dtype);
 hga_status launch_attend_backward(const Geo &g, const Rope &r, int dtype, const void *q,
                                   const int32_t *pos, const void *k_rot, const void *v,
-                                  const int32_t *sel_group, const void *out, const float *lse,
+                                  const int32_t *sel_group, const float *lse,
                                   const void *dout, float *dq, float *dk, float *dv, void *ws,
                                   cudaStream_t st);
 hga_status backward_error_take(cudaStream_t st, bool clear);

@@ -29,7 +29,10 @@
 // form one space per tensor (staging buffer 0, buffer 1, cache), so one
 // tensor map covers every key a wave reads.  The cache holds two waves'
 // worth of routed groups per (sequence, KV head) (the fewest that CLOCK can
-// always serve), or every group of the sequence when that is fewer.
+// always serve), or every group of the sequence when that is fewer, unless
+// the caller's workspace says otherwise: a larger one holds more slots (up
+// to every group), a smaller one shrinks the wave so the staging buffers and
+// the two-wave cache fit (down to one query block per wave).
 #include <mutex>
 
 #include "hga_internal.cuh"
@@ -302,15 +305,15 @@ struct TierWs {
 
 inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-TierWs tier_ws(const Geo &g) {
+// Workspace layout for waves of W query blocks and a warm cache of NS group
+// slots per (sequence, KV head).
+TierWs tier_ws(const Geo &g, int W, long long NS) {
     TierWs w;
-    w.W = g.NB < kWave ? g.NB : kWave;
+    w.W = W;
     const int Lw = g.L > 1 ? g.L : 1;
     w.Rs = g.F * g.C + (w.W + Lw) * g.C;          // sinks and window of one buffer
     w.NG = g.NC * g.gpc;                          // groups of the sequence's closed chunks
-    const long long two_waves = 2ll * w.W * g.K_g;
-    w.NS = (int)(w.NG < two_waves ? w.NG : two_waves);
-    if (w.NS < 1) w.NS = 1;
+    w.NS = (int)(NS < 1 ? 1 : NS);
     w.cache_row0 = 2 * w.Rs;
     w.RT = w.cache_row0 + w.NS * g.g_s;
     const size_t BH = (size_t)g.B * g.Hkv;
@@ -344,6 +347,46 @@ TierWs tier_ws(const Geo &g) {
     o += up256(2 * (size_t)g.B * w.W * g.Hkv * g.K_g * 4);
     w.total = o;
     return w;
+}
+
+// The fewest slots that CLOCK can always serve for waves of W blocks: a wave
+// reads at most W * K_g distinct groups and may not evict the previous
+// wave's, so two waves' worth; never more than the sequence has groups.
+long long min_slots(const Geo &g, int W) {
+    const long long ng = (long long)g.NC * g.gpc, two = 2ll * W * g.K_g;
+    return ng < two ? ng : two;
+}
+
+int full_wave(const Geo &g) { return g.NB < kWave ? g.NB : kWave; }
+
+// The default plan: full waves, a cache of two waves' worth of groups.
+TierWs tier_default(const Geo &g) { return tier_ws(g, full_wave(g), min_slots(g, full_wave(g))); }
+
+// The plan for a workspace of `budget` bytes (the warm tier's VRAM budget):
+// with at least the default size, full waves and as many cache slots as fit,
+// up to every group of the sequence; with less, the wave shrinks (its
+// staging buffers and the cache's two-wave floor with it) until the layout
+// fits, down to one query block per wave.  ok = false when even that does
+// not fit.
+TierWs tier_plan(const Geo &g, size_t budget, bool *ok) {
+    const TierWs def = tier_default(g);
+    *ok = true;
+    if (budget >= def.total) {
+        long long lo = def.NS, hi = (long long)g.NC * g.gpc;
+        if (hi < lo) hi = lo;
+        while (lo < hi) {                         // largest NS whose layout fits
+            const long long mid = lo + (hi - lo + 1) / 2;
+            if (tier_ws(g, def.W, mid).total <= budget) lo = mid;
+            else hi = mid - 1;
+        }
+        return tier_ws(g, def.W, lo);
+    }
+    for (int W = def.W - 1; W >= 1; --W) {
+        const TierWs t = tier_ws(g, W, min_slots(g, W));
+        if (t.total <= budget) return t;
+    }
+    *ok = false;
+    return tier_ws(g, 1, min_slots(g, 1));
 }
 
 // Per-device side stream and events, created on first use.  One mutex keeps
@@ -396,10 +439,23 @@ hga_status gather(const GatherArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-size_t hostkv_workspace_bytes(const Geo &g) { return tier_ws(g).total; }
+size_t hostkv_workspace_bytes(const Geo &g) { return tier_default(g).total; }
+
+hga_status hostkv_plan(const Geo &g, size_t workspace_bytes, hga_hostkv_plan *plan) {
+    bool ok = true;
+    const TierWs t = tier_plan(g, workspace_bytes, &ok);
+    plan->wave_blocks = t.W;
+    plan->cache_slots = t.NS;
+    plan->bytes = ok ? t.total : 0;
+    plan->min_bytes = tier_ws(g, 1, min_slots(g, 1)).total;
+    const long long ng = (long long)g.NC * g.gpc;
+    plan->max_bytes = tier_ws(g, full_wave(g), ng > min_slots(g, full_wave(g)) ? ng
+                                                 : min_slots(g, full_wave(g))).total;
+    return ok ? HGA_OK : HGA_ERR_WORKSPACE;
+}
 
 hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, void *ws,
-                                 cudaStream_t st) {
+                                 size_t ws_bytes, cudaStream_t st) {
     if (!attend_tc_supported(g, HGA_BF16)) return HGA_ERR_UNSUPPORTED;
     void *dk = nullptr, *dv = nullptr;
     if (cudaHostGetDevicePointer(&dk, const_cast<void *>(io.k), 0) != cudaSuccess ||
@@ -407,7 +463,9 @@ hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, 
         cudaGetLastError();   // not pinned and mapped host memory: not sticky
         return HGA_ERR_INVALID_ARG;
     }
-    const TierWs w = tier_ws(g);
+    bool fits = true;
+    const TierWs w = tier_plan(g, ws_bytes, &fits);
+    if (!fits) return HGA_ERR_WORKSPACE;
     char *base = static_cast<char *>(ws);
     float *s_chunk = reinterpret_cast<float *>(base + w.s_chunk);
     float *s_group = reinterpret_cast<float *>(base + w.s_group);

@@ -180,13 +180,16 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
  * no gradient reaches the summaries):
  *   P_ij = exp(q~_i . k~_j / sqrt(D) - LSE_i) over j in V(i) (q~, k~ rotated)
  *   dv_j = sum_i P_ij dO_i
- *   dS_ij = P_ij (dO_i . v_j - dO_i . O_i)
+ *   dS_ij = P_ij (dO_i . v_j - Delta_i),  Delta_i = sum_j P_ij dO_i . v_j
  *   dq_i = R_{p_i}^T sum_j dS_ij k~_j / sqrt(D)
  *   dk_j = R_{p_j}^T sum_i dS_ij q~_i / sqrt(D)
- * with i over the query rows of every query head of k_j's KV head.
- * Inputs: q (raw), pos, k_rot, v and sel_group as given to hga_attend; out
- * and lse as hga_attend returned them (lse is required); d_out [B, T, Hq, D]
- * in the dtype of q.  Outputs, fp32: dq [B, T, Hq, D] with respect to the raw
+ * with i over the query rows of every query head of k_j's KV head.  Delta_i
+ * equals dO_i . O_i; the library forms it from its own P and dO . v, so the
+ * forward output is not an input (with a rounded output, the cancellation in
+ * dO . v_j - Delta_i on rows whose weight sits on few keys would magnify its
+ * rounding error).
+ * Inputs: q (raw), pos, k_rot, v and sel_group as given to hga_attend; lse as
+ * hga_attend returned it (required); d_out [B, T, Hq, D] in the dtype of q.  Outputs, fp32: dq [B, T, Hq, D] with respect to the raw
  * q, dk [B, T, Hkv, D] with respect to the RAW k (the rotation undone at each
  * key's position), dv [B, T, Hkv, D]; every element is written.  workspace:
  * hga_workspace_size(HGA_ATTEND_BACKWARD) bytes, 256-byte aligned.  bf16 with
@@ -195,10 +198,9 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
  * atomic additions, so their low bits may differ between runs. */
 hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm,
                                const void *q, const int32_t *pos, const void *k_rot,
-                               const void *v, const int32_t *sel_group, const void *out,
-                               const float *lse, const void *d_out, float *dq, float *dk,
-                               float *dv, void *workspace, size_t workspace_bytes,
-                               void *stream);
+                               const void *v, const int32_t *sel_group, const float *lse,
+                               const void *d_out, float *dq, float *dk, float *dv,
+                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Bytes of device workspace hga_forward (or, for HGA_ATTEND_BACKWARD,
  * hga_attend_backward) needs for `mode` (0 if none). */
@@ -233,9 +235,11 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   query blocks whose sink, recent and current K/V rows are fetched by the
  *   GPU over the link into two HBM staging buffers in the workspace, and
  *   whose routed groups go through a warm tier: a cache of routed groups in
- *   the workspace (page section 3's warm VRAM tier; CLOCK replacement, two
- *   waves' worth of groups per sequence and KV head, or all of them when
- *   fewer) from which hits are read and into which misses are fetched.
+ *   the workspace (page section 3's warm VRAM tier; CLOCK replacement) from
+ *   which hits are read and into which misses are fetched.  The wave size
+ *   and the cache's slots follow the workspace size (hga_hostkv_plan_for):
+ *   by default 32 blocks and two waves' worth of groups per sequence and KV
+ *   head (or all of them when fewer).
  *   This runs on a library-owned side stream (one per device, created on
  *   the first such call), the next wave's fetch overlapping this wave's
  *   attention; the call joins that stream back into `stream` before
@@ -243,7 +247,8 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   for one call.  Host memory that is not pinned and
  *   mapped returns HGA_ERR_INVALID_ARG.  The outputs equal HGA_PREFILL's.
  * workspace: hga_workspace_size(mode) bytes of device memory, 256-byte
- * aligned.  For HGA_DECODE it must be zero-filled before its first use; the
+ * aligned (HGA_PREFILL_HOSTKV: any size from the plan's min_bytes up; see
+ * hga_hostkv_plan_for).  For HGA_DECODE it must be zero-filled before its first use; the
  * library leaves it zeroed between calls.  Calls that share a workspace must
  * not overlap on the GPU. */
 hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
@@ -279,6 +284,33 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
 hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hga_params *prm,
                                        const void *q, const void *k, const void *v,
                                        const int32_t *pos, void *out, float *lse, void *stream);
+
+/* How HGA_PREFILL_HOSTKV uses a workspace of a given size: the warm tier
+ * (page section 3's bounded VRAM cache of routed groups, which shrinks to
+ * leave a configurable VRAM headroom) takes whatever the caller's workspace
+ * holds.  hga_workspace_size(HGA_PREFILL_HOSTKV) is the default: waves of 32
+ * query blocks and a cache of two waves' worth of routed groups per
+ * (sequence, KV head).  A larger workspace keeps more groups cached (fewer
+ * link bytes), up to every group of the sequence (max_bytes); a smaller one
+ * shrinks the wave, and with it the staging buffers and the cache's floor of
+ * two waves' worth, down to one query block per wave (min_bytes).  Outputs
+ * are the same for every plan.  A caller that wants a headroom sizes the
+ * workspace as the free device memory minus the headroom, clamped to
+ * [min_bytes, max_bytes]. */
+typedef struct hga_hostkv_plan {
+    int32_t wave_blocks;   /* query blocks per wave                            */
+    int32_t cache_slots;   /* warm-cache slots (one routed group each) per
+                              (sequence, KV head)                              */
+    size_t bytes;          /* workspace bytes this plan uses (0 if none fits)  */
+    size_t min_bytes;      /* the smallest workspace any plan fits in          */
+    size_t max_bytes;      /* the workspace that caches every group            */
+} hga_hostkv_plan;
+
+/* The plan hga_forward(HGA_PREFILL_HOSTKV) follows for workspace_bytes.
+ * Host only.  Returns HGA_ERR_WORKSPACE (with min_bytes filled in) when the
+ * workspace is below min_bytes; *plan must be a host pointer. */
+hga_status hga_hostkv_plan_for(const hga_dims *dims, const hga_params *prm,
+                               size_t workspace_bytes, hga_hostkv_plan *plan);
 
 /* Status recorded by the kernels themselves since the last reset: a bounded
  * wait that gave up (HGA_ERR_TIMEOUT: the kernel recorded it, released what

@@ -205,3 +205,30 @@ def test_workspace_span_accounts_for_alignment(start, size, need, ok):
     else:
         with pytest.raises(hga.HGAError, match="workspace too small"):
             hga._aligned_span(start, size, need)
+
+
+def test_hostkv_plan_bounds_and_monotone_growth(lib):
+    """The host tier's plan for a workspace size (host-only): the smallest
+    plan is one block per wave with a two-wave cache, the default is 32-block
+    waves with two waves' worth of slots, a larger workspace only adds slots
+    (up to every group), a smaller one shrinks the wave; below the minimum
+    the call reports HGA_ERR_WORKSPACE."""
+    hp = hga.HGAParams(C=64, g_s=16, F=2, L=8, K_c=16, K_g=32, rope_theta=1e6)
+    b = hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp)
+    assert b["bytes"] == 0 and b["min_bytes"] < b["max_bytes"]
+    lo = hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp, b["min_bytes"])
+    assert (lo["wave_blocks"], lo["cache_slots"], lo["bytes"]) == (1, 64, b["min_bytes"])
+    assert hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp, b["min_bytes"] - 1)["bytes"] == 0
+    d = hga.hga_workspace_size(hga.PREFILL_HOSTKV, 1, 65536, 32, 4, 128, "bf16", hp)
+    mid = hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp, d)
+    assert (mid["wave_blocks"], mid["cache_slots"], mid["bytes"]) == (32, 2 * 32 * 32, d)
+    top = hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp, b["max_bytes"])
+    assert (top["wave_blocks"], top["cache_slots"]) == (32, 65536 // 16)
+    prev = None
+    for nb in range(b["min_bytes"], b["max_bytes"] + 1, (b["max_bytes"] - b["min_bytes"]) // 37):
+        pl = hga.hga_hostkv_plan(1, 65536, 32, 4, 128, hp, nb)
+        assert 0 < pl["bytes"] <= nb
+        assert pl["cache_slots"] >= 2 * pl["wave_blocks"] * 32
+        if prev is not None:
+            assert (pl["wave_blocks"], pl["cache_slots"]) >= (prev["wave_blocks"], prev["cache_slots"])
+        prev = pl

@@ -136,16 +136,16 @@ def test_hosttier_64k_full_size(gpu_lib):
     assert torch.equal(_bits(tier["out"]), _bits(ref["out"]))
 
 
-def _fixed_link_bytes(w, T):
+def _fixed_link_bytes(w, T, W=32):
     """Bytes of sinks and windows the gathers read from host memory: the sink
     chunks for each of the first two waves, and each wave's window minus the
     tokens the previous wave's buffer already holds (same wave plan as the
-    library: 32-block waves, window from max(c0 - max(L, 1), F) to c1)."""
+    library: W-block waves, window from max(c0 - max(L, 1), F) to c1)."""
     C, NB, Lw = w.C, (T + w.C - 1) // w.C, max(w.L, 1)
     row = w.Hkv * w.D * 2 * 2                     # K and V of one token, all heads
     tokens, prev = 0, (0, 0)
-    for wave, c0 in enumerate(range(0, NB, 32)):
-        c1 = min(c0 + 32, NB)
+    for wave, c0 in enumerate(range(0, NB, W)):
+        c1 = min(c0 + W, NB)
         if wave < 2:
             tokens += min(w.F * C, T)
         nsink = min(c0, w.F)
@@ -237,3 +237,63 @@ def test_hosttier_warm_cache_follows_clock(gpu_lib):
     ns = min((w.T // w.C) * (w.C // w.g_s), 2 * 32 * w.K_g)
     misses = _clock_misses(tier["sel_group"].cpu().numpy(), 32, ns)
     assert got == _fixed_link_bytes(w, w.T) + misses * w.g_s * w.D * 2 * 2
+
+
+def test_hosttier_warm_cache_follows_the_workspace_budget(gpu_lib):
+    """The warm tier sized by the caller's workspace (the pages' warm VRAM
+    tier that shrinks to leave a headroom): from the smallest plan (one query
+    block per wave, a two-wave cache of 2 K_g slots) through the default to
+    the one that caches every group.  Every plan gives the in-HBM path's
+    outputs bit for bit, and its link bytes are the sinks and windows of its
+    wave size plus exactly the misses CLOCK has at its wave size and slot
+    count."""
+    w = QWEN.replace(T=64 * 200, K_c=2, K_g=3)
+    (q, k, v, pos), ref, tier = _run_pair(gpu_lib, w, seed=19)
+    dev = torch.device("cuda")
+    hp = _hp(w)
+    sg = tier["sel_group"].cpu().numpy()
+    bounds = gpu_lib.hga_hostkv_plan(w.B, w.T, w.Hq, w.Hkv, w.D, hp)
+    default = gpu_lib.hga_workspace_size(gpu_lib.PREFILL_HOSTKV, w.B, w.T, w.Hq, w.Hkv, w.D,
+                                         torch.bfloat16, hp)
+    lo, hi = bounds["min_bytes"], bounds["max_bytes"]
+    budgets = [lo, (lo + default) // 2, default, (default + hi) // 2, hi]
+    plans = [gpu_lib.hga_hostkv_plan(w.B, w.T, w.Hq, w.Hkv, w.D, hp, nb) for nb in budgets]
+    assert plans[0]["wave_blocks"] == 1 and plans[0]["cache_slots"] == 2 * w.K_g
+    assert plans[2]["wave_blocks"] == 32 and plans[2]["cache_slots"] == 2 * 32 * w.K_g
+    assert plans[-1]["cache_slots"] == (w.T // 64) * (64 // w.g_s)
+    assert 1 < plans[1]["wave_blocks"] < 32 and plans[2]["cache_slots"] < plans[3]["cache_slots"]
+    qd, kh, vh, pd = q.to(dev), k.pin_memory(), v.pin_memory(), pos.to(dev)
+    group = w.g_s * w.D * 2 * 2
+    for nb, plan in zip(budgets, plans):
+        assert plan["bytes"] <= nb
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        # the caching allocator hands out 512-byte aligned blocks, so all nb
+        # bytes are usable
+        assert ws.data_ptr() % 256 == 0
+        gpu_lib.hga_hostkv_link_bytes(clear=True)
+        res = gpu_lib.hga_forward_prefill_hostkv(qd, kh, vh, pd, hp, workspace=ws)
+        got = gpu_lib.hga_hostkv_link_bytes(clear=True)
+        assert gpu_lib.hga_device_status(clear=True) == 0
+        assert res["plan"]["wave_blocks"] == plan["wave_blocks"]
+        assert res["plan"]["cache_slots"] == plan["cache_slots"]
+        assert torch.equal(_bits(res["out"]), _bits(ref["out"])), plan
+        misses = _clock_misses(sg, plan["wave_blocks"], plan["cache_slots"])
+        assert got == _fixed_link_bytes(w, w.T, plan["wave_blocks"]) + misses * group, plan
+    # every group cached: each distinct routed (sequence, head, group) crosses once
+    distinct = sum(np.unique(sg[b, :, h][sg[b, :, h] >= 0]).size
+                   for b in range(w.B) for h in range(w.Hkv))
+    assert _clock_misses(sg, 32, plans[-1]["cache_slots"]) == distinct
+
+
+def test_hosttier_vram_headroom_sizes_the_cache(gpu_lib):
+    """vram_headroom: the cache takes the device's free memory above the
+    headroom, clamped to the plan's bounds; a headroom larger than the free
+    memory gives the smallest plan, a zero headroom the largest."""
+    w = QWEN.replace(T=64 * 200, K_c=2, K_g=3)
+    hp = _hp(w)
+    bounds = gpu_lib.hga_hostkv_plan(w.B, w.T, w.Hq, w.Hkv, w.D, hp)
+    free, _ = torch.cuda.mem_get_info()
+    small = gpu_lib.hostkv_workspace_bytes(w.B, w.T, w.Hq, w.Hkv, w.D, hp,
+                                           vram_headroom=free + (1 << 30))
+    big = gpu_lib.hostkv_workspace_bytes(w.B, w.T, w.Hq, w.Hkv, w.D, hp, vram_headroom=0)
+    assert small == bounds["min_bytes"] and big == bounds["max_bytes"]
