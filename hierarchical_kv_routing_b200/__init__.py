@@ -71,7 +71,8 @@ class _IO(ctypes.Structure):
                 ("pos", ctypes.c_void_p), ("q_new", ctypes.c_void_p), ("k_new", ctypes.c_void_p),
                 ("v_new", ctypes.c_void_p), ("pos_new", ctypes.c_void_p), ("out", ctypes.c_void_p),
                 ("lse", ctypes.c_void_p), ("sel_chunk", ctypes.c_void_p),
-                ("sel_group", ctypes.c_void_p), ("cache", _Cache)]
+                ("sel_group", ctypes.c_void_p), ("cache", _Cache),
+                ("s_group_host", ctypes.c_void_p)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -493,14 +494,17 @@ def hostkv_workspace_bytes(B, T, Hq, Hkv, D, params: HGAParams, *, cache_bytes=N
 
 def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out=None,
                                want_lse=False, want_sel=False, workspace=None,
-                               cache_bytes=None, vram_headroom=None, stream=None):
+                               cache_bytes=None, vram_headroom=None, s_group_host=None,
+                               stream=None):
     """Prefill with the token K/V history in host RAM (the host-resident
     tier).  q [B,T,Hq,D] and pos [B,T] are CUDA tensors; k_host and v_host
     [B,T,Hkv,D] are pinned CPU tensors (raw keys, values).  Returns the same
     dict as hga_forward_prefill (the outputs equal that call's) plus "plan",
     the wave size and warm-cache slots the workspace gave (see
     hostkv_workspace_bytes for cache_bytes and vram_headroom; a caller's
-    workspace is used at its own size)."""
+    workspace is used at its own size).  s_group_host: a pinned CPU float32
+    tensor [B, Hkv, (T//C)*(C//g_s), D] to hold the group summaries in the
+    cold tier (written by stage 1, read by routing over the link)."""
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
@@ -516,6 +520,15 @@ def hga_forward_prefill_hostkv(q, k_host, v_host, pos, params: HGAParams, *, out
     res = {"out": torch.empty_like(q) if out is None else out}
     _need(res["out"], "out", (B, T, Hq, D), q.dtype, dev)
     io = _IO()
+    if s_group_host is not None:
+        ng = (T // params.C) * (params.C // params.g_s)
+        t = s_group_host
+        if (not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned()
+                or not t.is_contiguous() or t.dtype != torch.float32
+                or tuple(t.shape) != (B, Hkv, ng, D)):
+            raise HGAError(f"s_group_host must be a pinned contiguous float32 CPU tensor "
+                           f"{(B, Hkv, ng, D)}")
+        io.s_group_host = t.data_ptr()
     io.q, io.k, io.v, io.pos = q.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), pos.data_ptr()
     io.out = res["out"].data_ptr()
     if want_lse:

@@ -252,6 +252,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
         need == 0 || (workspace && workspace_bytes >= need && !((uintptr_t)workspace & 255u));
     char *ws = static_cast<char *>(workspace);
 
+    if (io->s_group_host && mode != HGA_PREFILL_HOSTKV) return HGA_ERR_INVALID_ARG;
     if (mode == HGA_PREFILL) {
         if (dims->T == 0) return HGA_OK;
         const hga_kv_cache &cc = io->cache;
@@ -311,7 +312,8 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
         if (dims->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
         if (!io->q || !io->k || !io->v || !io->pos || !io->out || io->cache.k_rot)
             return HGA_ERR_INVALID_ARG;
-        if (!aligned16(io->q) || !aligned16(io->k) || !aligned16(io->v) || !aligned16(io->out))
+        if (!aligned16(io->q) || !aligned16(io->k) || !aligned16(io->v) || !aligned16(io->out) ||
+            !aligned16(io->s_group_host))
             return HGA_ERR_INVALID_ARG;
         return launch_prefill_hostkv(g, r, *io, workspace, workspace_bytes, st);
     }

@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
     const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
     if (threadIdx.x < n)
         cand[threadIdx.x] = pack_key(
-            (float)thread_dot_row<D, 8>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
+            (float)thread_dot_row<D, false, 8>(qr, Sc + (int64_t)(first + threadIdx.x) * D),
             first + threadIdx.x);
     __syncthreads();
     // this CTA's top K_c keys, descending and 0-padded

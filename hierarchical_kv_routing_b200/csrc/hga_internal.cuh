@@ -130,10 +130,12 @@ hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *
                             float *s_group, int nc_cap, void *k_open, int32_t *lens,
                             cudaStream_t st, bool host_src = false);
 
-// Stage 2 (prefill blocks).
+// Stage 2 (prefill blocks).  host_groups: s_group is the device address of
+// pinned host memory (read with plain loads).
 hga_status launch_route(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                         const float *s_chunk, const float *s_group, int nc_cap,
-                        int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st);
+                        int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st,
+                        bool host_groups = false);
 
 // Stage 3 (prefill blocks).  k_T / v_T: token capacity per sequence of k_rot
 // and v.  The CUDA-core kernel takes every shape; the tensor-core kernel

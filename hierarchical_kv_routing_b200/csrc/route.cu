@@ -48,7 +48,9 @@ struct RouteArgs {
     Rope rope;
 };
 
-template <typename T, int D>
+// kHostGroups: the group summary table is in pinned host memory (the host
+// tier's cold store) and its rows are read over the link with plain loads.
+template <typename T, int D, bool kHostGroups>
 __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     constexpr int H = D / 2;
     constexpr int EPW = 16 / (int)sizeof(T);     // elements per 16-byte word
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
             if (r < kc_s[k] * A.gpc) {
                 const int gid = sel_s[k][r / A.gpc] * A.gpc + r % A.gpc;
                 cand[k * A.ncap + r] =
-                    pack_key((float)thread_dot_row<D>(qr + k * D, Sg + (int64_t)gid * D), gid);
+                    pack_key((float)thread_dot_row<D, kHostGroups>(qr + k * D, Sg + (int64_t)gid * D), gid);
             }
         }
         __syncthreads();
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
         const int ng = kc * A.gpc;
         for (int r = threadIdx.x; r < ng; r += kThreads) {
             const int gid = rs.sel_c[r / A.gpc] * A.gpc + r % A.gpc;
-            ck[r] = pack_key((float)thread_dot_row<D>(qr + k * D, Sg + (int64_t)gid * D), gid);
+            ck[r] = pack_key((float)thread_dot_row<D, kHostGroups>(qr + k * D, Sg + (int64_t)gid * D), gid);
         }
         __syncthreads();
         const int kg = min(A.K_g, ng);
@@ -283,7 +285,7 @@ cudaError_t residency(const void *kern, size_t smem, int *sms, int *per_sm) {
 template <typename T, int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                const float *s_chunk, const float *s_group, int nc_cap, int32_t *sel_chunk,
-               int32_t *sel_group, cudaStream_t st) {
+               int32_t *sel_group, cudaStream_t st, bool host_groups) {
     RouteArgs a;
     a.q = q;
     a.pos = pos;
@@ -311,7 +313,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     // shared memory sized for the longest run, so the residency does not
     // depend on the run length picked below
     const size_t smem = sizeof(double) * kBlk * D + row_bytes * nmax;
-    auto kern = k_route<T, D>;
+    auto kern = host_groups ? k_route<T, D, true> : k_route<T, D, false>;
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     int sms = 0, per_sm = 0;
@@ -330,17 +332,18 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
 
 hga_status launch_route(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                         const float *s_chunk, const float *s_group, int nc_cap,
-                        int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st) {
+                        int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st,
+                        bool host_groups) {
     if (g.NB <= 0) return HGA_OK;
     if (dtype == HGA_BF16)
         return g.D == 128 ? run<__nv_bfloat16, 128>(g, r, q, pos, s_chunk, s_group, nc_cap,
-                                                     sel_chunk, sel_group, st)
+                                                     sel_chunk, sel_group, st, host_groups)
                           : run<__nv_bfloat16, 64>(g, r, q, pos, s_chunk, s_group, nc_cap,
-                                                    sel_chunk, sel_group, st);
+                                                    sel_chunk, sel_group, st, host_groups);
     return g.D == 128 ? run<float, 128>(g, r, q, pos, s_chunk, s_group, nc_cap, sel_chunk,
-                                        sel_group, st)
+                                        sel_group, st, host_groups)
                       : run<float, 64>(g, r, q, pos, s_chunk, s_group, nc_cap, sel_chunk,
-                                       sel_group, st);
+                                       sel_group, st, host_groups);
 }
 
 }  // namespace hga

@@ -279,10 +279,12 @@ __device__ __forceinline__ double quad_dot_row(const double *qr, const float *__
 
 // fp64 dot product of q (shared, fp64) with one fp32 row, by one thread
 // (the whole row streams through this thread's 16-byte loads).
-template <int D, int kBatch = 8>
+template <int D, bool kPlain = false, int kBatch = 8>
 __device__ __forceinline__ double thread_dot_row(const double *qr, const float *__restrict__ row) {
     // kBatch 16-byte loads in flight per batch (8 by default: several rows per
-    // thread and CTAs per SM cover the latency, within few registers)
+    // thread and CTAs per SM cover the latency, within few registers).
+    // kPlain: the row is in pinned host memory, read with plain loads (not
+    // the read-only path)
     const float4 *r4 = reinterpret_cast<const float4 *>(row);
     const double2 *q2 = reinterpret_cast<const double2 *>(qr);
     double s0 = 0.0, s1 = 0.0;
@@ -290,7 +292,16 @@ __device__ __forceinline__ double thread_dot_row(const double *qr, const float *
     for (int base = 0; base < D / 4; base += kBatch) {
         float4 v[kBatch];
 #pragma unroll
-        for (int e = 0; e < kBatch; ++e) v[e] = __ldg(r4 + base + e);
+        for (int e = 0; e < kBatch; ++e) {
+            if constexpr (kPlain) {
+                const float4 *p = r4 + base + e;
+                asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v[e].x), "=f"(v[e].y), "=f"(v[e].z), "=f"(v[e].w)
+                             : "l"(p));
+            } else {
+                v[e] = __ldg(r4 + base + e);
+            }
+        }
 #pragma unroll
         for (int e = 0; e < kBatch; ++e) {
             const double2 a = q2[2 * (base + e)], b = q2[2 * (base + e) + 1];

@@ -195,6 +195,9 @@ __global__ void __launch_bounds__(kCacheThreads) k_tier_cache(const CacheArgs A)
     }
 }
 
+// Adds link bytes that no gather counted (the cold tier's group summaries).
+__global__ void k_tier_count(unsigned long long bytes) { atomicAdd(&g_tier_link_bytes, bytes); }
+
 // Plain 16-byte global load (host memory is read without the read-only path).
 __device__ __forceinline__ uint4 ld16(const bf16 *p) {
     uint4 w;
@@ -469,6 +472,16 @@ hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, 
     char *base = static_cast<char *>(ws);
     float *s_chunk = reinterpret_cast<float *>(base + w.s_chunk);
     float *s_group = reinterpret_cast<float *>(base + w.s_group);
+    // group summaries in the cold tier: the caller's pinned host table
+    const bool host_groups = io.s_group_host != nullptr;
+    if (host_groups) {
+        void *dg = nullptr;
+        if (cudaHostGetDevicePointer(&dg, io.s_group_host, 0) != cudaSuccess) {
+            cudaGetLastError();   // not pinned and mapped host memory: not sticky
+            return HGA_ERR_INVALID_ARG;
+        }
+        s_group = static_cast<float *>(dg);
+    }
     int32_t *sel_c = io.sel_chunk ? io.sel_chunk : reinterpret_cast<int32_t *>(base + w.sel_c);
     int32_t *sel_g = io.sel_group ? io.sel_group : reinterpret_cast<int32_t *>(base + w.sel_g);
     bf16 *kk = reinterpret_cast<bf16 *>(base + w.kk);
@@ -488,8 +501,23 @@ hga_status launch_prefill_hostkv(const Geo &g, const Rope &r, const hga_io &io, 
                                     nullptr, g.T, s_chunk, s_group, g.NC, nullptr, nullptr, st,
                                     /*host_src=*/true);
     if (s != HGA_OK) return s;
-    s = launch_route(g, r, HGA_BF16, io.q, io.pos, s_chunk, s_group, g.NC, sel_c, sel_g, st);
+    s = launch_route(g, r, HGA_BF16, io.q, io.pos, s_chunk, s_group, g.NC, sel_c, sel_g, st,
+                     host_groups);
     if (s != HGA_OK) return s;
+    if (host_groups) {
+        // the group table written over the link, and the group rows of every
+        // block's routed chunks read back
+        long long rows = 0;
+        for (int c = 0; c < g.NB; ++c) {
+            const int n_mid = max(0, (g.L == 0 ? c - 2 : c - g.L - 1) - g.F + 1);
+            rows += min(g.K_c, n_mid);
+        }
+        const unsigned long long bytes =
+            ((unsigned long long)g.NC + (unsigned long long)rows) * g.gpc * g.D * 4ull * g.B * g.Hkv;
+        k_tier_count<<<1, 1, 0, st>>>(bytes);
+        cudaError_t ce = cudaGetLastError();
+        if (ce != cudaSuccess) return cuda_status(ce);
+    }
     // an empty group cache for this call
     cudaError_t e = cudaMemsetAsync(slot_of, 0xff, BH * (w.NG > 0 ? w.NG : 1) * 4, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(gid_of, 0xff, BH * w.NS * 4, st);

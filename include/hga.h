@@ -130,6 +130,14 @@ typedef struct hga_io {
     int32_t *sel_group;        /* optional: prefill [B, NB, Hkv, K_g];
                                   decode [B, Hkv, K_g]                         */
     hga_kv_cache cache;        /* decode: required; prefill: optional output   */
+    /* HGA_PREFILL_HOSTKV only, optional: a HOST pointer to pinned, mapped
+     * memory [B, Hkv, NC*C/g_s, D] f32 that holds the group summaries in the
+     * cold tier (page section 3's store table puts them in host RAM beside
+     * the token K/V).  Stage 1 writes them there over the link and stage 2
+     * reads only the groups of each block's routed chunks over the link
+     * (store operation "fetch group summaries"); NULL keeps them in the
+     * workspace on the GPU. */
+    float *s_group_host;
 } hga_io;
 
 /* Stage 1 — rotate keys and build mixed-RoPE summaries ("append closed
@@ -231,7 +239,9 @@ size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm)
  *   pos and out (and lse, sel_chunk, sel_group when given) are device
  *   pointers; io.cache must be empty.  bf16 only, shapes the tensor-core
  *   attention takes (g_s a multiple of 8, Hq/Hkv a power of two <= 16).
- *   Stage 1 reads K over the host link once; stage 3 runs in waves of 32
+ *   Stage 1 reads K over the host link once (with io.s_group_host set, it
+ *   also writes the group summaries there, and stage 2 reads the routed
+ *   chunks' group rows from there); stage 3 runs in waves of 32
  *   query blocks whose sink, recent and current K/V rows are fetched by the
  *   GPU over the link into two HBM staging buffers in the workspace, and
  *   whose routed groups go through a warm tier: a cache of routed groups in
@@ -324,10 +334,11 @@ hga_status hga_hostkv_plan_for(const hga_dims *dims, const hga_params *prm,
  * status otherwise, or HGA_ERR_CUDA if the copies fail. */
 hga_status hga_device_status(void *stream, int clear);
 
-/* Bytes the host tier (HGA_PREFILL_HOSTKV) has read over the host link for
- * stage 3 since the last reset: the K and V rows of sinks, windows and the
- * routed groups its warm cache did not hold (stage 1's single pass over K is
- * not counted).  Waits for the work queued on `stream`; clear != 0 resets the
+/* Bytes the host tier (HGA_PREFILL_HOSTKV) has moved over the host link
+ * since the last reset: for stage 3 the K and V rows of sinks, windows and
+ * the routed groups its warm cache did not hold; with the group summaries in
+ * host memory also the summaries stage 1 wrote there and the group rows
+ * stage 2 read (stage 1's single pass over K is not counted).  Waits for the work queued on `stream`; clear != 0 resets the
  * count.  *bytes must be a host pointer (HGA_ERR_INVALID_ARG if NULL). */
 hga_status hga_hostkv_link_bytes(void *stream, unsigned long long *bytes, int clear);
 

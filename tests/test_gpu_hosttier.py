@@ -297,3 +297,36 @@ def test_hosttier_vram_headroom_sizes_the_cache(gpu_lib):
                                            vram_headroom=free + (1 << 30))
     big = gpu_lib.hostkv_workspace_bytes(w.B, w.T, w.Hq, w.Hkv, w.D, hp, vram_headroom=0)
     assert small == bounds["min_bytes"] and big == bounds["max_bytes"]
+
+
+def test_hosttier_group_summaries_in_host_memory(gpu_lib):
+    """Group summaries in the cold tier (the pages' store table keeps them in
+    host RAM with the token K/V): stage 1 writes them into a pinned host table
+    and routing reads the routed chunks' group rows over the link.  Routed
+    sets and outputs are the in-HBM path's bit for bit, the host table holds
+    exactly the summaries stage 1 builds on the GPU, and the link carries the
+    table once plus, per block and KV head, the groups of its routed chunks."""
+    w = QWEN.replace(T=64 * 70 + 37)
+    (q, k, v, pos), ref, tier = _run_pair(gpu_lib, w, seed=23)
+    dev = torch.device("cuda")
+    hp = _hp(w)
+    NC, gpc = w.T // 64, 64 // w.g_s
+    sgh = torch.full((w.B, w.Hkv, NC * gpc, w.D), float("nan")).pin_memory()
+    qd, kh, vh, pd = q.to(dev), k.pin_memory(), v.pin_memory(), pos.to(dev)
+    gpu_lib.hga_hostkv_link_bytes(clear=True)
+    gpu_lib.hga_forward_prefill_hostkv(qd, kh, vh, pd, hp)
+    base = gpu_lib.hga_hostkv_link_bytes(clear=True)
+    cold = gpu_lib.hga_forward_prefill_hostkv(qd, kh, vh, pd, hp, want_lse=True, want_sel=True,
+                                              s_group_host=sgh)
+    got = gpu_lib.hga_hostkv_link_bytes(clear=True)
+    assert gpu_lib.hga_device_status(clear=True) == 0
+    assert torch.equal(cold["sel_chunk"], ref["sel_chunk"])
+    assert torch.equal(cold["sel_group"], ref["sel_group"])
+    assert torch.equal(_bits(cold["out"]), _bits(ref["out"]))
+    assert torch.equal(_bits(cold["lse"]), _bits(ref["lse"]))
+    _, _, s_g = gpu_lib.hga_build_summaries(k.to(dev), pd, hp)
+    torch.cuda.synchronize()
+    assert torch.equal(sgh.view(torch.int32), s_g.cpu().view(torch.int32))
+    NB = (w.T + 63) // 64
+    rows = sum(min(w.K_c, max(0, c - w.L - 1 - w.F + 1)) for c in range(NB))
+    assert got - base == (NC + rows) * gpc * w.D * 4 * w.B * w.Hkv
