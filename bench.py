@@ -557,6 +557,24 @@ def bench_hosttier(args, dev, world, clk=None):
         torch.cuda.synchronize(dev)
         best = max(best, src.numel() / (a.elapsed_time(b) / 1e3) / 1e9)
     achieved = link / (ms / 1e3) / 1e9
+    # the same prefill with the group summaries in the cold tier as well
+    NC, gpc = w.T // w.C, w.C // w.g_s
+    sgh = torch.empty(w.B, w.Hkv, NC * gpc, w.D, dtype=torch.float32).pin_memory()
+    hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws, s_group_host=sgh)
+    torch.cuda.synchronize(dev)
+    hga.hga_hostkv_link_bytes(clear=True)
+    if world > 1:
+        dist.barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with (clk.leg("hosttier") if clk else contextlib.nullcontext()):
+        c0.record(stream)
+        for _ in range(steps):
+            hga.hga_forward_prefill_hostkv(q, kh, vh, pos, hp, out=out, workspace=ws,
+                                           s_group_host=sgh)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms_cold = max_over_ranks(c0.elapsed_time(c1) / steps, dev, world)
+    link_cold = hga.hga_hostkv_link_bytes(clear=True) / steps + w.B * w.T * w.Hkv * w.D * 2
     return {"metric": "host-tier prefill tokens/s", "value": whole_job_rate(w.B * w.T, world, ms),
             "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
             "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
@@ -568,7 +586,13 @@ def bench_hosttier(args, dev, world, clk=None):
                          "unit": "GB/s", "frac": achieved / best, "bytes_per_step": link,
                          "bytes_per_step_without_cache": uncached,
                          "peak_source": "measured in this run: pinned host -> device copy "
-                                        "of 256 MiB, best of 5"}}
+                                        "of 256 MiB, best of 5"},
+            "group_summaries_in_host_memory": {
+                "value": whole_job_rate(w.B * w.T, world, ms_cold), "unit": "tokens/s",
+                "ms_per_step": ms_cold, "link_bytes_per_step": link_cold,
+                "link_gbs": link_cold / (ms_cold / 1e3) / 1e9,
+                "what": "the group summary table in pinned host RAM: written over the link by "
+                        "stage 1, the routed chunks' group rows read over the link by routing"}}
 
 
 def bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp):
