@@ -105,7 +105,8 @@ def stage_bytes(w):
     every input read once and every output written once.  Summaries: K and
     positions in, rotated K and the chunk and group summary tables out.
     Routing: Q and positions in, the two summary tables read once, the chunk
-    and group selections out."""
+    and group selections out, and for bf16 the rotated queries it hands to
+    attention."""
     e = 2 if w.dtype == "bf16" else 4
     NC = w.T // w.C
     NB = (w.T + w.C - 1) // w.C
@@ -114,6 +115,8 @@ def stage_bytes(w):
     summaries = 2 * kv + w.B * w.T * 4 + tables
     route = (w.B * w.T * w.Hq * w.D * e + w.B * w.T * 4 + tables
              + w.B * NB * w.Hkv * (w.K_c + w.K_g) * 4)
+    if w.dtype == "bf16":
+        route += w.B * w.T * w.Hq * w.D * 2
     return summaries, route
 
 
@@ -679,9 +682,12 @@ def bench_smalllm(args, dev, world, clk):
     rank = int(os.environ.get("RANK", "0"))
     q, k, v, pos, _ = make_prefill_inputs(w, seed=args.seed + 500 + rank, device=dev)
     stream = torch.cuda.current_stream(dev)
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=args.seed + rank, device=dev)
+    stream = torch.cuda.current_stream(dev)
     k_rot, s_c, s_g = hga.hga_build_summaries(k, pos, hp)
     sel_c, sel_g = hga.hga_route(q, pos, s_c, s_g, hp)
     out = torch.empty_like(q)
+    q_rot = torch.empty_like(q)             # routing hands the rotated queries to attention
 
     def step(ev=None):
         if ev:
@@ -689,10 +695,10 @@ def bench_smalllm(args, dev, world, clk):
         hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c, s_group=s_g)
         if ev:
             ev[1].record(stream)
-        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)
+        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g, q_rot=q_rot)
         if ev:
             ev[2].record(stream)
-        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out)
+        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out, q_rot=q_rot)
         if ev:
             ev[3].record(stream)
 
@@ -772,6 +778,7 @@ def main():
     k_rot, s_c, s_g = hga.hga_build_summaries(k, pos, hp)
     sel_c, sel_g = hga.hga_route(q, pos, s_c, s_g, hp)
     out = torch.empty_like(q)
+    q_rot = torch.empty_like(q)             # routing hands the rotated queries to attention
 
     def step(ev=None):
         if ev:
@@ -779,10 +786,10 @@ def main():
         hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c, s_group=s_g)
         if ev:
             ev[1].record(stream)
-        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)
+        hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g, q_rot=q_rot)
         if ev:
             ev[2].record(stream)
-        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out)
+        hga.hga_attend(q, pos, k_rot, v, sel_g, hp, out=out, q_rot=q_rot)
         if ev:
             ev[3].record(stream)
 
@@ -816,7 +823,8 @@ def main():
                 cold = cold_l2_times(
                     [lambda: hga.hga_build_summaries(k, pos, hp, k_rot=k_rot, s_chunk=s_c,
                                                      s_group=s_g),
-                     lambda: hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g)],
+                     lambda: hga.hga_route(q, pos, s_c, s_g, hp, sel_chunk=sel_c, sel_group=sel_g,
+                                           q_rot=q_rot)],
                     stream, dev)
         except Exception as exc:               # noqa: BLE001 - reported, not raised
             cold = f"{type(exc).__name__}: {exc}"

@@ -110,8 +110,10 @@ def load():
         lib = ctypes.CDLL(_LIB_PATH)
         P = ctypes.c_void_p
         lib.hga_build_summaries.argtypes = [P, P, P, P, P, P, P, P]
-        lib.hga_route.argtypes = [P, P, P, P, P, P, P, P, P]
-        lib.hga_attend.argtypes = [P, P, P, P, P, P, P, P, P, P]
+        lib.hga_route.argtypes = [P] * 10
+        lib.hga_attend.argtypes = [P] * 11
+        lib.hga_prefill_workspace_min.argtypes = [P, P]
+        lib.hga_prefill_workspace_min.restype = ctypes.c_size_t
         lib.hga_workspace_size.argtypes = [ctypes.c_int, P, P]
         lib.hga_workspace_size.restype = ctypes.c_size_t
         lib.hga_forward.argtypes = [ctypes.c_int, P, P, P, P, ctypes.c_size_t, P]
@@ -226,8 +228,10 @@ def hga_build_summaries(k_raw: torch.Tensor, pos: torch.Tensor, params: HGAParam
 
 
 def hga_route(q: torch.Tensor, pos: torch.Tensor, s_chunk: torch.Tensor, s_group: torch.Tensor,
-              params: HGAParams, *, sel_chunk=None, sel_group=None, stream=None):
-    """Stage 2.  q [B,T,Hq,D] -> sel_chunk [B,NB,Hkv,K_c], sel_group [B,NB,Hkv,K_g]."""
+              params: HGAParams, *, sel_chunk=None, sel_group=None, q_rot=None, stream=None):
+    """Stage 2.  q [B,T,Hq,D] -> sel_chunk [B,NB,Hkv,K_c], sel_group [B,NB,Hkv,K_g].
+    q_rot (bf16 only): a [B,T,Hq,D] bf16 tensor that receives the rotated
+    queries, for hga_attend's q_rot."""
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
@@ -244,19 +248,23 @@ def hga_route(q: torch.Tensor, pos: torch.Tensor, s_chunk: torch.Tensor, s_group
         sel_group = torch.empty(B, NB, Hkv, params.K_g, device=q.device, dtype=torch.int32)
     _need(sel_chunk, "sel_chunk", (B, NB, Hkv, params.K_c), torch.int32, dev)
     _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
+    if q_rot is not None:
+        _need(q_rot, "q_rot", (B, T, Hq, D), torch.bfloat16, dev)
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
     with _on(dev):
         st = lib.hga_route(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(s_chunk),
-                           _ptr(s_group), _ptr(sel_chunk), _ptr(sel_group), _stream(stream, dev))
+                           _ptr(s_group), _ptr(sel_chunk), _ptr(sel_group), _ptr(q_rot),
+                           _stream(stream, dev))
     _check(st, "hga_route")
     return sel_chunk, sel_group
 
 
 def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch.Tensor,
                sel_group: torch.Tensor, params: HGAParams, *, out=None, want_lse: bool = False,
-               lse=None, stream=None):
-    """Stage 3.  -> out [B,T,Hq,D] (and lse [B,Hq,T] f32 when asked)."""
+               lse=None, q_rot=None, stream=None):
+    """Stage 3.  -> out [B,T,Hq,D] (and lse [B,Hq,T] f32 when asked).  q_rot:
+    the rotated queries hga_route wrote (bf16), used instead of rotating q."""
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
@@ -274,11 +282,14 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
     _need(out, "out", (B, T, Hq, D), q.dtype, dev)
     if lse is not None:
         _need(lse, "lse", (B, Hq, T), torch.float32, dev)
+    if q_rot is not None:
+        _need(q_rot, "q_rot", (B, T, Hq, D), torch.bfloat16, dev)
     dims = _dims(B, T, Hq, Hkv, D, _dtype_code(q))
     pc = params.c()
     with _on(dev):
         st = lib.hga_attend(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos), _ptr(k_rot),
-                            _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _stream(stream, dev))
+                            _ptr(v), _ptr(sel_group), _ptr(out), _ptr(lse), _ptr(q_rot),
+                            _stream(stream, dev))
     _check(st, "hga_attend")
     return (out, lse) if want_lse or lse is not None else out
 

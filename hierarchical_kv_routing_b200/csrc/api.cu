@@ -100,9 +100,12 @@ Geo make_geo(const hga_dims *d, const hga_params *p) {
 inline size_t esize(int dtype) { return dtype == HGA_BF16 ? 2 : 4; }
 inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Prefill workspace: K_rot, chunk and group summaries, selections.
+// Prefill workspace: K_rot, chunk and group summaries, selections, and (for
+// shapes the tensor-core attention takes, when the workspace has room) the
+// rotated queries stage 2 writes for stage 3.  `min` is the size without
+// them.
 struct PrefillWs {
-    size_t k_rot, s_chunk, s_group, sel_c, sel_g, total;
+    size_t k_rot, s_chunk, s_group, sel_c, sel_g, q_rot, min, total;
 };
 
 PrefillWs prefill_ws(const Geo &g, int dtype) {
@@ -118,15 +121,21 @@ PrefillWs prefill_ws(const Geo &g, int dtype) {
     o += up256((size_t)g.B * g.NB * g.Hkv * g.K_c * 4);
     w.sel_g = o;
     o += up256((size_t)g.B * g.NB * g.Hkv * g.K_g * 4);
+    w.min = o;
+    w.q_rot = o;
+    if (dtype == HGA_BF16 && attend_tc_supported(g, dtype))
+        o += up256((size_t)g.B * g.T * g.Hq * g.D * 2);
     w.total = o;
     return w;
 }
 
 hga_status attend_dispatch(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                            const void *k_rot, int k_T, const void *v, int v_T,
-                           const int32_t *sel_group, void *out, float *lse, cudaStream_t st) {
+                           const int32_t *sel_group, void *out, float *lse, cudaStream_t st,
+                           const void *q_rot = nullptr) {
     if (attend_tc_supported(g, dtype))
-        return launch_attend_tc(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
+        return launch_attend_tc(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st,
+                                nullptr, q_rot);
     return launch_attend_simt(g, r, dtype, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st);
 }
 
@@ -157,7 +166,7 @@ hga_status hga_build_summaries(const hga_dims *dims, const hga_params *prm, cons
 
 hga_status hga_route(const hga_dims *dims, const hga_params *prm, const void *q, const int32_t *pos,
                      const float *s_chunk, const float *s_group, int32_t *sel_chunk,
-                     int32_t *sel_group, void *stream) {
+                     int32_t *sel_group, void *q_rot, void *stream) {
     hga_status s = check_common(dims, prm);
     if (s != HGA_OK) return s;
     if (dims->T == 0) return HGA_OK;
@@ -165,29 +174,38 @@ hga_status hga_route(const hga_dims *dims, const hga_params *prm, const void *q,
     if (!q || !pos || (has_closed && (!s_chunk || !s_group)) ||
         (prm->K_c > 0 && !sel_chunk) || (prm->K_g > 0 && !sel_group))
         return HGA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(s_chunk) || !aligned16(s_group)) return HGA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(s_chunk) || !aligned16(s_group) || !aligned16(q_rot))
+        return HGA_ERR_INVALID_ARG;
+    if (q_rot && dims->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
     const Geo g = make_geo(dims, prm);
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
     return launch_route(g, r, dims->dtype, q, pos, s_chunk, s_group, g.NC, sel_chunk, sel_group,
-                        (cudaStream_t)stream);
+                        (cudaStream_t)stream, false, q_rot);
 }
 
 hga_status hga_attend(const hga_dims *dims, const hga_params *prm, const void *q, const int32_t *pos,
                       const void *k_rot, const void *v, const int32_t *sel_group, void *out,
-                      float *lse, void *stream) {
+                      float *lse, const void *q_rot, void *stream) {
     hga_status s = check_common(dims, prm);
     if (s != HGA_OK) return s;
     if (dims->T == 0) return HGA_OK;
     if (!q || !pos || !k_rot || !v || (prm->K_g > 0 && !sel_group) || !out)
         return HGA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(out))
+    if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(q_rot))
         return HGA_ERR_INVALID_ARG;
+    if (q_rot && dims->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
     const Geo g = make_geo(dims, prm);
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
     return attend_dispatch(g, r, dims->dtype, q, pos, k_rot, g.T, v, g.T, sel_group, out, lse,
-                           (cudaStream_t)stream);
+                           (cudaStream_t)stream, q_rot);
+}
+
+size_t hga_prefill_workspace_min(const hga_dims *dims, const hga_params *prm) {
+    if (check_common(dims, prm) != HGA_OK) return 0;
+    return prefill_ws(make_geo(dims, prm), dims->dtype).min;
 }
 
 size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm) {
@@ -242,6 +260,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
     size_t need = hga_workspace_size(mode, dims, prm);
+    if (mode == HGA_PREFILL) need = prefill_ws(g, dims->dtype).min;   // q_rot when it fits
     if (mode == HGA_PREFILL_HOSTKV) {
         // any workspace the warm tier's smallest plan fits in
         hga_hostkv_plan pl;
@@ -286,11 +305,15 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, co
                              fill ? cc.v : nullptr, fill ? cc.pos : nullptr, k_T, s_chunk, s_group,
                              nc_cap, fill ? cc.k_open : nullptr, fill ? cc.lens : nullptr, st);
         if (s != HGA_OK || fill_only) return s;
+        // the rotated queries pass from stage 2 to stage 3 when the shape
+        // takes the tensor-core attention and the workspace holds them
+        void *q_rot = w.total > w.min && workspace_bytes >= w.total ? (void *)(ws + w.q_rot)
+                                                                    : nullptr;
         s = launch_route(g, r, dims->dtype, io->q, io->pos, s_chunk, s_group, nc_cap, sel_c, sel_g,
-                         st);
+                         st, false, q_rot);
         if (s != HGA_OK) return s;
         return attend_dispatch(g, r, dims->dtype, io->q, io->pos, k_rot, k_T, io->v, g.T, sel_g,
-                               io->out, io->lse, st);
+                               io->out, io->lse, st, q_rot);
     }
     if (mode == HGA_DECODE) {
         if (!ws_ok) return HGA_ERR_WORKSPACE;

@@ -17,7 +17,9 @@
 //               (SS form), then O += P V with P read from TMEM (TS form).
 //   warps 2-3   build the segment list at start.
 //   warps 4-11  two softmax warpgroups, one per M-tile; thread = TMEM lane =
-//               query row.  They rotate their Q rows in shared memory (RoPE),
+//               query row.  Unless stage 2 already wrote the rotated queries
+//               (then the Q tiles are loaded rotated), they rotate their Q
+//               rows in shared memory (RoPE),
 //               read S from TMEM, keep a running max in base 2 and rescale O
 //               in TMEM only when the max grows by more than 2^8 (exact: the
 //               final normalisation uses the same reference), write P (bf16)
@@ -74,6 +76,7 @@ struct TcArgs {
     int T, Hq, Hkv, G, NB, F, L, K_g, g_s, k_T, v_T;
     int rows_per_unit, ctas_per_unit, tokM;
     int cs_tokens;            // > 0: the CTA's (token, pair) cos/sin table is in smem
+    int prerot;               // the Q tiles are already rotated (stage 2 wrote them)
     int c0;                   // first query block of this launch
     // Host-resident tier: K/V rows come from the tier's buffers, not from the
     // token layout.  Tokens below sink_rows sit at row buf_row0 + token, other
@@ -360,7 +363,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             // RoPE of this row's query, in place in the swizzled Q tile
             bool ok = mbar_wait(&ctl.q_full[mt], 0);
             if (!ok) fail(ctl);
-            if (ok && valid) {
+            if (ok && valid && !A.prerot) {
                 uint8_t *qt = smem + C::oQ + mt * C::kTileBytes;
                 const int32_t p = ctl.s_pos[tok - tok0];
                 const float2 *csr = cs_tab + (tok - tok0) * (D / 2 + 1);
@@ -548,8 +551,9 @@ bool make_map(CUtensorMap *m, const void *base, int D, int heads, long long n_ro
 template <int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, const void *k_rot,
                int k_T, const void *v, int v_T, const int32_t *sel_group, void *out, float *lse,
-               cudaStream_t st, const TierWave *tw) {
+               cudaStream_t st, const TierWave *tw, const void *q_rot) {
     TcArgs a;
+    a.prerot = q_rot != nullptr;
     a.c0 = tw ? tw->c0 : 0;
     a.sink_rows = tw ? tw->sink_rows : 0;
     a.win_tok0 = tw ? tw->win_tok0 : 0;
@@ -576,7 +580,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         // the table costs tokens x D/2 x 8 bytes; keep the CTA inside 227 KB
         const int tok_cta = (min(256, a.rows_per_unit) + g.G - 1) / g.G;
         const size_t tab = (size_t)tok_cta * (D / 2 + 1) * sizeof(float2);
-        a.cs_tokens = Cfg<D>::oEnd + 1024 + tab + sizeof(Ctl) <= 232448 ? tok_cta : 0;
+        a.cs_tokens = !a.prerot && Cfg<D>::oEnd + 1024 + tab + sizeof(Ctl) <= 232448 ? tok_cta : 0;
     }
     a.sel_group = sel_group;
     a.pos = pos;
@@ -585,7 +589,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     a.rope = r;
     CUtensorMap mq, mk, mv, mk16, mv16, mk64, mv64;
-    if (!make_map(&mq, q, D, g.Hq, (long long)g.B * g.T, g.G, a.tokM) ||
+    if (!make_map(&mq, q_rot ? q_rot : q, D, g.Hq, (long long)g.B * g.T, g.G, a.tokM) ||
         !make_map(&mk, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 8) ||
         !make_map(&mv, v, D, g.Hkv, (long long)g.B * v_T, 1, 8) ||
         !make_map(&mk16, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 16) ||
@@ -615,10 +619,11 @@ bool attend_tc_supported(const Geo &g, int dtype) {
 hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                             const void *k_rot, int k_T, const void *v, int v_T,
                             const int32_t *sel_group, void *out, float *lse, cudaStream_t st,
-                            const TierWave *tw) {
+                            const TierWave *tw, const void *q_rot) {
     if (g.NB <= 0 || (tw && tw->c1 <= tw->c0)) return HGA_OK;
-    return g.D == 128 ? run<128>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw)
-                      : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw);
+    return g.D == 128
+        ? run<128>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw, q_rot)
+        : run<64>(g, r, q, pos, k_rot, k_T, v, v_T, sel_group, out, lse, st, tw, q_rot);
 }
 
 

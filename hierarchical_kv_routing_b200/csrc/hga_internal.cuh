@@ -131,11 +131,13 @@ hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *
                             cudaStream_t st, bool host_src = false);
 
 // Stage 2 (prefill blocks).  host_groups: s_group is the device address of
-// pinned host memory (read with plain loads).
+// pinned host memory (read with plain loads).  q_rot (bf16 only, may be
+// null): the rotated queries [B, T, Hq, D] are written there, rounded as the
+// tensor-core attention rounds its own rotation.
 hga_status launch_route(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                         const float *s_chunk, const float *s_group, int nc_cap,
                         int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st,
-                        bool host_groups = false);
+                        bool host_groups = false, void *q_rot = nullptr);
 
 // Stage 3 (prefill blocks).  k_T / v_T: token capacity per sequence of k_rot
 // and v.  The CUDA-core kernel takes every shape; the tensor-core kernel
@@ -162,11 +164,13 @@ struct TierWave {
     const int32_t *rt_map;
 };
 
-// tw == nullptr: every query block, keys at their token rows.
+// tw == nullptr: every query block, keys at their token rows.  q_rot
+// non-null: the queries are already rotated (stage 2 wrote them) and q is
+// not read.
 hga_status launch_attend_tc(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                             const void *k_rot, int k_T, const void *v, int v_T,
                             const int32_t *sel_group, void *out, float *lse, cudaStream_t st,
-                            const TierWave *tw = nullptr);
+                            const TierWave *tw = nullptr, const void *q_rot = nullptr);
 
 // Prefill with K and V in pinned host memory (hga_forward HGA_PREFILL_HOSTKV).
 size_t hostkv_workspace_bytes(const Geo &g);

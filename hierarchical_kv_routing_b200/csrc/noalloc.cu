@@ -41,8 +41,10 @@ extern "C" hga_status hga_forward_prefill_noalloc(const hga_dims *dims, const hg
                                                   const int32_t *pos, void *out, float *lse,
                                                   void *stream) {
     using namespace hga;
-    // 0 for malformed arguments: hga_forward then reports them
-    const size_t need = hga_workspace_size(HGA_PREFILL, dims, prm);
+    // the smallest prefill workspace (0 for malformed arguments: hga_forward
+    // then reports them); with room to spare hga_forward also keeps the
+    // rotated queries in the scratch
+    const size_t need = hga_prefill_workspace_min(dims, prm);
     if (need > kNoAllocScratchBytes) return HGA_ERR_WORKSPACE;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -41,6 +41,7 @@ constexpr size_t kCandBytes = 160 * 1024;        // shared candidate table budge
 
 struct RouteArgs {
     const void *q;
+    __nv_bfloat16 *q_rot;        // optional (bf16 only): rotated queries out
     const int32_t *pos;
     int T, Hq, Hkv, G, NB, F, L, K_c, K_g, gpc, nc_cap, nblk, ncap;
     const float *s_chunk, *s_group;
@@ -50,13 +51,16 @@ struct RouteArgs {
 
 // kHostGroups: the group summary table is in pinned host memory (the host
 // tier's cold store) and its rows are read over the link with plain loads.
-template <typename T, int D, bool kHostGroups>
+// kWriteQ (bf16): every head's rotated query is also written to A.q_rot; the
+// (token, pair) angles are then held across the head loop, so fewer head
+// rows are kept in flight to stay within the register budget.
+template <typename T, int D, bool kHostGroups, bool kWriteQ>
 __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     constexpr int H = D / 2;
     constexpr int EPW = 16 / (int)sizeof(T);     // elements per 16-byte word
     constexpr int NS = H / EPW;                  // words per half row
     constexpr int TP = kThreads / NS;            // tokens per pass
-    constexpr int HB = sizeof(T) == 2 ? 8 : 4;   // head rows in flight per thread
+    constexpr int HB = sizeof(T) == 2 && !kWriteQ ? 8 : 4;   // head rows in flight per thread
     extern __shared__ __align__(16) unsigned char smem[];
     double *qr = reinterpret_cast<double *>(smem);                            // [kBlk][D]
     unsigned long long *cand = reinterpret_cast<unsigned long long *>(qr + kBlk * D);
@@ -84,7 +88,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
 #pragma unroll
         for (int e = 0; e < EPW; ++e) al[e] = ah[e] = 0.0;
         for (int j = jt; j < n; j += TP) {
-            const T *row = q + (((int64_t)b * A.T + t0 + j) * A.Hq + (int64_t)h * A.G) * D;
+            const int64_t row0 = ((int64_t)b * A.T + t0 + j) * A.Hq + (int64_t)h * A.G;
+            const T *row = q + row0 * D;
+            const int32_t p = A.pos[(int64_t)b * A.T + t0 + j];
+            // the angles of this word's pairs serve every head and the sum
+            // (formed up front only when every head is rotated and written)
+            float2 cs[EPW];
+            if constexpr (kWriteQ)
+#pragma unroll
+                for (int e = 0; e < EPW; ++e) cs[e] = rope_cs_int(A.rope, p, w * EPW + e);
             float lo[EPW], hi[EPW];
 #pragma unroll
             for (int e = 0; e < EPW; ++e) lo[e] = hi[e] = 0.f;
@@ -107,12 +119,31 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
                             lo[e] += a[e];
                             hi[e] += c[e];
                         }
+                        if constexpr (kWriteQ && sizeof(T) == 2) {
+                            // this head's rotated query, rounded as the
+                            // attention kernel rounds its own rotation
+                            {
+                                uint4 ol, oh;
+                                __nv_bfloat162 *pl = reinterpret_cast<__nv_bfloat162 *>(&ol);
+                                __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&oh);
+#pragma unroll
+                                for (int e = 0; e < EPW / 2; ++e) {
+                                    const float2 r0 = rot_pair(a[2 * e], c[2 * e], cs[2 * e]);
+                                    const float2 r1 = rot_pair(a[2 * e + 1], c[2 * e + 1], cs[2 * e + 1]);
+                                    pl[e] = __floats2bfloat162_rn(r0.x, r1.x);
+                                    ph[e] = __floats2bfloat162_rn(r0.y, r1.y);
+                                }
+                                __nv_bfloat16 *orow = A.q_rot + (row0 + g0 + u) * D;
+                                reinterpret_cast<uint4 *>(orow)[w] = ol;
+                                reinterpret_cast<uint4 *>(orow + H)[w] = oh;
+                            }
+                        }
                     }
             }
-            const int32_t p = A.pos[(int64_t)b * A.T + t0 + j];
 #pragma unroll
             for (int e = 0; e < EPW; ++e) {
-                const float2 rr = rot_pair(lo[e], hi[e], rope_cs_int(A.rope, p, w * EPW + e));
+                if constexpr (!kWriteQ) cs[e] = rope_cs_int(A.rope, p, w * EPW + e);
+                const float2 rr = rot_pair(lo[e], hi[e], cs[e]);
                 al[e] += (double)rr.x;
                 ah[e] += (double)rr.y;
             }
@@ -285,9 +316,10 @@ cudaError_t residency(const void *kern, size_t smem, int *sms, int *per_sm) {
 template <typename T, int D>
 hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
                const float *s_chunk, const float *s_group, int nc_cap, int32_t *sel_chunk,
-               int32_t *sel_group, cudaStream_t st, bool host_groups) {
+               int32_t *sel_group, cudaStream_t st, bool host_groups, void *q_rot) {
     RouteArgs a;
     a.q = q;
+    a.q_rot = static_cast<__nv_bfloat16 *>(q_rot);
     a.pos = pos;
     a.T = g.T;
     a.Hq = g.Hq;
@@ -313,7 +345,8 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     // shared memory sized for the longest run, so the residency does not
     // depend on the run length picked below
     const size_t smem = sizeof(double) * kBlk * D + row_bytes * nmax;
-    auto kern = host_groups ? k_route<T, D, true> : k_route<T, D, false>;
+    auto kern = host_groups ? k_route<T, D, true, false>
+                            : (q_rot ? k_route<T, D, false, true> : k_route<T, D, false, false>);
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     int sms = 0, per_sm = 0;
@@ -333,17 +366,18 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
 hga_status launch_route(const Geo &g, const Rope &r, int dtype, const void *q, const int32_t *pos,
                         const float *s_chunk, const float *s_group, int nc_cap,
                         int32_t *sel_chunk, int32_t *sel_group, cudaStream_t st,
-                        bool host_groups) {
+                        bool host_groups, void *q_rot) {
     if (g.NB <= 0) return HGA_OK;
     if (dtype == HGA_BF16)
         return g.D == 128 ? run<__nv_bfloat16, 128>(g, r, q, pos, s_chunk, s_group, nc_cap,
-                                                     sel_chunk, sel_group, st, host_groups)
+                                                     sel_chunk, sel_group, st, host_groups, q_rot)
                           : run<__nv_bfloat16, 64>(g, r, q, pos, s_chunk, s_group, nc_cap,
-                                                    sel_chunk, sel_group, st, host_groups);
+                                                    sel_chunk, sel_group, st, host_groups, q_rot);
+    if (q_rot) return HGA_ERR_UNSUPPORTED;       // rotated queries are written in bf16 only
     return g.D == 128 ? run<float, 128>(g, r, q, pos, s_chunk, s_group, nc_cap, sel_chunk,
-                                        sel_group, st, host_groups)
+                                        sel_group, st, host_groups, nullptr)
                       : run<float, 64>(g, r, q, pos, s_chunk, s_group, nc_cap, sel_chunk,
-                                       sel_group, st, host_groups);
+                                       sel_group, st, host_groups, nullptr);
 }
 
 }  // namespace hga

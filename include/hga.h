@@ -157,11 +157,14 @@ hga_status hga_build_summaries(const hga_dims *dims, const hga_params *prm,
  * over the KV head's query heads; middle chunks F..b-L-1 (minus the forced
  * previous chunk when L == 0) are scored by q.c_m, the top K_c kept, their
  * groups scored by q.g_{m,g} and the top K_g kept.  Ties in score go to the
- * lower index.  Outputs sel_chunk / sel_group as in the header comment. */
+ * lower index.  Outputs sel_chunk / sel_group as in the header comment.
+ * q_rot (bf16 only, may be NULL; HGA_ERR_UNSUPPORTED for fp32): when given,
+ * [B, T, Hq, D] bf16 receives every query rotated at its position, rounded
+ * as hga_attend rounds its own rotation, for hga_attend's q_rot. */
 hga_status hga_route(const hga_dims *dims, const hga_params *prm,
                      const void *q, const int32_t *pos,
                      const float *s_chunk, const float *s_group,
-                     int32_t *sel_chunk, int32_t *sel_group, void *stream);
+                     int32_t *sel_chunk, int32_t *sel_group, void *q_rot, void *stream);
 
 /* Stage 3 — exact softmax attention over the routed token set.  Page section
  * 3, "精确 Token 输出注意力" (exact token output attention) with eq. (1): each
@@ -169,6 +172,9 @@ hga_status hga_route(const hga_dims *dims, const hga_params *prm,
  * sink chunks 0..F-1, recent chunks b-L..b-1, chunk b-1, the tokens of
  * sel_group, and tokens b*C..i of its own chunk.  q is raw (pre-RoPE) and is
  * rotated inside; k_rot comes from hga_build_summaries.  lse may be NULL.
+ * q_rot (bf16 only, may be NULL): the rotated queries hga_route wrote; the
+ * tensor-core kernel then loads them as they are instead of rotating q (the
+ * result is bit-identical), q is still required for the CUDA-core kernel.
  * Which kernel runs: bf16 with Hq/Hkv a power of two <= 16, g_s a multiple
  * of 8 and a visible set of at most 2048 8-token segments runs on the tensor
  * cores (tcgen05); fp32, and bf16 outside those limits, run on the CUDA cores
@@ -178,7 +184,7 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
                       const void *q, const int32_t *pos,
                       const void *k_rot, const void *v,
                       const int32_t *sel_group, void *out, float *lse,
-                      void *stream);
+                      const void *q_rot, void *stream);
 
 /* Backward of stage 3 (training through the routed attention).  Page
  * section 6, Tab. 8 (a training step through HGA attention) and Sec. 5.9
@@ -211,8 +217,16 @@ hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm,
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /* Bytes of device workspace hga_forward (or, for HGA_ATTEND_BACKWARD,
- * hga_attend_backward) needs for `mode` (0 if none). */
+ * hga_attend_backward) needs for `mode` (0 if none).  For HGA_PREFILL this
+ * includes room for the rotated queries stage 2 hands to stage 3 (bf16
+ * shapes of the tensor-core attention); hga_forward(HGA_PREFILL) also accepts
+ * a workspace of hga_prefill_workspace_min bytes and then rotates the
+ * queries inside stage 3 instead (same results). */
 size_t hga_workspace_size(int mode, const hga_dims *dims, const hga_params *prm);
+
+/* The smallest workspace hga_forward(HGA_PREFILL) accepts (0 if the
+ * arguments are malformed): rotated keys, summaries and routed ids only. */
+size_t hga_prefill_workspace_min(const hga_dims *dims, const hga_params *prm);
 
 /* The whole path in one call.
  * HGA_PREFILL: stages 1-3 over the T prompt tokens (K_rot, summaries and
@@ -278,7 +292,7 @@ hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm,
  * scratch (rotated keys, summaries, routed ids) lives in one fixed 16 MiB
  * array inside the library's device image, which every GPU that loads the
  * library keeps until the process exits.  A shape whose scratch
- * (hga_workspace_size(HGA_PREFILL, ...)) exceeds 16 MiB is rejected with
+ * (hga_prefill_workspace_min) exceeds 16 MiB is rejected with
  * HGA_ERR_WORKSPACE before anything is launched; about 14K tokens fit at
  * Hkv=4, D=128, bf16.  Nothing in the scratch needs to start at zero.
  *

@@ -79,7 +79,8 @@ def test_bad_params_rejected_before_launch(lib, bad, code):
 def test_null_buffers_rejected(lib):
     p = hga.HGAParams(rope_theta=1e4).c()
     d = _dims()
-    st = lib.hga_route(ctypes.byref(d), ctypes.byref(p), None, None, None, None, None, None, None)
+    st = lib.hga_route(ctypes.byref(d), ctypes.byref(p), None, None, None, None, None, None, None,
+                       None)
     assert st == 1
     io = hga._IO()
     st = lib.hga_forward(0, ctypes.byref(d), ctypes.byref(p), ctypes.byref(io), None, 0, None)

@@ -67,10 +67,19 @@ def run_and_check(hga, w, seed, units=None, sample_rows=None, pos_mod=None):
     out, lse = hga.hga_attend(qd, pd, k_rot, vd, sel_g, hp, want_lse=True)
     res = hga.hga_forward_prefill(qd, kd, vd, pd, hp, want_lse=True, want_sel=True)
     torch.cuda.synchronize()
-    # the one-call path runs the same kernels: identical results
+    # the one-call path runs the same kernels (for bf16 with the rotated
+    # queries handed from routing to attention): identical results
+    bits = torch.int16 if w.dtype == "bf16" else torch.int32
     assert torch.equal(res["sel_chunk"], sel_c) and torch.equal(res["sel_group"], sel_g)
-    assert torch.equal(res["out"].view(torch.int16 if w.dtype == "bf16" else torch.int32),
-                       out.view(torch.int16 if w.dtype == "bf16" else torch.int32))
+    assert torch.equal(res["out"].view(bits), out.view(bits))
+    if w.dtype == "bf16":
+        # the stage calls with the hand-off: the same bits again
+        q_rot = torch.empty_like(qd)
+        sc2, sg2 = hga.hga_route(qd, pd, s_c, s_g, hp, q_rot=q_rot)
+        out2, lse2 = hga.hga_attend(qd, pd, k_rot, vd, sg2, hp, want_lse=True, q_rot=q_rot)
+        torch.cuda.synchronize()
+        assert torch.equal(sg2, sel_g) and torch.equal(out2.view(bits), out.view(bits))
+        assert torch.equal(lse2, lse)
 
     # stage 1: K_rot and summaries
     ref = RouteRef(q, k, pos, p, w.Hkv)
