@@ -598,10 +598,11 @@ def bench_hosttier(args, dev, world, clk=None):
                         "stage 1, the routed chunks' group rows read over the link by routing"}}
 
 
-def bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp):
+def bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp, q_rot):
     """The backward of routed attention on the main workload (training
     through HGA attention): hga_attend_backward after one forward with LSE,
-    timed with CUDA events; the tensor-core roofline of its algorithmic work
+    given the rotated queries the forward's routing wrote, timed with CUDA
+    events; the tensor-core roofline of its algorithmic work
     (five products per visible (row, key): S, dP, dQ, dK, dV, 2 D FLOPs each,
     i.e. 2.5 times the forward's; the recomputations of S and dP, for Delta
     and inside the dK/dV kernel, are not counted)."""
@@ -624,7 +625,7 @@ def bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp):
 
     def call():
         hga.hga_attend_backward(q, pos, k_rot, v, sel_g, lse, d_out, hp, dq=dq, dk=dk, dv=dv,
-                                workspace=ws)
+                                workspace=ws, q_rot=q_rot)
 
     for _ in range(max(3, args.warmup)):
         call()
@@ -895,7 +896,7 @@ def main():
     bwd = None
     if not (args.no_backward or args.seq):
         try:
-            bwd = bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp)
+            bwd = bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp, q_rot)
         except Exception as exc:               # noqa: BLE001 - reported, not raised
             bwd = {"error": f"{type(exc).__name__}: {exc}"}
     dec = None if args.no_decode else bench_decode(args, dev, world, clk)

@@ -126,7 +126,7 @@ def load():
         lib.hga_device_status.restype = ctypes.c_int
         lib.hga_hostkv_link_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         lib.hga_hostkv_link_bytes.restype = ctypes.c_int
-        lib.hga_attend_backward.argtypes = [P] * 13 + [ctypes.c_size_t, P]
+        lib.hga_attend_backward.argtypes = [P] * 14 + [ctypes.c_size_t, P]
         lib.hga_hostkv_plan_for.argtypes = [P, P, ctypes.c_size_t, P]
         lib.hga_hostkv_plan_for.restype = ctypes.c_int
         for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward",
@@ -297,12 +297,13 @@ def hga_attend(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch
 def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor, v: torch.Tensor,
                         sel_group: torch.Tensor, lse: torch.Tensor, d_out: torch.Tensor,
                         params: HGAParams, *, dq=None, dk=None, dv=None, workspace=None,
-                        stream=None):
+                        q_rot=None, stream=None):
     """Backward of stage 3 with the routed groups held fixed.  q, pos, k_rot,
     v, sel_group as given to hga_attend; lse as it returned it; d_out
     [B,T,Hq,D] the gradient of the loss with respect to its output.  Returns
     (dq [B,T,Hq,D], dk [B,T,Hkv,D], dv [B,T,Hkv,D]) in fp32, dq and dk with
-    respect to the raw (pre-RoPE) q and k."""
+    respect to the raw (pre-RoPE) q and k.  q_rot: the rotated queries the
+    forward's hga_route wrote (bf16), which spares rotating q again."""
     lib = load()
     _need(q, "q")
     B, T, Hq, D = q.shape
@@ -315,6 +316,8 @@ def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor,
     _need(sel_group, "sel_group", (B, NB, Hkv, params.K_g), torch.int32, dev)
     _need(lse, "lse", (B, Hq, T), torch.float32, dev)
     _need(d_out, "d_out", (B, T, Hq, D), q.dtype, dev)
+    if q_rot is not None:
+        _need(q_rot, "q_rot", (B, T, Hq, D), torch.bfloat16, dev)
     f32 = dict(device=dev, dtype=torch.float32)
     dq = torch.empty(B, T, Hq, D, **f32) if dq is None else dq
     dk = torch.empty(B, T, Hkv, D, **f32) if dk is None else dk
@@ -329,7 +332,7 @@ def hga_attend_backward(q: torch.Tensor, pos: torch.Tensor, k_rot: torch.Tensor,
     with _on(dev):
         st = lib.hga_attend_backward(ctypes.byref(dims), ctypes.byref(pc), _ptr(q), _ptr(pos),
                                      _ptr(k_rot), _ptr(v), _ptr(sel_group), _ptr(lse),
-                                     _ptr(d_out), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _ptr(d_out), _ptr(q_rot), _ptr(dq), _ptr(dk), _ptr(dv),
                                      None if base is None else ctypes.c_void_p(base), avail,
                                      _stream(stream, dev))
     _check(st, "hga_attend_backward")

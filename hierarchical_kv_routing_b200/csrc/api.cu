@@ -229,8 +229,8 @@ hga_status hga_hostkv_plan_for(const hga_dims *dims, const hga_params *prm,
 hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, const void *q,
                                const int32_t *pos, const void *k_rot, const void *v,
                                const int32_t *sel_group, const float *lse, const void *d_out,
-                               float *dq, float *dk, float *dv, void *workspace,
-                               size_t workspace_bytes, void *stream) {
+                               const void *q_rot, float *dq, float *dk, float *dv,
+                               void *workspace, size_t workspace_bytes, void *stream) {
     hga_status s = check_common(dims, prm);
     if (s != HGA_OK) return s;
     if (dims->T == 0) return HGA_OK;
@@ -238,8 +238,9 @@ hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, cons
         !dk || !dv)
         return HGA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_rot) || !aligned16(v) || !aligned16(d_out) ||
-        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(q_rot))
         return HGA_ERR_INVALID_ARG;
+    if (q_rot && dims->dtype != HGA_BF16) return HGA_ERR_UNSUPPORTED;
     const Geo g = make_geo(dims, prm);
     const size_t need = backward_workspace_bytes(g, dims->dtype);
     if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))
@@ -247,7 +248,7 @@ hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm, cons
     Rope r;
     set_rope(&r, g.D, prm->rope_theta, prm->hf_wavelength, prm->C);
     return launch_attend_backward(g, r, dims->dtype, q, pos, k_rot, v, sel_group, lse, d_out,
-                                  dq, dk, dv, workspace, (cudaStream_t)stream);
+                                  dq, dk, dv, workspace, q_rot, (cudaStream_t)stream);
 }
 
 hga_status hga_forward(int mode, const hga_dims *dims, const hga_params *prm, const hga_io *io,

@@ -158,8 +158,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         tmem_alloc(&ctl.tmem_base, 512);
         tc_fence_before();
     }
-    if (warp == 3) {
-        // positions of the CTA's tokens, one coalesced load
+    if (warp == 3 && !A.prerot) {
+        // positions of the CTA's tokens (for the rotation), one coalesced load
         const int tk0 = t0 + row0 / A.G;
         for (int j = lane; j < kChunk; j += 32)
             ctl.s_pos[j] = tk0 + j < A.T ? A.pos[(int64_t)b * A.T + tk0 + j] : 0;
@@ -271,7 +271,9 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
             bool ok = true;
-            for (int mt = 0; mt < NT && ok; ++mt) ok = mbar_wait(&ctl.q_ready[mt], 0);
+            // rotated Q tiles are ready as soon as they land
+            for (int mt = 0; mt < NT && ok; ++mt)
+                ok = mbar_wait(A.prerot ? &ctl.q_full[mt] : &ctl.q_ready[mt], 0);
             tc_fence_after();
             auto issue_pv = [&](int mt, int jj) {
                 const int sp = jj % C::kStages;
@@ -361,7 +363,8 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
         if (mt < NT) {
             // RoPE of this row's query, in place in the swizzled Q tile
-            bool ok = mbar_wait(&ctl.q_full[mt], 0);
+            // (rotated tiles need no wait here: the MMA issuer waits for them)
+            bool ok = A.prerot || mbar_wait(&ctl.q_full[mt], 0);
             if (!ok) fail(ctl);
             if (ok && valid && !A.prerot) {
                 uint8_t *qt = smem + C::oQ + mt * C::kTileBytes;

@@ -77,37 +77,48 @@ __device__ __forceinline__ float2 unrot_pair(float x, float y, float2 cs) {
 }
 
 // ------------------------------------------------------------------ prep --
-// One warp per query row (b, t, hq).  Writes q~ (bf16, rounded exactly as
-// the forward rounds its rotated queries) when qt is non-null, and
-// rowstat.x = LSE, to base 2 (times log2 e) for the tensor-core kernels,
-// which exponentiate with ex2, natural for the CUDA-core kernel.  rowstat.y
-// (Delta) is written by the main kernels' first pass.
+// One thread per 8 rotate-half pairs of a query row (b, t, hq): 16-byte
+// loads of the pairs' low and high halves; writes q~ (bf16, rounded exactly
+// as the forward rounds its rotated queries) when qt is non-null.  The
+// word's first thread also writes rowstat.x = LSE, to base 2 (times log2 e)
+// for the tensor-core kernels, which exponentiate with ex2, natural for the
+// CUDA-core kernel.  rowstat.y (Delta) is written by the main kernels' first
+// pass.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 k_bwd_prep(const T *__restrict__ q, const int32_t *__restrict__ pos,
-           const float *__restrict__ lse, int Tlen, int Hq, long long rows,
+           const float *__restrict__ lse, int Tlen, int Hq, long long rows, int log2_lse,
            __nv_bfloat16 *__restrict__ qt, float2 *__restrict__ rowstat, Rope rope) {
-    constexpr int H = D / 2, PL = H / 32;     // pairs per lane
-    const int lane = threadIdx.x & 31;
-    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (r >= rows) return;                    // whole warps leave together
+    constexpr int H = D / 2, W = H / 8;       // words of 8 pairs per row
+    const long long x = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (x >= rows * W) return;
+    const long long r = x / W;
+    const int w = (int)(x % W);
     const long long bt = r / Hq;              // (b, t)
     const int hq = (int)(r % Hq);
     const long long b = bt / Tlen, t = bt % Tlen;
     if (qt) {
-        const T *qr = q + r * D;
+        float lo[8], hi[8];
+        load_slice<T, 8>(q + r * D + w * 8, lo);
+        load_slice<T, 8>(q + r * D + H + w * 8, hi);
         const int32_t p = pos[bt];
+        uint4 ol, oh;
+        __nv_bfloat162 *pl = reinterpret_cast<__nv_bfloat162 *>(&ol);
+        __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&oh);
 #pragma unroll
-        for (int e = 0; e < PL; ++e) {
-            const int i = lane * PL + e;
-            const float2 rr = rot_pair(to_f(qr[i]), to_f(qr[i + H]), rope_cs_int(rope, p, i));
-            qt[r * D + i] = __float2bfloat16_rn(rr.x);
-            qt[r * D + i + H] = __float2bfloat16_rn(rr.y);
+        for (int e = 0; e < 4; ++e) {
+            const float2 r0 = rot_pair(lo[2 * e], hi[2 * e], rope_cs_int(rope, p, w * 8 + 2 * e));
+            const float2 r1 =
+                rot_pair(lo[2 * e + 1], hi[2 * e + 1], rope_cs_int(rope, p, w * 8 + 2 * e + 1));
+            pl[e] = __floats2bfloat162_rn(r0.x, r1.x);
+            ph[e] = __floats2bfloat162_rn(r0.y, r1.y);
         }
+        reinterpret_cast<uint4 *>(qt + r * D)[w] = ol;
+        reinterpret_cast<uint4 *>(qt + r * D + H)[w] = oh;
     }
-    if (lane == 0) {
+    if (w == 0) {
         const float l = lse[(b * Hq + hq) * Tlen + t];
-        rowstat[r] = make_float2(qt ? l * kLog2e : l, 0.f);
+        rowstat[r] = make_float2(log2_lse ? l * kLog2e : l, 0.f);
     }
 }
 
@@ -1006,18 +1017,22 @@ template <typename T, int D>
 hga_status run_all(const Geo &g, const Rope &r, bool tc, const void *q, const int32_t *pos,
                    const void *k_rot, const void *v, const int32_t *sel_group,
                    const float *lse, const void *dout, float *dq, float *dk, float *dv, void *ws,
-                   cudaStream_t st) {
+                   const void *q_rot, cudaStream_t st) {
     const long long qrows = (long long)g.B * g.T * g.Hq, krows = (long long)g.B * g.T * g.Hkv;
     char *w = static_cast<char *>(ws);
     float2 *rowstat = reinterpret_cast<float2 *>(w);
-    __nv_bfloat16 *qt = tc ? reinterpret_cast<__nv_bfloat16 *>(
-                                 w + ((sizeof(float2) * qrows + 255) & ~(size_t)255))
-                           : nullptr;
+    // the rotated queries: the caller's (the forward's routing wrote them),
+    // else rotated here into the workspace
+    __nv_bfloat16 *qt = tc && !q_rot ? reinterpret_cast<__nv_bfloat16 *>(
+                                           w + ((sizeof(float2) * qrows + 255) & ~(size_t)255))
+                                     : nullptr;
     cudaError_t e = cudaMemsetAsync(dk, 0, sizeof(float) * krows * D, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, sizeof(float) * krows * D, st);
     if (e != cudaSuccess) return cuda_status(e);
-    k_bwd_prep<T, D><<<(unsigned)((qrows + 7) / 8), 256, 0, st>>>(
-        static_cast<const T *>(q), pos, lse, g.T, g.Hq, qrows, qt, rowstat, r);
+    constexpr int W = D / 16;
+    k_bwd_prep<T, D><<<(unsigned)((qrows * W + 255) / 256), 256, 0, st>>>(
+        static_cast<const T *>(q), pos, lse, g.T, g.Hq, qrows, tc ? 1 : 0, qt, rowstat, r);
+    if (tc && q_rot) qt = const_cast<__nv_bfloat16 *>(static_cast<const __nv_bfloat16 *>(q_rot));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     hga_status s;
     if constexpr (sizeof(T) == 2) {
@@ -1045,18 +1060,18 @@ hga_status launch_attend_backward(const Geo &g, const Rope &r, int dtype, const 
                                   const int32_t *pos, const void *k_rot, const void *v,
                                   const int32_t *sel_group, const float *lse,
                                   const void *dout, float *dq, float *dk, float *dv, void *ws,
-                                  cudaStream_t st) {
+                                  const void *q_rot, cudaStream_t st) {
     if (g.NB <= 0) return HGA_OK;
     const bool tc = dtype == HGA_BF16 && attend_tc_supported(g, dtype);
     if (dtype == HGA_BF16)
         return g.D == 128 ? run_all<__nv_bfloat16, 128>(g, r, tc, q, pos, k_rot, v, sel_group,
-                                                        lse, dout, dq, dk, dv, ws, st)
+                                                        lse, dout, dq, dk, dv, ws, q_rot, st)
                           : run_all<__nv_bfloat16, 64>(g, r, tc, q, pos, k_rot, v, sel_group,
-                                                       lse, dout, dq, dk, dv, ws, st);
+                                                       lse, dout, dq, dk, dv, ws, q_rot, st);
     return g.D == 128 ? run_all<float, 128>(g, r, false, q, pos, k_rot, v, sel_group, lse,
-                                            dout, dq, dk, dv, ws, st)
+                                            dout, dq, dk, dv, ws, q_rot, st)
                       : run_all<float, 64>(g, r, false, q, pos, k_rot, v, sel_group, lse,
-                                           dout, dq, dk, dv, ws, st);
+                                           dout, dq, dk, dv, ws, q_rot, st);
 }
 
 hga_status backward_error_take(cudaStream_t st, bool clear) {

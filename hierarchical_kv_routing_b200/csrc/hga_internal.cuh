@@ -186,7 +186,7 @@ hga_status launch_attend_backward(const Geo &g, const Rope &r, int dtype, const 
                                   const int32_t *pos, const void *k_rot, const void *v,
                                   const int32_t *sel_group, const float *lse,
                                   const void *dout, float *dq, float *dk, float *dv, void *ws,
-                                  cudaStream_t st);
+                                  const void *q_rot, cudaStream_t st);
 hga_status backward_error_take(cudaStream_t st, bool clear);
 
 // Device error words (bounded-wait timeouts, bounds checks) of each kernel

@@ -203,7 +203,9 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
  * dO . v_j - Delta_i on rows whose weight sits on few keys would magnify its
  * rounding error).
  * Inputs: q (raw), pos, k_rot, v and sel_group as given to hga_attend; lse as
- * hga_attend returned it (required); d_out [B, T, Hq, D] in the dtype of q.  Outputs, fp32: dq [B, T, Hq, D] with respect to the raw
+ * hga_attend returned it (required); d_out [B, T, Hq, D] in the dtype of q;
+ * q_rot (bf16, may be NULL) the rotated queries hga_route wrote for the
+ * forward, which spares the backward rotating q again (same results).  Outputs, fp32: dq [B, T, Hq, D] with respect to the raw
  * q, dk [B, T, Hkv, D] with respect to the RAW k (the rotation undone at each
  * key's position), dv [B, T, Hkv, D]; every element is written.  workspace:
  * hga_workspace_size(HGA_ATTEND_BACKWARD) bytes, 256-byte aligned.  bf16 with
@@ -213,8 +215,9 @@ hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
 hga_status hga_attend_backward(const hga_dims *dims, const hga_params *prm,
                                const void *q, const int32_t *pos, const void *k_rot,
                                const void *v, const int32_t *sel_group, const float *lse,
-                               const void *d_out, float *dq, float *dk, float *dv,
-                               void *workspace, size_t workspace_bytes, void *stream);
+                               const void *d_out, const void *q_rot, float *dq, float *dk,
+                               float *dv, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /* Bytes of device workspace hga_forward (or, for HGA_ATTEND_BACKWARD,
  * hga_attend_backward) needs for `mode` (0 if none).  For HGA_PREFILL this

@@ -170,9 +170,10 @@ def test_backward_full_budget_equals_dense_gradients(gpu_lib):
 
 
 def test_backward_twice_is_stable(gpu_lib):
-    """Two calls in a row on the same inputs: dq is bit-identical (its rows
-    are owned by one CTA each); dk and dv are sums formed by atomic additions
-    and agree to rounding."""
+    """Two calls in a row on the same inputs, and a third given the rotated
+    queries from routing: dq is bit-identical (its rows are owned by one CTA
+    each); dk and dv are sums formed by atomic additions and agree to
+    rounding."""
     w = QWEN.replace(T=1024)
     dev = torch.device("cuda")
     q, k, v, pos, _ = make_prefill_inputs(w, seed=35, device=dev)
@@ -184,10 +185,15 @@ def test_backward_twice_is_stable(gpu_lib):
     out, lse = gpu_lib.hga_attend(q, pos, k_rot, v, sel_g, hp, want_lse=True)
     a = gpu_lib.hga_attend_backward(q, pos, k_rot, v, sel_g, lse, dO, hp)
     b = gpu_lib.hga_attend_backward(q, pos, k_rot, v, sel_g, lse, dO, hp)
+    # with the rotated queries the forward's routing wrote: the same dq bits
+    q_rot = torch.empty_like(q)
+    gpu_lib.hga_route(q, pos, s_c, s_g, hp, q_rot=q_rot)
+    c = gpu_lib.hga_attend_backward(q, pos, k_rot, v, sel_g, lse, dO, hp, q_rot=q_rot)
     torch.cuda.synchronize()
-    assert torch.equal(a[0], b[0])
-    for x, y in zip(a[1:], b[1:]):
+    assert torch.equal(a[0], b[0]) and torch.equal(a[0], c[0])
+    for x, y, z in zip(a[1:], b[1:], c[1:]):
         assert (x - y).abs().max().item() <= 1e-5 * max(1.0, x.abs().max().item())
+        assert (x - z).abs().max().item() <= 1e-5 * max(1.0, x.abs().max().item())
 
 
 @pytest.mark.slow
