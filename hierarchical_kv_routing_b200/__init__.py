@@ -127,6 +127,8 @@ def load():
         lib.hga_hostkv_link_bytes.argtypes = [P, ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         lib.hga_hostkv_link_bytes.restype = ctypes.c_int
         lib.hga_attend_backward.argtypes = [P] * 14 + [ctypes.c_size_t, P]
+        lib.hga_set_test_hooks.argtypes = [ctypes.c_int, ctypes.c_ulonglong, P]
+        lib.hga_set_test_hooks.restype = ctypes.c_int
         lib.hga_hostkv_plan_for.argtypes = [P, P, ctypes.c_size_t, P]
         lib.hga_hostkv_plan_for.restype = ctypes.c_int
         for f in ("hga_build_summaries", "hga_route", "hga_attend", "hga_forward",

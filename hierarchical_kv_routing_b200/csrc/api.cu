@@ -372,6 +372,12 @@ hga_status hga_device_status(void *stream, int clear) {
     return first;
 }
 
+hga_status hga_set_test_hooks(int skip_summaries_copy, unsigned long long summaries_wait_ns,
+                              void *stream) {
+    return summaries_test_hooks(skip_summaries_copy != 0 ? 1 : 0, summaries_wait_ns,
+                                (cudaStream_t)stream);
+}
+
 hga_status hga_hostkv_link_bytes(void *stream, unsigned long long *bytes, int clear) {
     if (!bytes) return HGA_ERR_INVALID_ARG;
     return tier_link_bytes_take((cudaStream_t)stream, bytes, clear != 0);

@@ -424,14 +424,17 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     for (int e = 0; e < 128; ++e)
                         if (gc0 + e >= nvis) v[e] = __float_as_uint(-INFINITY);
                 }
-                // row max with 8 independent chains (no 128-long dependency)
+                // row max with 8 independent chains of three-input maxima
                 float mx8[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(v[u]);
+                for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(__uint_as_float(v[u]), __uint_as_float(v[u + 8]));
 #pragma unroll
-                for (int e = 8; e < 128; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(v[e]));
-                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                for (int e = 16; e < 128; e += 16)
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        mx8[u] = max3f(mx8[u], __uint_as_float(v[e + u]), __uint_as_float(v[e + 8 + u]));
+                float mx = fmaxf(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]));
+                mx = max3f(mx, mx8[6], mx8[7]);
                 if (!valid) mx = -INFINITY;
                 const float mt_new = mx * sc;
                 // The reference grows only when the row max rises by more than
@@ -445,20 +448,26 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
                 const bool live = m_ref != -INFINITY;
                 const float neg = -m_ref;
-                float l8[8];
+                // pairs of columns in packed two-lane fp32: s * scale - m_ref
+                // and the row sum (4 chains of pairs), ex2 per column
+                const uint64_t sc2 = f2_pack(sc, sc), neg2 = f2_pack(neg, neg);
+                uint64_t l4[4];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) l8[u] = 0.f;
+                for (int u = 0; u < 4; ++u) l4[u] = f2_pack(0.f, 0.f);
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     float p0 = 0.f, p1 = 0.f;
                     if (live) {
-                        p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, neg));
-                        p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, neg));
+                        const float2 x = f2_unpack(f2_fma(
+                            f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2));
+                        p0 = ex2(x.x);
+                        p1 = ex2(x.y);
                     }
-                    l8[e & 7] += p0 + p1;
+                    l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
                     v[e] = pack_bf16(p0, p1);
                 }
-                l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+                const float2 la = f2_unpack(f2_add(l4[0], l4[1])), lb = f2_unpack(f2_add(l4[2], l4[3]));
+                l += (la.x + la.y) + (lb.x + lb.y);
                 tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
                 tmem_st32(lane_base + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
                 // tcgen05.ld/st are warp-collective: the warp rescales O

@@ -360,6 +360,212 @@ __device__ void attend_part(const DecodeArgs &A, int b, int h, int t, int nk, Ke
     }
 }
 
+// ---- bf16 slices on warp-level tensor-core tiles (mma.sync m16n8k16) ----
+// A slice is a [G x D] . [D x keys] product: the G <= 16 query heads of a KV
+// head are the 16 rows of an m16 tile (rows >= G are zero).  Rows in shared
+// memory are padded by 16 bytes, so the eight 16-byte rows an ldmatrix reads
+// fall in distinct banks.
+constexpr int kQRows = 16;
+
+__device__ __forceinline__ uint32_t su32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(su32(p))
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm4_t(uint32_t (&r)[4], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(su32(p))
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm2_t(uint32_t (&r)[2], const void *p) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(su32(p))
+                 : "memory");
+}
+// d (16x8 f32) += a (16x16 bf16, row major) . b (16x8 bf16, column major)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
+__host__ __device__ constexpr int tc_row() { return D + 8; }                                // K, V and Q rows
+template <int D>
+__host__ __device__ constexpr int tc_prow() { return (32 * 1024) / (D * 2) + 8; }  // P rows
+template <int D>
+__host__ __device__ constexpr size_t tc_tile_bytes() {                                      // Q and P tiles
+    return sizeof(__nv_bfloat16) * kQRows * (size_t)(tc_row<D>() + tc_prow<D>());
+}
+template <int D>
+__host__ __device__ constexpr size_t tc_dyn_bytes() {                   // K and V rows
+    return 2 * sizeof(__nv_bfloat16) * (size_t)(tc_prow<D>() - 8) * tc_row<D>();
+}
+
+// Rotated queries of the KV head's G heads, scaled by log2(e)/sqrt(D) and
+// rounded to bf16, as the 16-row A tile Qb (rows >= G zero).
+template <int D>
+__device__ __forceinline__ void load_queries_tc(const DecodeArgs &A, int b, int h, int32_t pnew,
+                                                __nv_bfloat16 *Qb) {
+    constexpr int H = D / 2, RE = tc_row<D>();
+    const __nv_bfloat16 *qb =
+        static_cast<const __nv_bfloat16 *>(A.q_new) + ((int64_t)b * A.Hq + (int64_t)h * A.G) * D;
+    for (int e = threadIdx.x; e < kQRows * H; e += blockDim.x) {
+        const int g = e / H, i = e % H;
+        float o0 = 0.f, o1 = 0.f;
+        if (g < A.G) {
+            const float2 r = rope_cs_int(A.rope, pnew, i);
+            const float x = to_f(qb[g * D + i]), y = to_f(qb[g * D + i + H]);
+            o0 = (x * r.x - y * r.y) * A.scale_log2;
+            o1 = (y * r.x + x * r.y) * A.scale_log2;
+        }
+        Qb[g * RE + i] = __float2bfloat16_rn(o0);
+        Qb[g * RE + i + H] = __float2bfloat16_rn(o1);
+    }
+}
+
+// attend_part for bf16 on tensor-core tiles.  Same inputs and partial
+// (m, l, o[D]) output; P is rounded to bf16 for P.V and l sums the rounded
+// weights, so the weights of a row sum to exactly l.
+template <int D, typename KeyOf>
+__device__ void attend_part_tc(const DecodeArgs &A, int b, int h, int t, int nk, KeyOf key_of,
+                               int pi, const __nv_bfloat16 *Qb, const __nv_bfloat16 *knew,
+                               float *sc, int *kt_s, __nv_bfloat16 *Pb, __nv_bfloat16 *Ks,
+                               __nv_bfloat16 *Vs) {
+    using bf = __nv_bfloat16;
+    constexpr int RE = tc_row<D>(), PE = tc_prow<D>();
+    constexpr int NV = D / 8;                           // 16-byte chunks per row
+    static_assert(D % 32 == 0 && kThreads == 256, "8 warps, two k-steps per ldmatrix");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nk16 = (nk + 15) & ~15;
+    for (int k = threadIdx.x; k < nk; k += blockDim.x) kt_s[k] = key_of(k);
+    __syncthreads();
+    const bf *kbase = static_cast<const bf *>(A.k_rot);
+    const bf *vbase = static_cast<const bf *>(A.v);
+    const bf *vn = static_cast<const bf *>(A.v_new) + ((int64_t)b * A.Hkv + h) * D;
+    for (int idx = threadIdx.x; idx < nk16 * NV; idx += blockDim.x) {
+        const int k = idx / NV, pv = idx % NV;
+        uint4 *kd = reinterpret_cast<uint4 *>(Ks + (size_t)k * RE) + pv;
+        uint4 *vd = reinterpret_cast<uint4 *>(Vs + (size_t)k * RE) + pv;
+        if (k >= nk) {                                  // pad rows: P.V must see zeros
+            *kd = make_uint4(0u, 0u, 0u, 0u);
+            *vd = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+        }
+        const int kv = kt_s[k];
+        const int64_t row = (((int64_t)b * A.Tc + kv) * A.Hkv + h) * D;
+        if (kv == t) *kd = reinterpret_cast<const uint4 *>(knew)[pv];
+        else cp_async16(kd, reinterpret_cast<const uint4 *>(kbase + row) + pv);
+        cp_async16(vd, reinterpret_cast<const uint4 *>(kv == t ? vn : vbase + row) + pv);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
+    const int g_lo = lane >> 2, c2 = (lane & 3) * 2;
+    // S = Q K^T: 8-key column tiles over the warps, the Q fragments held
+    {
+        uint32_t qa[D / 16][4];
+        const int r = (lane & 7) + ((lane >> 3) & 1) * 8, cc = (lane >> 4) * 8;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) ldsm4(qa[kk], Qb + r * RE + kk * 16 + cc);
+        for (int nt = warp; nt < nk16 / 8; nt += nw) {
+            const int n0 = nt * 8;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk += 2) {
+                uint32_t kb[4];
+                ldsm4(kb, Ks + (size_t)(n0 + (lane & 7)) * RE + kk * 16 + (lane >> 3) * 8);
+                mma16816(acc, qa[kk], kb[0], kb[1]);
+                mma16816(acc, qa[kk + 1], kb[2], kb[3]);
+            }
+            const int key = n0 + c2;
+            if (g_lo < A.G) {
+                if (key < nk) sc[g_lo * kThreads + key] = acc[0];
+                if (key + 1 < nk) sc[g_lo * kThreads + key + 1] = acc[1];
+            }
+            if (g_lo + 8 < A.G) {
+                if (key < nk) sc[(g_lo + 8) * kThreads + key] = acc[2];
+                if (key + 1 < nk) sc[(g_lo + 8) * kThreads + key + 1] = acc[3];
+            }
+        }
+    }
+    __syncthreads();
+    // softmax per head (base 2, scores pre-scaled): P as bf16 into the A tile
+    float *part_b = A.part + ((int64_t)b * A.Hq + (int64_t)h * A.G) * A.nparts * (D + 2);
+    for (int g = warp; g < kQRows; g += nw) {
+        if (g >= A.G) {
+            for (int k = lane; k < nk16; k += 32) Pb[g * PE + k] = __float2bfloat16_rn(0.f);
+            continue;
+        }
+        float m = -INFINITY;
+        for (int k = lane; k < nk; k += 32) m = fmaxf(m, sc[g * kThreads + k]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        for (int k = lane; k < nk16; k += 32) {
+            const bf p = __float2bfloat16_rn(k < nk ? exp2f(sc[g * kThreads + k] - m) : 0.f);
+            Pb[g * PE + k] = p;
+            l += __bfloat162float(p);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+            float *dst = part_b + ((int64_t)g * A.nparts + pi) * (D + 2);
+            dst[0] = nk > 0 ? m : -INFINITY;
+            dst[1] = l;
+        }
+    }
+    __syncthreads();
+    // O = P V: warp w owns output dims [w D/8, (w + 1) D/8)
+    {
+        constexpr int NT = D / 64;                      // 8-dim column tiles per warp
+        const int d0 = warp * (D / 8);
+        float o[NT][4];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        const int pr = (lane & 7) + ((lane >> 3) & 1) * 8, pc = (lane >> 4) * 8;
+        const int vr = (lane & 7) + ((lane >> 3) & 1) * 8;
+        for (int k0 = 0; k0 < nk16; k0 += 16) {
+            uint32_t pa[4];
+            ldsm4(pa, Pb + pr * PE + k0 + pc);
+            if constexpr (NT == 2) {
+                uint32_t vb[4];
+                ldsm4_t(vb, Vs + (size_t)(k0 + vr) * RE + d0 + (lane >> 4) * 8);
+                mma16816(o[0], pa, vb[0], vb[1]);
+                mma16816(o[1], pa, vb[2], vb[3]);
+            } else {
+                uint32_t vb[2];
+                ldsm2_t(vb, Vs + (size_t)(k0 + vr) * RE + d0);
+                mma16816(o[0], pa, vb[0], vb[1]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int d = d0 + 8 * j + c2;
+            if (g_lo < A.G) {
+                float *dst = part_b + ((int64_t)g_lo * A.nparts + pi) * (D + 2) + 2;
+                dst[d] = o[j][0];
+                dst[d + 1] = o[j][1];
+            }
+            if (g_lo + 8 < A.G) {
+                float *dst = part_b + ((int64_t)(g_lo + 8) * A.nparts + pi) * (D + 2) + 2;
+                dst[d] = o[j][2];
+                dst[d + 1] = o[j][3];
+            }
+        }
+    }
+}
+
 // Every slice CTA (fixed or routed) ends here: the last of the nparts
 // slices of (b, h) to finish combines all partial softmax sums into the
 // output, and the last (b, h) of a sequence increments its lens.
@@ -419,14 +625,20 @@ __device__ void finish_slice(const DecodeArgs &A, int b, int h, int t, int *s_la
 // Runs beside k_decode_a on a second stream: it needs no routing.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A) {
-    __shared__ __align__(16) float qs[kMaxG * D];
+    constexpr bool kTc = sizeof(T) == 2;                              // bf16: tensor-core tiles
+    __shared__ __align__(16) float qs[kTc ? 4 : kMaxG * D];
+    __shared__ __align__(16) unsigned char tct[kTc ? tc_tile_bytes<D>() : 16];
     __shared__ __align__(16) T knew[D];
     __shared__ float sc[kMaxG * kThreads];
     __shared__ int kt_s[kThreads];
     __shared__ int s_last;
     extern __shared__ __align__(16) unsigned char dyn[];
-    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][D]
-    T *Vs = Ks + (size_t)slice_keys<T, D>() * D;                      // [slice_keys][D]
+    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][row]
+    constexpr int kSK = (32 * 1024) / (D * (int)sizeof(T)) < kThreads ? (32 * 1024) / (D * (int)sizeof(T)) : kThreads;
+    constexpr int kRow = kTc ? tc_row<D>() : D;
+    T *Vs = Ks + (size_t)kSK * kRow;
+    __nv_bfloat16 *Qb = reinterpret_cast<__nv_bfloat16 *>(tct);
+    __nv_bfloat16 *Pb = Qb + kQRows * tc_row<D>();
     const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];
     if (t < 0 || t >= A.Tc) {
@@ -441,14 +653,18 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_fixed(const DecodeArgs A
     const int nfix = n2 + (t - c * A.C + 1);
     const int per = (nfix + A.nF - 1) / A.nF;
     const int k0 = min(nfix, f * per), nk = min(nfix, k0 + per) - k0;
-    load_queries<T, D>(A, b, h, pnew, qs);
+    if constexpr (kTc) load_queries_tc<D>(A, b, h, pnew, Qb);
+    else load_queries<T, D>(A, b, h, pnew, qs);
     rotate_new_key<T, D>(A, b, h, pnew, knew);
     __syncthreads();
     auto key_of = [&](int k) {
         const int i = k0 + k;
         return i < n1 ? i : (i < n2 ? rec_lo * A.C + (i - n1) : c * A.C + (i - n2));
     };
-    attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Ks, Vs);
+    if constexpr (kTc)
+        attend_part_tc<D>(A, b, h, t, nk, key_of, f, Qb, knew, sc, kt_s, Pb, Ks, Vs);
+    else
+        attend_part<T, D>(A, b, h, t, nk, key_of, f, qs, knew, sc, kt_s, Ks, Vs);
     finish_slice<T, D>(A, b, h, t, &s_last);
 }
 
@@ -582,20 +798,29 @@ __global__ void __launch_bounds__(kThreads, 4) k_decode_a(const DecodeArgs A) {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
-    __shared__ __align__(16) float qs[kMaxG * D];
+    constexpr bool kTc = sizeof(T) == 2;                              // bf16: tensor-core tiles
+    __shared__ __align__(16) float qs[kTc ? 4 : kMaxG * D];
+    __shared__ __align__(16) unsigned char tct[kTc ? tc_tile_bytes<D>() : 16];
     __shared__ __align__(16) T knew[D];
     __shared__ float sc[kMaxG * kThreads];
     __shared__ int kt_s[kThreads];
     __shared__ int sel[kMaxK];
     __shared__ int s_last;
     extern __shared__ __align__(16) unsigned char dyn[];
-    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][D]
-    T *Vs = Ks + (size_t)slice_keys<T, D>() * D;                      // [slice_keys][D]
+    T *Ks = reinterpret_cast<T *>(dyn);                               // [slice_keys][row]
+    constexpr int kSK = (32 * 1024) / (D * (int)sizeof(T)) < kThreads ? (32 * 1024) / (D * (int)sizeof(T)) : kThreads;
+    constexpr int kRow = kTc ? tc_row<D>() : D;
+    T *Vs = Ks + (size_t)kSK * kRow;
+    __nv_bfloat16 *Qb = reinterpret_cast<__nv_bfloat16 *>(tct);
+    __nv_bfloat16 *Pb = Qb + kQRows * tc_row<D>();
 
     const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t = A.lens[b];          // written only by the previous step
     const int32_t pnew = A.pos_new[b];
-    if (t >= 0 && t < A.Tc) load_queries<T, D>(A, b, h, pnew, qs);
+    if (t >= 0 && t < A.Tc) {
+        if constexpr (kTc) load_queries_tc<D>(A, b, h, pnew, Qb);
+        else load_queries<T, D>(A, b, h, pnew, qs);
+    }
     // everything below reads what k_decode_a wrote
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (t < 0 || t >= A.Tc) return;
@@ -611,7 +836,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_decode_b(const DecodeArgs A) {
         const int i = k0 + k;
         return sel[i / A.g_s] * A.g_s + i % A.g_s;
     };
-    attend_part<T, D>(A, b, h, t, nk, key_of, A.nF + r, qs, knew, sc, kt_s, Ks, Vs);
+    if constexpr (kTc)
+        attend_part_tc<D>(A, b, h, t, nk, key_of, A.nF + r, Qb, knew, sc, kt_s, Pb, Ks, Vs);
+    else
+        attend_part<T, D>(A, b, h, t, nk, key_of, A.nF + r, qs, knew, sc, kt_s, Ks, Vs);
 
     finish_slice<T, D>(A, b, h, t, &s_last);
 }
@@ -739,7 +967,8 @@ hga_status run(const Geo &g, const Rope &r, const hga_io &io, void *ws, cudaStre
     A.nF = sl.nF;
     A.nR = sl.nR;
     A.nparts = sl.nF + sl.nR;
-    const size_t vs_bytes = 2 * sizeof(T) * (size_t)slice_keys<T, D>() * D;
+    const size_t vs_bytes = sizeof(T) == 2 ? tc_dyn_bytes<D>()
+                                           : 2 * sizeof(T) * (size_t)slice_keys<T, D>() * D;
     cudaError_t e = ensure_smem((const void *)k_decode_fixed<T, D>, vs_bytes);
     if (e == cudaSuccess) e = ensure_smem((const void *)k_decode_b<T, D>, vs_bytes);
     if (e != cudaSuccess) return cuda_status(e);

@@ -194,6 +194,7 @@ hga_status backward_error_take(cudaStream_t st, bool clear);
 hga_status attend_tc_error_take(cudaStream_t st, bool clear);
 hga_status decode_error_take(cudaStream_t st, bool clear);
 hga_status summaries_error_take(cudaStream_t st, bool clear);
+hga_status summaries_test_hooks(int skip_copy, unsigned long long wait_ns, cudaStream_t st);
 hga_status tier_error_take(cudaStream_t st, bool clear);
 hga_status tier_link_bytes_take(cudaStream_t st, unsigned long long *bytes, bool clear);
 

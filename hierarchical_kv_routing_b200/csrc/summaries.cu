@@ -21,6 +21,10 @@
 namespace hga {
 
 __device__ int g_summaries_error = 0;
+// Test hooks (hga_set_test_hooks): skip the keys' bulk copy, so the wait for
+// it runs out, and the limit of that wait.
+__device__ int g_summaries_skip_copy = 0;
+__device__ unsigned long long g_summaries_wait_ns = sm100::kMaxWaitNs;
 
 namespace {
 
@@ -106,7 +110,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
         if constexpr (!kHost) {
             if (threadIdx.x == 0) {
                 mbar_arrive_expect_tx(&bar, row_bytes * n);
-                if (nh == A.Hkv) {
+                if (g_summaries_skip_copy) {
+                    // test hook: the copy is not issued and the wait below runs out
+                } else if (nh == A.Hkv) {
                     bulk_load(kb, src0, row_bytes * n, &bar);       // contiguous rows
                 } else {
                     for (int j = 0; j < n; ++j)
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
         }
         __syncthreads();
         if constexpr (!kHost) {
-            if (!mbar_wait(&bar, pass & 1)) {
+            if (!mbar_wait(&bar, pass & 1, g_summaries_wait_ns)) {
                 if (threadIdx.x == 0) atomicExch(&g_summaries_error, (int)HGA_ERR_TIMEOUT);
                 return;
             }
@@ -319,6 +325,17 @@ hga_status launch_summaries(const Geo &g, const Rope &r, int dtype, const void *
 
 // Reads this file's device error word on `st` (after the work queued on it)
 // and optionally resets it; returns the recorded status (HGA_OK if none).
+hga_status summaries_test_hooks(int skip_copy, unsigned long long wait_ns, cudaStream_t st) {
+    const unsigned long long ns = wait_ns ? wait_ns : sm100::kMaxWaitNs;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_summaries_skip_copy, &skip_copy, sizeof(int), 0,
+                                            cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(g_summaries_wait_ns, &ns, sizeof(ns), 0,
+                                    cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
+}
+
 hga_status summaries_error_take(cudaStream_t st, bool clear) {
     int v = 0;
     cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_summaries_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);

@@ -359,6 +359,18 @@ hga_status hga_device_status(void *stream, int clear);
  * count.  *bytes must be a host pointer (HGA_ERR_INVALID_ARG if NULL). */
 hga_status hga_hostkv_link_bytes(void *stream, unsigned long long *bytes, int clear);
 
+/* Test hook, not for production use: exercises the bounded-wait timeout
+ * path of a real kernel without a GPU fault.  With skip_summaries_copy != 0
+ * the summaries kernel (stage 1, device-memory keys) does not issue the bulk
+ * copy of its keys, so its wait for them runs out after summaries_wait_ns
+ * (0 = the default limit of 2 s); the kernel then records HGA_ERR_TIMEOUT
+ * (read by hga_device_status) and returns with nothing in flight, and its
+ * outputs are left unwritten.  hga_set_test_hooks(0, 0, stream) restores
+ * normal operation.  The settings are per device and apply to every call
+ * that follows; the call waits for `stream`. */
+hga_status hga_set_test_hooks(int skip_summaries_copy, unsigned long long summaries_wait_ns,
+                              void *stream);
+
 /* Static description of a status code. */
 const char *hga_status_string(hga_status s);
 
