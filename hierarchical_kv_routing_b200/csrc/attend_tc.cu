@@ -40,22 +40,32 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
-constexpr uint32_t kRegsLaunch = 168;   // 65536 / 384, rounded down to 8
-constexpr uint32_t kRegsCtl = 56;       // warps 0-3: TMA producers, MMA issuer
-constexpr uint32_t kRegsSoftmax = 224;  // warps 4-11: softmax and epilogue
+// Two shapes of CTA.  The general one: 384 threads, two 128-row M-tiles,
+// one CTA per SM (all 512 TMEM columns).  kOne (units of at most 128 query
+// rows, i.e. Hq/Hkv <= 2): 256 threads, one M-tile, 256 TMEM columns and a
+// 2-stage ring, so two CTAs share an SM and one's softmax, set-up and
+// epilogue overlap the other's products.
+template <bool kOne> struct Shape {
+    static constexpr int kThreads = kOne ? 256 : 384;
+    static constexpr uint32_t kRegsLaunch = kOne ? 128 : 168;   // 65536 / (threads x CTAs per SM)
+    static constexpr uint32_t kRegsCtl = 56;                    // warps 0-3: TMA producers, MMA issuer
+    static constexpr uint32_t kRegsSoftmax = kOne ? 200 : 224;  // softmax and epilogue warps
+    static constexpr uint32_t kTmemCols = kOne ? 256 : 512;
+    static_assert(128 * kRegsCtl + (kThreads - 128) * kRegsSoftmax <= kThreads * kRegsLaunch,
+                  "register split");
+};
 constexpr int kMaxSeg = 2048;
 constexpr int kSegPerTile = 16;          // 16 x 8 tokens = 128 keys
 constexpr int kDummy = 0x7fffffff;       // padding segment
 
-template <int D>
+template <int D, bool kOne = false>
 struct Cfg {
     static constexpr int kHalves = D / 64;
-    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kStages = (D == 128 || kOne) ? 2 : 4;
     static constexpr uint32_t kHalfBytes = 128 * 128;          // 128 rows x 128 B
     static constexpr uint32_t kTileBytes = kHalves * kHalfBytes;
     static constexpr uint32_t oQ = 0;
-    static constexpr uint32_t oK = oQ + 2 * kTileBytes;
+    static constexpr uint32_t oK = oQ + (kOne ? 1 : 2) * kTileBytes;
     static constexpr uint32_t oV = oK + kStages * kTileBytes;
     static constexpr uint32_t oEnd = oV + kStages * kTileBytes;
     static constexpr uint32_t oCS = oEnd;                       // optional cos/sin table
@@ -67,6 +77,7 @@ struct Ctl {
     uint64_t fin;
     uint32_t tmem_base;
     int nseg, first_cur;
+    int early;                // tile 0 was issued during set-up
     volatile int abort;
     int s_pos[kChunk];        // positions of this CTA's query tokens
     int seg_tok[kMaxSeg];
@@ -97,6 +108,33 @@ __device__ __forceinline__ void fail(Ctl &ctl) {
     atomicExch(&g_attend_tc_error, (int)HGA_ERR_TIMEOUT);
 }
 
+// Loads nsj segments (8 key rows each, rows sg[e] of sequence b's token
+// layout) of one tensor into a 128B-swizzled tile whose D-halves are
+// half_bytes apart; runs of 8 or 2 consecutive segments go as one 64- or
+// 16-row box.
+template <int kHalves>
+__device__ __forceinline__ void load_tile(uint8_t *tile, uint32_t half_bytes, const int *sg,
+                                          int nsj, const CUtensorMap *m8, const CUtensorMap *m16,
+                                          const CUtensorMap *m64, uint64_t *full, int h, int zb) {
+    for (int e = 0; e < nsj;) {
+        const int st = sg[e];
+        int run = 1;
+        if (st != kDummy) {
+            if ((e & 7) == 0 && e + 8 <= nsj) {
+                run = 8;
+                for (int i = 1; i < 8; ++i)
+                    if (sg[e + i] != st + 8 * i) { run = 1; break; }
+            }
+            if (run == 1 && (e & 1) == 0 && e + 2 <= nsj && sg[e + 1] == st + 8) run = 2;
+        }
+        const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
+        const int z = zb + (st == kDummy ? 0 : st);
+        for (int hf = 0; hf < kHalves; ++hf)
+            tma_load_3d(tile + hf * half_bytes + e * 1024, m, full, hf * 64, h, z);
+        e += run;
+    }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -105,13 +143,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // kTier: keys come from the host tier's buffers and group cache (TcArgs tier
 // fields) instead of the token layout; a separate instantiation, so the
 // in-HBM prefill's code is not touched by it.
-template <int D, bool kTier>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool kTier, bool kOne>
+__global__ void __launch_bounds__(Shape<kOne>::kThreads, kOne ? 2 : 1)
 k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
             const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmK64,
             const __grid_constant__ CUtensorMap tmV64, const TcArgs A) {
-    using C = Cfg<D>;
+    using C = Cfg<D, kOne>;
+    using SH = Shape<kOne>;
+    constexpr int kThreads = SH::kThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -153,9 +193,33 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 tma_load_3d(smem + C::oQ + mt * C::kTileBytes + hf * C::kHalfBytes, &tmQ,
                             &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first);
         }
+        // The first key tile, when the fixed windows fill it, depends on no
+        // routed id: its K and V start loading now, before the segment list
+        // is built (its 16 segments are the list's first 16, the same rule).
+        const int nsink = min(A.F, c);
+        const int rec_lo = max(c - max(A.L, 1), nsink);
+        ctl.early = 8 * (nsink + (c - rec_lo)) >= kSegPerTile;
+        if (ctl.early) {
+            int sg[kSegPerTile];
+            for (int e = 0; e < kSegPerTile; ++e) {
+                const int tok = e < 8 * nsink ? e * 8 : rec_lo * kChunk + (e - 8 * nsink) * 8;
+                if constexpr (kTier)
+                    sg[e] = A.buf_row0 + (tok < A.sink_rows ? tok : A.win_row0 + tok - A.win_tok0);
+                else
+                    sg[e] = tok;
+            }
+            prefetch_tensormap(&tmK64);
+            prefetch_tensormap(&tmV64);
+            mbar_arrive_expect_tx(&ctl.k_full[0], (uint32_t)kSegPerTile * 8 * D * 2);
+            load_tile<C::kHalves>(smem + C::oK, C::kHalfBytes, sg, kSegPerTile, &tmK, &tmK16,
+                                  &tmK64, &ctl.k_full[0], h, b * A.k_T);
+            mbar_arrive_expect_tx(&ctl.v_full[0], (uint32_t)kSegPerTile * 8 * D * 2);
+            load_tile<C::kHalves>(smem + C::oV, C::kHalfBytes, sg, kSegPerTile, &tmV, &tmV16,
+                                  &tmV64, &ctl.v_full[0], h, b * A.v_T);
+        }
     }
     if (warp == 1) {
-        tmem_alloc(&ctl.tmem_base, 512);
+        tmem_alloc(&ctl.tmem_base, SH::kTmemCols);
         tc_fence_before();
     }
     if (warp == 3 && !A.prerot) {
@@ -211,14 +275,14 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     // Registers: the producer / MMA warpgroup needs few, the two softmax
     // warpgroups hold a 128-column S row each.  128 x 56 + 256 x 224 equals
     // the launch allocation of 384 x 168.
-    static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+
     const uint32_t tmem = ctl.tmem_base;
     const int nseg = ctl.nseg;
     const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
     const int first_cur = ctl.first_cur;
 
     if (warp < 4) {
-    regs_dec<kRegsCtl>();
+    regs_dec<SH::kRegsCtl>();
     if (warp == 0 || warp == 2) {
         // ------------------------------------------------------ producers --
         // warp 0 streams the K tiles, warp 2 the V tiles, each through its own
@@ -242,28 +306,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     fail(ctl);
                     break;
                 }
+                if (j == 0 && ctl.early) continue;      // tile 0 is already loading
                 const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
                 uint8_t *tile = smem + (is_k ? C::oK : C::oV) + s * C::kTileBytes;
                 mbar_arrive_expect_tx(full, (uint32_t)nsj * 8 * D * 2);
-                // runs of consecutive segments go as one 64- or 16-row box
-                const int *sg = ctl.seg_tok + j * kSegPerTile;
-                for (int e = 0; e < nsj;) {
-                    const int st = sg[e];
-                    int run = 1;
-                    if (st != kDummy) {
-                        if ((e & 7) == 0 && e + 8 <= nsj) {
-                            run = 8;
-                            for (int i = 1; i < 8; ++i)
-                                if (sg[e + i] != st + 8 * i) { run = 1; break; }
-                        }
-                        if (run == 1 && (e & 1) == 0 && e + 2 <= nsj && sg[e + 1] == st + 8) run = 2;
-                    }
-                    const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
-                    const int z = b * kvT + (st == kDummy ? 0 : st);
-                    for (int hf = 0; hf < C::kHalves; ++hf)
-                        tma_load_3d(tile + hf * C::kHalfBytes + e * 1024, m, full, hf * 64, h, z);
-                    e += run;
-                }
+                load_tile<C::kHalves>(tile, C::kHalfBytes, ctl.seg_tok + j * kSegPerTile, nsj, m8,
+                                      m16, m64, full, h, b * kvT);
             }
         }
     } else if (warp == 1) {
@@ -333,7 +381,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         }
     }
     } else {
-        regs_inc<kRegsSoftmax>();
+        regs_inc<SH::kRegsSoftmax>();
         // ------------------------------------------------------- softmax --
         // cos/sin of every (token, pair) of this CTA's rows, shared by the G
         // query heads of a token (each angle formed once instead of G times);
@@ -527,7 +575,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, SH::kTmemCols);
     }
 }
 
@@ -594,6 +642,8 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         const size_t tab = (size_t)tok_cta * (D / 2 + 1) * sizeof(float2);
         a.cs_tokens = !a.prerot && Cfg<D>::oEnd + 1024 + tab + sizeof(Ctl) <= 232448 ? tok_cta : 0;
     }
+    // units of at most 128 rows take the one-M-tile CTA (two per SM)
+    const bool one = a.rows_per_unit <= 128;
     a.sel_group = sel_group;
     a.pos = pos;
     a.out = static_cast<__nv_bfloat16 *>(out);
@@ -609,12 +659,15 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         !make_map(&mk64, k_rot, D, g.Hkv, (long long)g.B * k_T, 1, 64) ||
         !make_map(&mv64, v, D, g.Hkv, (long long)g.B * v_T, 1, 64))
         return HGA_ERR_CUDA;
-    const size_t smem = Cfg<D>::oEnd + 1024 + (size_t)a.cs_tokens * (D / 2 + 1) * sizeof(float2);
-    auto kern = tw ? k_attend_tc<D, true> : k_attend_tc<D, false>;
+    const size_t smem = (one ? Cfg<D, true>::oEnd : Cfg<D>::oEnd) + 1024 +
+                        (size_t)a.cs_tokens * (D / 2 + 1) * sizeof(float2);
+    auto kern = tw ? (one ? k_attend_tc<D, true, true> : k_attend_tc<D, true, false>)
+                   : (one ? k_attend_tc<D, false, true> : k_attend_tc<D, false, false>);
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(nblk * a.ctas_per_unit, g.Hkv, g.B);
-    kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mk16, mv16, mk64, mv64, a);
+    kern<<<grid, one ? Shape<true>::kThreads : Shape<false>::kThreads, smem, st>>>(
+        mq, mk, mv, mk16, mv16, mk64, mv64, a);
     return cuda_status(cudaGetLastError());
 }
 

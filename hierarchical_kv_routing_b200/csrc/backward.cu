@@ -324,7 +324,7 @@ __device__ __forceinline__ void build_segments(BwdCtl &ctl, const BwdArgs &A, in
 __device__ __forceinline__ void load_segments(uint8_t *tile, uint32_t half_bytes, int halves,
                                               const int *sg, int nsj, const CUtensorMap *m8,
                                               const CUtensorMap *m16, const CUtensorMap *m64,
-                                              uint64_t *bar, int h, int zbase) {
+                                              uint64_t *bar, int h, int zbase, uint64_t policy) {
     for (int e = 0; e < nsj;) {
         const int st = sg[e];
         int run = 1;
@@ -339,7 +339,7 @@ __device__ __forceinline__ void load_segments(uint8_t *tile, uint32_t half_bytes
         const CUtensorMap *m = run == 8 ? m64 : (run == 2 ? m16 : m8);
         const int z = zbase + (st == kDummy ? 0 : st);
         for (int hf = 0; hf < halves; ++hf)
-            tma_load_3d(tile + hf * half_bytes + e * 1024, m, bar, hf * 64, h, z);
+            tma_load_3d_hint(tile + hf * half_bytes + e * 1024, m, bar, hf * 64, h, z, policy);
         e += run;
     }
 }
@@ -402,14 +402,17 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
         fence_barrier_init();
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmG);
+        // this CTA's query rows are read once: they should not push the
+        // gathered K and V (read twice by every unit that sees them) out of L2
+        const uint64_t once = l2_policy_evict_first();
         for (int mt = 0; mt < NT; ++mt) {
             const int tok_first = t0 + (row0 + mt * 128) / A.G;
             mbar_arrive_expect_tx(&ctl.q_full[mt], (uint32_t)(2 * A.G * A.tokM * D * 2));
             for (int hf = 0; hf < C::kHalves; ++hf) {
-                tma_load_3d(smem + C::oQ + mt * C::kQTile + hf * C::kQHalf, &tmQ, &ctl.q_full[mt],
-                            hf * 64, h * A.G, b * A.T + tok_first);
-                tma_load_3d(smem + C::oG + mt * C::kQTile + hf * C::kQHalf, &tmG, &ctl.q_full[mt],
-                            hf * 64, h * A.G, b * A.T + tok_first);
+                tma_load_3d_hint(smem + C::oQ + mt * C::kQTile + hf * C::kQHalf, &tmQ,
+                                 &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first, once);
+                tma_load_3d_hint(smem + C::oG + mt * C::kQTile + hf * C::kQHalf, &tmG,
+                                 &ctl.q_full[mt], hf * 64, h * A.G, b * A.T + tok_first, once);
             }
         }
     }
@@ -437,6 +440,7 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
             prefetch_tensormap(&tmK64);
             prefetch_tensormap(&tmV64);
             // every tile twice: the Delta pass, then the dS / dQ pass
+            const uint64_t keep = l2_policy_evict_last();
             for (int t = 0; t < 2 * ntiles && !ctl.abort; ++t) {
                 const int j = t % ntiles, s = t % C::kStages;
                 if (t >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((t / C::kStages) - 1) & 1)) {
@@ -447,9 +451,9 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 mbar_arrive_expect_tx(&ctl.kv_full[s], (uint32_t)(2 * nsj * 8 * D * 2));
                 const int *sg = ctl.seg_tok + j * C::kSegPerTile;
                 load_segments(smem + C::oK + s * C::kKTile, C::kKHalf, C::kHalves, sg, nsj, &tmK,
-                              &tmK16, &tmK64, &ctl.kv_full[s], h, b * A.T);
+                              &tmK16, &tmK64, &ctl.kv_full[s], h, b * A.T, keep);
                 load_segments(smem + C::oV + s * C::kKTile, C::kKHalf, C::kHalves, sg, nsj, &tmV,
-                              &tmV16, &tmV64, &ctl.kv_full[s], h, b * A.T);
+                              &tmV16, &tmV64, &ctl.kv_full[s], h, b * A.T, keep);
             }
         } else if (warp == 1 && lane == 0) {
             // ---- MMA issuer
@@ -607,10 +611,10 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                                 a[u] = o.x;
                                 bb[u] = o.y;
                             }
-                            reinterpret_cast<float4 *>(dqrow + cb * 32)[e4] =
-                                make_float4(a[0], a[1], a[2], a[3]);
-                            reinterpret_cast<float4 *>(dqrow + H + cb * 32)[e4] =
-                                make_float4(bb[0], bb[1], bb[2], bb[3]);
+                            __stcs(reinterpret_cast<float4 *>(dqrow + cb * 32) + e4,
+                                   make_float4(a[0], a[1], a[2], a[3]));
+                            __stcs(reinterpret_cast<float4 *>(dqrow + H + cb * 32) + e4,
+                                   make_float4(bb[0], bb[1], bb[2], bb[3]));
                         }
                     }
                 }
@@ -719,6 +723,7 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             prefetch_tensormap(&tmV16);
             prefetch_tensormap(&tmK64);
             prefetch_tensormap(&tmV64);
+            const uint64_t keep = l2_policy_evict_last();   // other units read these keys too
             for (int j = 0; j < ntiles && !ctl.abort; ++j) {
                 if (j > 0 && !mbar_wait(&ctl.kv_empty[0], (j - 1) & 1)) {
                     bwd_fail(ctl);
@@ -728,14 +733,16 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 mbar_arrive_expect_tx(&ctl.kv_full[0], (uint32_t)(2 * nsj * 8 * D * 2));
                 const int *sg = ctl.seg_tok + j * C::kSegPerTile;
                 load_segments(smem + C::oK, C::kKHalf, C::kHalves, sg, nsj, &tmK, &tmK16, &tmK64,
-                              &ctl.kv_full[0], h, b * A.T);
+                              &ctl.kv_full[0], h, b * A.T, keep);
                 load_segments(smem + C::oV, C::kKHalf, C::kHalves, sg, nsj, &tmV, &tmV16, &tmV64,
-                              &ctl.kv_full[0], h, b * A.T);
+                              &ctl.kv_full[0], h, b * A.T, keep);
             }
         } else if (warp == 2 && lane == 0) {
             // ---- producer: q~ and dO row subtiles of 64 rows, re-streamed per key tile
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmG);
+            // the unit's query rows are re-read once per key tile
+            const uint64_t keep = l2_policy_evict_last();
             for (int n = 0; n < nsteps && !ctl.abort; ++n) {
                 const int s = n % C::kRowStages;
                 if (n >= C::kRowStages &&
@@ -747,10 +754,10 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 const int tok_first = t0 + i * A.tokS;
                 mbar_arrive_expect_tx(&ctl.row_full[s], (uint32_t)(2 * A.G * A.tokS * D * 2));
                 for (int hf = 0; hf < C::kHalves; ++hf) {
-                    tma_load_3d(smem + C::oQ + s * C::kRTile + hf * C::kRHalf, &tmQ,
-                                &ctl.row_full[s], hf * 64, h * A.G, b * A.T + tok_first);
-                    tma_load_3d(smem + C::oG + s * C::kRTile + hf * C::kRHalf, &tmG,
-                                &ctl.row_full[s], hf * 64, h * A.G, b * A.T + tok_first);
+                    tma_load_3d_hint(smem + C::oQ + s * C::kRTile + hf * C::kRHalf, &tmQ,
+                                     &ctl.row_full[s], hf * 64, h * A.G, b * A.T + tok_first, keep);
+                    tma_load_3d_hint(smem + C::oG + s * C::kRTile + hf * C::kRHalf, &tmG,
+                                     &ctl.row_full[s], hf * 64, h * A.G, b * A.T + tok_first, keep);
                 }
             }
         } else if (warp == 1 && lane == 0) {
