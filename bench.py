@@ -894,7 +894,7 @@ def main():
     d2h = houts[0].numel() * houts[0].element_size()
 
     bwd = None
-    if not (args.no_backward or args.seq):
+    if not args.no_backward:
         try:
             bwd = bench_backward(args, dev, world, clk, w, q, k_rot, v, pos, sel_g, hp, q_rot)
         except Exception as exc:               # noqa: BLE001 - reported, not raised

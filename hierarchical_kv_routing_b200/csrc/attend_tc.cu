@@ -29,6 +29,8 @@
 // records an error word and the CTA winds down.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "hga_internal.cuh"
 #include "sm100.cuh"
 
@@ -88,7 +90,9 @@ struct TcArgs {
     int rows_per_unit, ctas_per_unit, tokM;
     int cs_tokens;            // > 0: the CTA's (token, pair) cos/sin table is in smem
     int prerot;               // the Q tiles are already rotated (stage 2 wrote them)
+    int tma_out;              // O leaves through the output map (else row stores)
     int c0;                   // first query block of this launch
+    int B, nblk;              // sequences and query blocks of this launch (persistent form)
     // Host-resident tier: K/V rows come from the tier's buffers, not from the
     // token layout.  Tokens below sink_rows sit at row buf_row0 + token, other
     // fixed tokens at buf_row0 + win_row0 + token - win_tok0; routed group
@@ -140,6 +144,90 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// One key tile of the online softmax for one query row (thread = TMEM lane
+// of its M-tile; lane_base addresses the row's S columns, O follows at +128):
+// reads S, masks the columns at or past nvis (gc0 = the tile's first column
+// in the key list), updates the base-2 reference m_ref and the row sum l,
+// writes P (bf16) over the S columns and rescales O in TMEM when the
+// reference grows.  Ends with the TMEM stores complete.
+template <int D>
+__device__ __forceinline__ void softmax_tile(uint32_t lane_base, int gc0, int nvis, bool valid,
+                                             float sc, float &m_ref, float &l) {
+    // the row's visible keys are the first nvis columns of the list
+    const bool need_mask = gc0 + kSegPerTile * 8 > nvis;
+    // one TMEM pass: the S row (up to 128 columns) into registers
+    uint32_t v[128];
+    tmem_ld32(lane_base + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+    tmem_ld32(lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+    tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
+    tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
+    tmem_ld_wait();
+    if (need_mask) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e)
+            if (gc0 + e >= nvis) v[e] = __float_as_uint(-INFINITY);
+    }
+    // row max with 8 independent chains of three-input maxima
+    float mx8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(__uint_as_float(v[u]), __uint_as_float(v[u + 8]));
+#pragma unroll
+    for (int e = 16; e < 128; e += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            mx8[u] = max3f(mx8[u], __uint_as_float(v[e + u]), __uint_as_float(v[e + 8 + u]));
+    float mx = fmaxf(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]));
+    mx = max3f(mx, mx8[6], mx8[7]);
+    if (!valid) mx = -INFINITY;
+    const float mt_new = mx * sc;
+    // The reference grows only when the row max rises by more than
+    // 2^8; P uses the new reference, and O (accumulated under the
+    // old one) is rescaled below, before this tile's P.V.
+    const bool grow = mt_new > m_ref + 8.0f;
+    const bool rescale = grow && m_ref != -INFINITY;
+    const float f = rescale ? ex2(m_ref - mt_new) : 1.0f;
+    if (grow) m_ref = mt_new;
+    l *= f;
+    // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
+    const bool live = m_ref != -INFINITY;
+    const float neg = -m_ref;
+    // pairs of columns in packed two-lane fp32: s * scale - m_ref
+    // and the row sum (4 chains of pairs), ex2 per column
+    const uint64_t sc2 = f2_pack(sc, sc), neg2 = f2_pack(neg, neg);
+    uint64_t l4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) l4[u] = f2_pack(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+        float p0 = 0.f, p1 = 0.f;
+        if (live) {
+            const float2 x = f2_unpack(f2_fma(
+                f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2));
+            p0 = ex2(x.x);
+            p1 = ex2(x.y);
+        }
+        l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
+        v[e] = pack_bf16(p0, p1);
+    }
+    const float2 la = f2_unpack(f2_add(l4[0], l4[1])), lb = f2_unpack(f2_add(l4[2], l4[3]));
+    l += (la.x + la.y) + (lb.x + lb.y);
+    tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
+    tmem_st32(lane_base + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
+    // tcgen05.ld/st are warp-collective: the warp rescales O
+    // together when any of its rows needs it (factor 1 elsewhere)
+    if (__any_sync(0xffffffffu, rescale)) {
+        for (int cb = 0; cb < D / 32; ++cb) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + 128 + cb * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(lane_base + 128 + cb * 32, o);
+        }
+    }
+    tmem_st_wait();
+}
+
 // kTier: keys come from the host tier's buffers and group cache (TcArgs tier
 // fields) instead of the token layout; a separate instantiation, so the
 // in-HBM prefill's code is not touched by it.
@@ -148,7 +236,8 @@ __global__ void __launch_bounds__(Shape<kOne>::kThreads, kOne ? 2 : 1)
 k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
             const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmK64,
-            const __grid_constant__ CUtensorMap tmV64, const TcArgs A) {
+            const __grid_constant__ CUtensorMap tmV64, const __grid_constant__ CUtensorMap tmO,
+            const TcArgs A) {
     using C = Cfg<D, kOne>;
     using SH = Shape<kOne>;
     constexpr int kThreads = SH::kThreads;
@@ -457,80 +546,7 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     break;
                 }
                 tc_fence_after();
-                // the row's visible keys are the first nvis columns of the list
-                const int gc0 = j * kSegPerTile * 8;
-                const bool need_mask = gc0 + kSegPerTile * 8 > nvis;
-                // one TMEM pass: the S row (up to 128 columns) into registers
-                uint32_t v[128];
-                tmem_ld32(lane_base + 0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tmem_ld32(lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&v[64]));
-                tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&v[96]));
-                tmem_ld_wait();
-                if (need_mask) {
-#pragma unroll
-                    for (int e = 0; e < 128; ++e)
-                        if (gc0 + e >= nvis) v[e] = __float_as_uint(-INFINITY);
-                }
-                // row max with 8 independent chains of three-input maxima
-                float mx8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(__uint_as_float(v[u]), __uint_as_float(v[u + 8]));
-#pragma unroll
-                for (int e = 16; e < 128; e += 16)
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        mx8[u] = max3f(mx8[u], __uint_as_float(v[e + u]), __uint_as_float(v[e + 8 + u]));
-                float mx = fmaxf(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]));
-                mx = max3f(mx, mx8[6], mx8[7]);
-                if (!valid) mx = -INFINITY;
-                const float mt_new = mx * sc;
-                // The reference grows only when the row max rises by more than
-                // 2^8; P uses the new reference, and O (accumulated under the
-                // old one) is rescaled below, before this tile's P.V.
-                const bool grow = mt_new > m_ref + 8.0f;
-                const bool rescale = grow && m_ref != -INFINITY;
-                const float f = rescale ? ex2(m_ref - mt_new) : 1.0f;
-                if (grow) m_ref = mt_new;
-                l *= f;
-                // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
-                const bool live = m_ref != -INFINITY;
-                const float neg = -m_ref;
-                // pairs of columns in packed two-lane fp32: s * scale - m_ref
-                // and the row sum (4 chains of pairs), ex2 per column
-                const uint64_t sc2 = f2_pack(sc, sc), neg2 = f2_pack(neg, neg);
-                uint64_t l4[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) l4[u] = f2_pack(0.f, 0.f);
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    float p0 = 0.f, p1 = 0.f;
-                    if (live) {
-                        const float2 x = f2_unpack(f2_fma(
-                            f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2));
-                        p0 = ex2(x.x);
-                        p1 = ex2(x.y);
-                    }
-                    l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
-                    v[e] = pack_bf16(p0, p1);
-                }
-                const float2 la = f2_unpack(f2_add(l4[0], l4[1])), lb = f2_unpack(f2_add(l4[2], l4[3]));
-                l += (la.x + la.y) + (lb.x + lb.y);
-                tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&v[0]));
-                tmem_st32(lane_base + 32, *reinterpret_cast<const uint32_t(*)[32]>(&v[32]));
-                // tcgen05.ld/st are warp-collective: the warp rescales O
-                // together when any of its rows needs it (factor 1 elsewhere)
-                if (__any_sync(0xffffffffu, rescale)) {
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        uint32_t o[32];
-                        tmem_ld32(lane_base + 128 + cb * 32, o);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                        tmem_st32(lane_base + 128 + cb * 32, o);
-                    }
-                }
-                tmem_st_wait();
+                softmax_tile<D>(lane_base, j * kSegPerTile * 8, nvis, valid, sc, m_ref, l);
                 tc_fence_before();
                 mbar_arrive(&ctl.p_full[mt]);
             }
@@ -542,6 +558,12 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 }
             }
             tc_fence_after();
+            // With the output map, the normalised rows are staged in this
+            // M-tile's Q tile (its last S product completed before its last
+            // P.V), in the 128B-swizzled layout of the map's box (the Q
+            // tile's own), and leave as one tensor store per D-half; rows
+            // past the sequence's end fall outside the map and are not written.
+            uint8_t *ot = smem + C::oQ + mt * C::kTileBytes;
             if (ok) {
                 const float inv = valid && l > 0.f ? 1.f / l : 0.f;
                 __nv_bfloat16 *orow =
@@ -561,7 +583,11 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                             for (int e = 0; e < 4; ++e)
                                 wp[e] = pack_bf16(__uint_as_float(v[q8 * 8 + 2 * e]) * inv,
                                                   __uint_as_float(v[q8 * 8 + 2 * e + 1]) * inv);
-                            reinterpret_cast<uint4 *>(orow)[hb * 8 + q8] = w;
+                            if (A.tma_out)
+                                *reinterpret_cast<uint4 *>(ot + hb * C::kHalfBytes + r * 128 +
+                                                           ((q8 ^ (r & 7)) << 4)) = w;
+                            else
+                                reinterpret_cast<uint4 *>(orow)[hb * 8 + q8] = w;
                         }
                     }
                 }
@@ -569,7 +595,393 @@ k_attend_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                     A.lse[((int64_t)b * A.Hq + (int64_t)h * A.G + head) * A.T + tok] =
                         (m_ref + __log2f(l)) * 0.6931471805599453f;
             }
+            if (A.tma_out) {
+                // every thread of the warpgroup reaches this barrier once
+                fence_proxy_async_smem();
+                if (mt == 0) named_bar(2, 128);
+                else named_bar(3, 128);
+                if (r == 0 && ok && !ctl.abort) {
+                    const int tok_first = t0 + (row0 + mt * 128) / A.G;
+                    for (int hf = 0; hf < C::kHalves; ++hf)
+                        tma_store_4d(&tmO, ot + hf * C::kHalfBytes, hf * 64, h * A.G, tok_first, b);
+                    bulk_commit();
+                    bulk_wait_read();      // the tile is read before the CTA exits
+                }
+            }
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, SH::kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------
+// Persistent form (rotated queries given, units of at least 256 rows, no
+// tier): one CTA per SM walks the units blockIdx.x, blockIdx.x + gridDim.x,
+// ... (the order of the one-unit-per-CTA grid).  Stage rings and barrier
+// phases run on across units, so a unit's set-up and epilogue overlap the
+// key loops around it:
+//   warp 3      builds the segment list of each unit into one of two buffers
+//               and loads its two rotated Q tiles, each as soon as the
+//               previous unit's last S product on that tile has completed.
+//   warps 0, 2  stream the K and V tiles of unit after unit.
+//   warp 1      issues the products; a unit's first S follows the previous
+//               unit's last P.V on the same M-tile.
+//   warps 4-11  softmax as above; each M-tile's epilogue (O from TMEM to
+//               row stores) runs while the tensor core starts the next unit,
+//               whose first P.V waits for the softmax warps anyway.
+constexpr int kMaxSegP = 1024;
+
+struct CtlP {
+    uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2];
+    uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
+    uint64_t seg_full[2], seg_empty[2];
+    uint64_t fin;
+    uint32_t tmem_base;
+    volatile int abort;
+    int nseg[2], first_cur[2];
+    int seg_tok[2][kMaxSegP];
+};
+constexpr uint32_t kSegConsumers = 3 + 8;   // K, V producers, MMA issuer, 8 softmax warps
+
+struct UnitP {
+    int c, cu, h, b;
+};
+
+// Unit u in the one-unit-per-CTA grid's order: (block, row half) fastest,
+// then KV head, then sequence.
+__device__ __forceinline__ UnitP unit_at(const TcArgs &A, int u) {
+    UnitP p;
+    const int per_h = A.nblk * A.ctas_per_unit;
+    const int per_b = per_h * A.Hkv;
+    p.b = u / per_b;
+    const int rem = u - p.b * per_b;
+    p.h = rem / per_h;
+    const int x = rem - p.h * per_h;
+    p.c = A.c0 + x / A.ctas_per_unit;
+    p.cu = x - (x / A.ctas_per_unit) * A.ctas_per_unit;
+    return p;
+}
+
+__device__ __forceinline__ void fail_p(CtlP &ctl) {
+    ctl.abort = 1;
+    atomicExch(&g_attend_tc_error, (int)HGA_ERR_TIMEOUT);
+}
+
+// The visible set of one unit's rows as 8-token segments (sinks, recent
+// chunks, routed groups, then the current chunk up to the unit's last query
+// token), written by one whole warp into buffer buf.
+__device__ __forceinline__ void build_segments_p(CtlP &ctl, int buf, const TcArgs &A,
+                                                 const UnitP &un) {
+    const int lane = threadIdx.x & 31;
+    const int c = un.c, t0 = c * kChunk;
+    const int row0 = un.cu * 256;
+    const int rows = min(256, A.rows_per_unit - row0);
+    const int max_tok = min(t0 + (row0 + rows - 1) / A.G, A.T - 1);
+    int *seg = ctl.seg_tok[buf];
+    const int nsink = min(A.F, c);
+    const int rec_lo = max(c - max(A.L, 1), nsink);
+    const int n_fixed = 8 * (nsink + (c - rec_lo));
+    for (int s = lane; s < n_fixed; s += 32)
+        seg[s] = s < 8 * nsink ? s * 8 : rec_lo * kChunk + (s - 8 * nsink) * 8;
+    const int32_t *sel = A.sel_group + (((int64_t)un.b * A.NB + c) * A.Hkv + un.h) * A.K_g;
+    const int gseg = A.g_s / 8;
+    int kg = 0;
+    for (int base = 0; base < A.K_g; base += 32) {
+        const int v = base + lane < A.K_g ? sel[base + lane] : -1;
+        kg += __popc(__ballot_sync(0xffffffffu, v >= 0));
+    }
+    for (int j = lane; j < kg; j += 32) {
+        const int r0 = sel[j] * A.g_s;
+        for (int e = 0; e < gseg; ++e) seg[n_fixed + j * gseg + e] = r0 + e * 8;
+    }
+    const int n_route = n_fixed + kg * gseg;
+    const int ncur = (max_tok - t0) / 8 + 1;
+    for (int e = lane; e < ncur; e += 32) seg[n_route + e] = t0 + e * 8;
+    __syncwarp();
+    if (lane == 0) {
+        int nseg = n_route + ncur;
+        if (nseg & 1) seg[nseg++] = kDummy;
+        ctl.nseg[buf] = nseg;
+        ctl.first_cur[buf] = n_route;
+    }
+    __syncwarp();
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+k_attend_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+             const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
+             const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmK64,
+             const __grid_constant__ CUtensorMap tmV64, const TcArgs A) {
+    using C = Cfg<D, false>;
+    using SH = Shape<false>;
+    constexpr int kS = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ CtlP ctl;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NU = A.B * A.Hkv * A.nblk * A.ctas_per_unit;
+
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl.q_full[i], 1);
+            mbar_init(&ctl.q_empty[i], 1);
+            mbar_init(&ctl.s_full[i], 1);
+            mbar_init(&ctl.p_full[i], 128);
+            mbar_init(&ctl.o_full[i], 1);
+            mbar_init(&ctl.seg_full[i], 1);
+            mbar_init(&ctl.seg_empty[i], kSegConsumers);
+        }
+        for (int i = 0; i < kS; ++i) {
+            mbar_init(&ctl.k_full[i], 1);
+            mbar_init(&ctl.v_full[i], 1);
+            mbar_init(&ctl.k_empty[i], 1);
+            mbar_init(&ctl.v_empty[i], 1);
+        }
+        mbar_init(&ctl.fin, 1);
+        ctl.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl.tmem_base, SH::kTmemCols);
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    if (warp < 4) {
+        regs_dec<SH::kRegsCtl>();
+        if ((warp == 0 || warp == 2) && lane == 0) {
+            // ------------------------------------------------- producers --
+            const bool is_k = warp == 0;
+            const CUtensorMap *m8 = is_k ? &tmK : &tmV;
+            const CUtensorMap *m16 = is_k ? &tmK16 : &tmV16;
+            const CUtensorMap *m64 = is_k ? &tmK64 : &tmV64;
+            prefetch_tensormap(m8);
+            prefetch_tensormap(m16);
+            prefetch_tensormap(m64);
+            uint64_t *full = is_k ? ctl.k_full : ctl.v_full;
+            uint64_t *empty = is_k ? ctl.k_empty : ctl.v_empty;
+            const uint32_t ring = is_k ? C::oK : C::oV;
+            const int kvT = is_k ? A.k_T : A.v_T;
+            int gt = 0;          // tiles issued so far, over all units
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int u = blockIdx.x + i * gridDim.x;
+                if (u >= NU || ctl.abort) break;
+                const int buf = i & 1;
+                if (!(ok = mbar_wait_ab(&ctl.seg_full[buf], (i >> 1) & 1, &ctl.abort))) break;
+                const UnitP un = unit_at(A, u);
+                const int nseg = ctl.nseg[buf];
+                const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
+                const int *sg = ctl.seg_tok[buf];
+                for (int j = 0; j < ntiles; ++j, ++gt) {
+                    const int s = gt % kS;
+                    if (gt >= kS && !(ok = mbar_wait_ab(&empty[s], ((gt / kS) - 1) & 1, &ctl.abort)))
+                        break;
+                    const int nsj = min(kSegPerTile, nseg - j * kSegPerTile);
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)nsj * 8 * D * 2);
+                    load_tile<C::kHalves>(smem + ring + s * C::kTileBytes, C::kHalfBytes,
+                                          sg + j * kSegPerTile, nsj, m8, m16, m64, &full[s], un.h,
+                                          un.b * kvT);
+                }
+                if (ok) mbar_arrive(&ctl.seg_empty[buf]);
+            }
+            if (!ok) {
+                fail_p(ctl);
+                // let the copies already issued land before the CTA exits
+                for (int t = max(0, gt - kS); t < gt; ++t)
+                    mbar_wait(&full[t % kS], (t / kS) & 1, 100000000ull);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------------------------ MMA issuer --
+            const uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            auto issue_pv = [&](int mt, int sp, int nsj, bool acc) {
+                const uint32_t vbase = smem_addr(smem + C::oV + sp * C::kTileBytes);
+                for (int ks = 0; ks < nsj / 2; ++ks) {
+                    const uint64_t bd = smem_desc_sw128(vbase + ks * 2048, C::kHalfBytes, 1024);
+                    mma_ts(tmem + mt * 256 + 128, tmem + mt * 256 + ks * 8, bd, idesc_pv,
+                           (acc || ks > 0) ? 1u : 0u);
+                }
+            };
+            auto issue_s = [&](int mt, int s, int nsj) {
+                const uint32_t idesc = idesc_bf16_f32(128, nsj * 8, false, false);
+                const uint32_t qb = smem_addr(smem + C::oQ + mt * C::kTileBytes);
+                const uint32_t kb = smem_addr(smem + C::oK + s * C::kTileBytes);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+                    mma_ss(tmem + mt * 256, smem_desc_sw128(qb + off, 16, 1024),
+                           smem_desc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                }
+            };
+            bool ok = true;
+            int g0 = 0;          // global index of the unit's first tile
+            for (int i = 0; ok; ++i) {
+                const int u = blockIdx.x + i * gridDim.x;
+                if (u >= NU || ctl.abort) break;
+                const int buf = i & 1;
+                if (!(ok = mbar_wait_ab(&ctl.seg_full[buf], (i >> 1) & 1, &ctl.abort))) break;
+                const int nseg = ctl.nseg[buf];
+                mbar_arrive(&ctl.seg_empty[buf]);
+                const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
+                // per tile j: P.V of tile j-1 (it needs no new data), then S
+                // of tile j; K stages are released after both S products, V
+                // stages after both P.V products
+                for (int j = 0; j <= ntiles && ok; ++j) {
+                    const int gs = g0 + j;
+                    const int s = gs % kS;
+                    for (int mt = 0; mt < 2 && ok; ++mt) {
+                        if (j > 0) {
+                            if (!(ok = mbar_wait_ab(&ctl.p_full[mt], (gs - 1) & 1, &ctl.abort))) break;
+                            tc_fence_after();
+                            const int sp = (gs - 1) % kS;
+                            if (mt == 0) {
+                                if (!(ok = mbar_wait_ab(&ctl.v_full[sp], ((gs - 1) / kS) & 1, &ctl.abort)))
+                                    break;
+                                tc_fence_after();
+                            }
+                            issue_pv(mt, sp, min(kSegPerTile, nseg - (j - 1) * kSegPerTile), j > 1);
+                            if (j == ntiles) mma_commit(&ctl.o_full[mt]);
+                            if (mt == 1) mma_commit(&ctl.v_empty[sp]);
+                        }
+                        if (j < ntiles) {
+                            if (j == 0) {
+                                if (!(ok = mbar_wait_ab(&ctl.q_full[mt], i & 1, &ctl.abort))) break;
+                                tc_fence_after();
+                            }
+                            if (mt == 0) {
+                                if (!(ok = mbar_wait_ab(&ctl.k_full[s], (gs / kS) & 1, &ctl.abort))) break;
+                                tc_fence_after();
+                            }
+                            issue_s(mt, s, min(kSegPerTile, nseg - j * kSegPerTile));
+                            mma_commit(&ctl.s_full[mt]);
+                            if (j == ntiles - 1) mma_commit(&ctl.q_empty[mt]);
+                            if (mt == 1) mma_commit(&ctl.k_empty[s]);
+                        }
+                    }
+                }
+                g0 += ntiles;
+            }
+            if (!ok) fail_p(ctl);
+            // all issued tensor-core work retires before TMEM is released
+            mma_commit(&ctl.fin);
+            if (!mbar_wait(&ctl.fin, 0)) fail_p(ctl);
+        } else if (warp == 3) {
+            // ------------------------------- segment lists and Q tiles --
+            bool ok = true;
+            int issued = 0;      // units whose Q tiles were issued
+            for (int i = 0; ok; ++i) {
+                const int u = blockIdx.x + i * gridDim.x;
+                if (u >= NU || ctl.abort) break;
+                const int buf = i & 1;
+                if (i >= 2) {
+                    if (lane == 0)
+                        ok = mbar_wait_ab(&ctl.seg_empty[buf], ((i >> 1) - 1) & 1, &ctl.abort);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                }
+                const UnitP un = unit_at(A, u);
+                build_segments_p(ctl, buf, A, un);
+                if (lane == 0) {
+                    mbar_arrive(&ctl.seg_full[buf]);
+                    if (i == 0) prefetch_tensormap(&tmQ);
+                    for (int mt = 0; mt < 2 && ok; ++mt) {
+                        if (i >= 1 && !(ok = mbar_wait_ab(&ctl.q_empty[mt], (i - 1) & 1, &ctl.abort)))
+                            break;
+                        const int tok_first = un.c * kChunk + (un.cu * 256 + mt * 128) / A.G;
+                        mbar_arrive_expect_tx(&ctl.q_full[mt], (uint32_t)(A.G * A.tokM * D * 2));
+                        for (int hf = 0; hf < C::kHalves; ++hf)
+                            tma_load_3d(smem + C::oQ + mt * C::kTileBytes + hf * C::kHalfBytes, &tmQ,
+                                        &ctl.q_full[mt], hf * 64, un.h * A.G,
+                                        un.b * A.T + tok_first);
+                    }
+                    if (ok) issued = i + 1;
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+            }
+            if (lane == 0 && !ok) {
+                fail_p(ctl);
+                // the last unit's Q tiles land before the CTA exits
+                if (issued > 0)
+                    for (int mt = 0; mt < 2; ++mt)
+                        mbar_wait(&ctl.q_full[mt], (issued - 1) & 1, 100000000ull);
+            }
+        }
+    } else {
+        regs_inc<SH::kRegsSoftmax>();
+        // ------------------------------------------------------- softmax --
+        const int mt = (warp - 4) >> 2;
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16) + mt * 256;
+        const float sc = A.scale_log2;
+        bool ok = true;
+        int g0 = 0;
+        for (int i = 0; ok; ++i) {
+            const int u = blockIdx.x + i * gridDim.x;
+            if (u >= NU || ctl.abort) break;
+            const int buf = i & 1;
+            if (!(ok = mbar_wait_ab(&ctl.seg_full[buf], (i >> 1) & 1, &ctl.abort))) break;
+            const int first_cur = ctl.first_cur[buf];
+            const int nseg = ctl.nseg[buf];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.seg_empty[buf]);
+            const UnitP un = unit_at(A, u);
+            const int t0 = un.c * kChunk;
+            const int R = un.cu * 256 + mt * 128 + r;
+            const int tok = t0 + R / A.G;
+            const int head = R % A.G;
+            const bool valid = tok < A.T;
+            const int nvis = first_cur * 8 + (tok - t0 + 1);
+            const int ntiles = (nseg + kSegPerTile - 1) / kSegPerTile;
+            float m_ref = -INFINITY, l = 0.f;
+            for (int j = 0; j < ntiles; ++j) {
+                if (!(ok = mbar_wait_ab(&ctl.s_full[mt], (g0 + j) & 1, &ctl.abort))) break;
+                tc_fence_after();
+                softmax_tile<D>(lane_base, j * kSegPerTile * 8, nvis, valid, sc, m_ref, l);
+                tc_fence_before();
+                mbar_arrive(&ctl.p_full[mt]);
+            }
+            g0 += ntiles;
+            if (!ok || !(ok = mbar_wait_ab(&ctl.o_full[mt], i & 1, &ctl.abort))) break;
+            tc_fence_after();
+            // epilogue: O / l -> out (row stores), LSE; the TMEM reads complete
+            // before this warp's next p_full arrival lets the next unit's
+            // first P.V overwrite O
+            const float inv = valid && l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16 *orow =
+                A.out + (((int64_t)un.b * A.T + tok) * A.Hq + (int64_t)un.h * A.G + head) * D;
+#pragma unroll
+            for (int hb = 0; hb < D / 64; ++hb) {
+                uint32_t v[64];
+                tmem_ld32(lane_base + 128 + hb * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tmem_ld32(lane_base + 128 + hb * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                tmem_ld_wait();
+                if (valid) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        uint4 w;
+                        uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            wp[e] = pack_bf16(__uint_as_float(v[q8 * 8 + 2 * e]) * inv,
+                                              __uint_as_float(v[q8 * 8 + 2 * e + 1]) * inv);
+                        reinterpret_cast<uint4 *>(orow)[hb * 8 + q8] = w;
+                    }
+                }
+            }
+            if (valid && A.lse)
+                A.lse[((int64_t)un.b * A.Hq + (int64_t)un.h * A.G + head) * A.T + tok] =
+                    (m_ref + __log2f(l)) * 0.6931471805599453f;
+        }
+        if (!ok) fail_p(ctl);
     }
     tc_fence_before();
     __syncthreads();
@@ -605,6 +1017,23 @@ bool make_map(CUtensorMap *m, const void *base, int D, int heads, long long n_ro
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 4-D bf16 map over [n_seq][T][heads][D]: box (64, box_heads, box_rows, 1),
+// 128-byte swizzle; a box never reaches past its own sequence's last token.
+bool make_map_4d(CUtensorMap *m, const void *base, int D, int heads, int T, int n_seq,
+                 int box_heads, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)n_seq};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2,
+                             (cuuint64_t)T * heads * D * 2};
+    cuuint32_t box[4] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1u};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -663,11 +1092,35 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
                         (size_t)a.cs_tokens * (D / 2 + 1) * sizeof(float2);
     auto kern = tw ? (one ? k_attend_tc<D, true, true> : k_attend_tc<D, true, false>)
                    : (one ? k_attend_tc<D, false, true> : k_attend_tc<D, false, false>);
+    a.B = g.B;
+    a.nblk = nblk;
+    // rotated queries, no tier, units of at least 256 rows: the persistent
+    // form, one CTA per SM
+    const long long n_units = (long long)g.B * g.Hkv * nblk * a.ctas_per_unit;
+    const long long segs = 8ll * (g.F + max(g.L, 1) + 1) + (long long)g.K_g * (g.g_s / 8) + 2;
+    if (q_rot && !tw && a.rows_per_unit >= 256 && segs <= kMaxSegP && n_units < (1ll << 30)) {
+        int dev = 0, nsm = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_status(e);
+        const size_t psmem = Cfg<D>::oEnd + 1024;
+        auto pk = k_attend_tcp<D>;
+        if ((e = ensure_smem((const void *)pk, psmem)) != cudaSuccess) return cuda_status(e);
+        const int grid = (int)std::min<long long>(n_units, std::max(nsm, 1));
+        pk<<<grid, Shape<false>::kThreads, psmem, st>>>(mq, mk, mv, mk16, mv16, mk64, mv64, a);
+        return cuda_status(cudaGetLastError());
+    }
+    // the calls check that out is 16-byte aligned (the map needs it); row
+    // stores remain for any other base
+    CUtensorMap mo;
+    a.tma_out = (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
+                make_map_4d(&mo, out, D, g.Hq, g.T, g.B, g.G, a.tokM);
+    if (!a.tma_out) mo = mq;      // unused
     cudaError_t e = ensure_smem((const void *)kern, smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid(nblk * a.ctas_per_unit, g.Hkv, g.B);
     kern<<<grid, one ? Shape<true>::kThreads : Shape<false>::kThreads, smem, st>>>(
-        mq, mk, mv, mk16, mv16, mk64, mv64, a);
+        mq, mk, mv, mk16, mv16, mk64, mv64, mo, a);
     return cuda_status(cudaGetLastError());
 }
 

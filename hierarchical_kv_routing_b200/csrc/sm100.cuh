@@ -71,6 +71,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     return false;
 }
 
+// mbar_wait that also gives up once *abort is set (checked every 1024 polls),
+// so that the roles of a CTA that already failed stop waiting for each other.
+__device__ __forceinline__ bool mbar_wait_ab(uint64_t *bar, uint32_t parity,
+                                             const volatile int *abort,
+                                             uint64_t limit_ns = kMaxWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && (*abort || global_ns() - t0 > limit_ns)) break;
+    }
+    return false;
+}
+
 // -------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar,
@@ -128,6 +142,17 @@ __device__ __forceinline__ void bulk_commit() {
 // Wait until this thread's committed bulk stores have read their shared source.
 __device__ __forceinline__ void bulk_wait_read() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Tiled store shared -> global through a 4-D tensor map (coordinates x
+// innermost; elements outside the tensor are not written), tracked by this
+// thread's bulk groups like bulk_store.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src, int x, int y,
+                                             int z, int w) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(src)), "r"(x), "r"(y),
+                 "r"(z), "r"(w)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {

@@ -35,6 +35,8 @@
  *  - dtype (hga_dims.dtype) is the element type of Q, K, V, K_rot and O:
  *    HGA_F32 or HGA_BF16.  Summaries, scores and accumulation are fp32 or
  *    wider.
+ *  - Every tensor pointer (inputs, outputs, caches, summaries) must be
+ *    16-byte aligned; another base is HGA_ERR_INVALID_ARG.
  *  - Errors: arguments are checked on the host first; a failing check
  *    returns HGA_ERR_INVALID_ARG or HGA_ERR_UNSUPPORTED and launches nothing.
  *    Size limits of this build (HGA_ERR_UNSUPPORTED beyond them): B <= 65535,

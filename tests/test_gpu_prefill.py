@@ -35,6 +35,9 @@ CASES = {
     "bf16_qwen_2048": QWEN.replace(T=2048),
     "bf16_qwen_ragged": QWEN.replace(T=64 * 20 + 33),
     "bf16_qwen_L0_F0": QWEN.replace(T=1280, F=0, L=0, K_c=5, K_g=9),
+    # two sequences with a ragged last block: the output tiles of the first
+    # sequence's last block must not reach into the second sequence
+    "bf16_qwen_2x_ragged": QWEN.replace(B=2, T=64 * 9 + 17),
     # bf16 shapes the tensor-core kernel does not take (Hq/Hkv not a power of
     # two; groups shorter than its 8-token segments) run on the CUDA cores
     "bf16_G3_cuda_cores": QWEN.replace(T=64 * 12 + 5, Hq=6, Hkv=2, K_c=4, K_g=8),
@@ -165,6 +168,26 @@ def test_exact_token_chunk_variant(gpu_lib):
             chunks = sc[0, blk, h][sc[0, blk, h] >= 0]
             groups = sg[0, blk, h][sg[0, blk, h] >= 0]
             assert sorted(groups.tolist()) == sorted((chunks[:, None] * gpc + np.arange(gpc)).ravel().tolist())
+
+
+def test_attend_rejects_unaligned_output(gpu_lib):
+    """Tensor pointers must be 16-byte aligned (the output leaves by tensor
+    stores): another base is refused before any launch."""
+    hga = gpu_lib
+    w = CASES["bf16_qwen_2x_ragged"]
+    q, k, v, pos, _ = make_prefill_inputs(w, seed=3)
+    dev = torch.device("cuda")
+    qd, kd, vd, pd = (x.to(dev) for x in (q, k, v, pos))
+    hp = _hp(w)
+    k_rot, s_c, s_g = hga.hga_build_summaries(kd, pd, hp)
+    _, sel_g = hga.hga_route(qd, pd, s_c, s_g, hp)
+    raw = torch.zeros((qd.numel() + 1,), dtype=qd.dtype, device=dev)
+    shifted = raw[1:].view(qd.shape)
+    assert shifted.data_ptr() % 16 != 0
+    with pytest.raises(hga.HGAError, match="invalid argument"):
+        hga.hga_attend(qd, pd, k_rot, vd, sel_g, hp, out=shifted)
+    torch.cuda.synchronize()
+    assert not raw.any()
 
 
 @pytest.mark.parametrize("name,mod", [("f32_ragged_1000", 300), ("bf16_qwen_ragged", 1000)])
