@@ -201,10 +201,13 @@ __device__ __forceinline__ void softmax_tile(uint32_t lane_base, int gc0, int nv
     for (int e = 0; e < 64; ++e) {
         float p0 = 0.f, p1 = 0.f;
         if (live) {
-            const float2 x = f2_unpack(f2_fma(
-                f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2));
-            p0 = ex2(x.x);
-            p1 = ex2(x.y);
+            const uint64_t x2 = f2_fma(
+                f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2);
+            {
+                const float2 x = f2_unpack(x2);
+                p0 = ex2(x.x);
+                p1 = ex2(x.y);
+            }
         }
         l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
         v[e] = pack_bf16(p0, p1);
@@ -958,22 +961,22 @@ k_attend_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             const float inv = valid && l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow =
                 A.out + (((int64_t)un.b * A.T + tok) * A.Hq + (int64_t)un.h * A.G + head) * D;
+            {
+                uint32_t v[D];
 #pragma unroll
-            for (int hb = 0; hb < D / 64; ++hb) {
-                uint32_t v[64];
-                tmem_ld32(lane_base + 128 + hb * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tmem_ld32(lane_base + 128 + hb * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                for (int cb = 0; cb < D / 32; ++cb)
+                    tmem_ld32(lane_base + 128 + cb * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[cb * 32]));
                 tmem_ld_wait();
                 if (valid) {
 #pragma unroll
-                    for (int q8 = 0; q8 < 8; ++q8) {
+                    for (int q8 = 0; q8 < D / 8; ++q8) {
                         uint4 w;
                         uint32_t *wp = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
                             wp[e] = pack_bf16(__uint_as_float(v[q8 * 8 + 2 * e]) * inv,
                                               __uint_as_float(v[q8 * 8 + 2 * e + 1]) * inv);
-                        reinterpret_cast<uint4 *>(orow)[hb * 8 + q8] = w;
+                        reinterpret_cast<uint4 *>(orow)[q8] = w;
                     }
                 }
             }
