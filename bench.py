@@ -915,7 +915,7 @@ def main():
     peak = pk.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic_for_current_kernel(),
-            "kernel": "k_attend_tc<128> (routed attention, tcgen05)",
+            "kernel": "k_attend_tcp<128> (routed attention, tcgen05, persistent)",
             "flops_per_launch": flops, "avg_launch_ms": stage_ms[2],
             "peak_source": f"{src} bf16_tflops (burst; the kernel is timed alone per launch)"}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
