@@ -758,6 +758,9 @@ k_attend_tcp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
+    // launched as a programmatic dependent of stage 2: the set-up above ran
+    // while it finished; the routed sets and rotated queries are read below
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp < 4) {
         regs_dec<SH::kRegsCtl>();
@@ -1109,9 +1112,17 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos, c
         const size_t psmem = Cfg<D>::oEnd + 1024;
         auto pk = k_attend_tcp<D>;
         if ((e = ensure_smem((const void *)pk, psmem)) != cudaSuccess) return cuda_status(e);
-        const int grid = (int)std::min<long long>(n_units, std::max(nsm, 1));
-        pk<<<grid, Shape<false>::kThreads, psmem, st>>>(mq, mk, mv, mk16, mv16, mk64, mv64, a);
-        return cuda_status(cudaGetLastError());
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)std::min<long long>(n_units, std::max(nsm, 1)));
+        cfg.blockDim = dim3(Shape<false>::kThreads);
+        cfg.dynamicSmemBytes = psmem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cuda_status(cudaLaunchKernelEx(&cfg, pk, mq, mk, mv, mk16, mv16, mk64, mv64, a));
     }
     // the calls check that out is 16-byte aligned (the map needs it); row
     // stores remain for any other base

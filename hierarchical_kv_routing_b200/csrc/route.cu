@@ -172,6 +172,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
         __syncthreads();
     }
 
+    // Phase 1 reads only the queries and positions.  Launched as a
+    // programmatic dependent of stage 1, the kernel overlaps it with the
+    // summaries and waits here for them (and their memory) to complete; the
+    // next kernel (stage 3) may then be launched as this one winds down.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
     // ---- phase 2: chunk scores for every block of the run, one row read once
     const float *Sc = A.s_chunk + ((int64_t)b * A.Hkv + h) * A.nc_cap * D;
     const float *Sg = A.s_group + ((int64_t)b * A.Hkv + h) * A.nc_cap * A.gpc * D;
@@ -356,9 +363,19 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     // the kernel forms a 32-bit linear CTA index
     if ((long long)((g.NB + a.nblk - 1) / a.nblk) * g.Hkv * g.B > (long long)INT32_MAX)
         return HGA_ERR_UNSUPPORTED;
-    dim3 grid((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
-    kern<<<grid, kThreads, smem, st>>>(a);
-    return cuda_status(cudaGetLastError());
+    // a programmatic dependent of the previous kernel on the stream: when
+    // that is stage 1 (which triggers early), the query stream overlaps it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, a));
 }
 
 }  // namespace

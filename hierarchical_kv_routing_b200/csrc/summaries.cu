@@ -101,6 +101,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_summaries(const SumArgs A) {
     // the chunk's positions, one coalesced load
     if (threadIdx.x < n) s_pos[threadIdx.x] = pb[threadIdx.x];
     __syncthreads();
+    // a kernel launched after this one as a programmatic dependent (stage 2)
+    // may start now: it reads what this kernel writes only after its
+    // griddepcontrol.wait
+    asm volatile("griddepcontrol.launch_dependents;");
 
     int pass = 0;
     for (int hs0 = 0; hs0 < A.Hkv; hs0 += A.HS, ++pass) {
