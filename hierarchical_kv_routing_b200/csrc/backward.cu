@@ -550,33 +550,46 @@ k_bwd_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUt
                 tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
                 tmem_ld_wait();
                 const int gc0 = (t % ntiles) * C::kSegPerTile * 8;
+                if (gc0 + 64 > nvis) {
+                    // the row's visible keys end inside this tile: the later
+                    // columns (and any past the tile's keys, which hold stale
+                    // values) get P = 0 and dP = 0, with no per-column branch
+#pragma unroll
+                    for (int col = 0; col < 64; ++col)
+                        if (gc0 + col >= nvis) {
+                            sv[col] = __float_as_uint(-INFINITY);
+                            dp[col] = 0u;
+                        }
+                }
+                // pairs of columns in packed two-lane fp32: x = s * scale - LSE
+                const uint64_t sc2 = f2_pack(sc, sc), nl2 = f2_pack(-lse2, -lse2);
                 if (t < ntiles) {
                     // Delta pass: sum of P dP over the row's visible keys
-                    float d8[8];
+                    uint64_t d4[4];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) d8[u] = 0.f;
-#pragma unroll
-                    for (int col = 0; col < 64; ++col) {
-                        const float p = gc0 + col < nvis
-                            ? ex2(fmaf(__uint_as_float(sv[col]), sc, -lse2)) : 0.f;
-                        // columns past the tile's keys hold stale values: only
-                        // visible keys (p > 0) contribute
-                        d8[col & 7] += p > 0.f ? p * __uint_as_float(dp[col]) : 0.f;
-                    }
-                    delta += ((d8[0] + d8[1]) + (d8[2] + d8[3])) + ((d8[4] + d8[5]) + (d8[6] + d8[7]));
-                    if (t == ntiles - 1 && valid) A.rowstat[grow].y = delta;
-                } else {
+                    for (int u = 0; u < 4; ++u) d4[u] = f2_pack(0.f, 0.f);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        float ds[2];
+                        const float2 x = f2_unpack(f2_fma(
+                            f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2, nl2));
+                        d4[e & 3] = f2_fma(f2_pack(ex2(x.x), ex2(x.y)),
+                                           f2_pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                                           d4[e & 3]);
+                    }
+                    const float2 da = f2_unpack(f2_add(d4[0], d4[1])), db = f2_unpack(f2_add(d4[2], d4[3]));
+                    delta += (da.x + da.y) + (db.x + db.y);
+                    if (t == ntiles - 1 && valid) A.rowstat[grow].y = delta;
+                } else {
+                    const uint64_t nd2 = f2_pack(-delta, -delta), is2 = f2_pack(isd, isd);
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int col = 2 * e + u;
-                            const float p = gc0 + col < nvis
-                                ? ex2(fmaf(__uint_as_float(sv[col]), sc, -lse2)) : 0.f;
-                            ds[u] = p > 0.f ? p * (__uint_as_float(dp[col]) - delta) * isd : 0.f;
-                        }
-                        sv[e] = pack_bf16(ds[0], ds[1]);
+                    for (int e = 0; e < 32; ++e) {
+                        const float2 x = f2_unpack(f2_fma(
+                            f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2, nl2));
+                        const float2 ds = f2_unpack(f2_mul(
+                            f2_mul(f2_pack(ex2(x.x), ex2(x.y)),
+                                   f2_add(f2_pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])), nd2)),
+                            is2));
+                        sv[e] = pack_bf16(ds.x, ds.y);
                     }
                     tmem_st32(lane_base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sv[0]));
                     tmem_st_wait();
@@ -694,13 +707,17 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     }
     if (warp == 2) build_segments(ctl, A, b, c, h, max_tok);
     if (warp == 3) {
-        // (LSE * log2 e, Delta) of every row of the unit; rows past the end
-        // of the sequence get +inf, so their probabilities are zero
+        // (-LSE * log2 e, -Delta) of every row of the unit (negated: they
+        // are added below); rows past the end of the sequence get -inf, so
+        // their probabilities are zero
         for (int R = lane; R < nsub * 64; R += 32) {
             const int tok = t0 + R / A.G;
-            stat[R] = R < nrows
-                ? A.rowstat[((int64_t)b * A.T + tok) * A.Hq + (int64_t)h * A.G + R % A.G]
-                : make_float2(INFINITY, 0.f);
+            float2 st = make_float2(-INFINITY, 0.f);
+            if (R < nrows) {
+                st = A.rowstat[((int64_t)b * A.T + tok) * A.Hq + (int64_t)h * A.G + R % A.G];
+                st = make_float2(-st.x, -st.y);
+            }
+            stat[R] = st;
         }
     }
     __syncthreads();
@@ -850,21 +867,33 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 tmem_ld32(base + 96, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
                 tmem_ld_wait();
                 const int R0 = i * 64;
+                if (R0 < rmin) {
+                    // rows before rmin do not see this key (and keys past the
+                    // last real one are seen by none): their entries get
+                    // P = 0 and dS = 0 whatever the tile's unused rows hold
+#pragma unroll
+                    for (int col = 0; col < 64; ++col)
+                        if (R0 + col < rmin) {
+                            sv[col] = __float_as_uint(-INFINITY);
+                            dp[col] = 0u;
+                        }
+                }
+                const uint64_t sc2 = f2_pack(sc, sc), is2 = f2_pack(isd, isd);
+                const float4 *st4 = reinterpret_cast<const float4 *>(stat + R0);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    float p[2], ds[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = 2 * e + u;
-                        const float2 st = stat[R0 + col];
-                        p[u] = R0 + col >= rmin
-                            ? ex2(fmaf(__uint_as_float(sv[col]), sc, -st.x)) : 0.f;
-                        // masked entries are exact zeros whatever the tile's
-                        // unused rows hold
-                        ds[u] = p[u] > 0.f ? p[u] * (__uint_as_float(dp[col]) - st.y) * isd : 0.f;
-                    }
-                    sv[e] = pack_bf16(p[0], p[1]);
-                    dp[e] = pack_bf16(ds[0], ds[1]);
+                    const float4 st = st4[e];           // (-lse, -delta) of rows R0 + 2e, + 1
+                    const float2 x = f2_unpack(f2_fma(
+                        f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2,
+                        f2_pack(st.x, st.z)));
+                    const float p0 = ex2(x.x), p1 = ex2(x.y);
+                    const float2 ds = f2_unpack(f2_mul(
+                        f2_mul(f2_pack(p0, p1),
+                               f2_add(f2_pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                                      f2_pack(st.y, st.w))),
+                        is2));
+                    sv[e] = pack_bf16(p0, p1);
+                    dp[e] = pack_bf16(ds.x, ds.y);
                 }
                 tmem_st32(base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sv[0]));
                 tmem_st32(base + 64, *reinterpret_cast<const uint32_t(*)[32]>(&dp[0]));
