@@ -878,22 +878,16 @@ k_bwd_dkv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                             dp[col] = 0u;
                         }
                 }
-                const uint64_t sc2 = f2_pack(sc, sc), is2 = f2_pack(isd, isd);
                 const float4 *st4 = reinterpret_cast<const float4 *>(stat + R0);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const float4 st = st4[e];           // (-lse, -delta) of rows R0 + 2e, + 1
-                    const float2 x = f2_unpack(f2_fma(
-                        f2_pack(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2,
-                        f2_pack(st.x, st.z)));
-                    const float p0 = ex2(x.x), p1 = ex2(x.y);
-                    const float2 ds = f2_unpack(f2_mul(
-                        f2_mul(f2_pack(p0, p1),
-                               f2_add(f2_pack(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
-                                      f2_pack(st.y, st.w))),
-                        is2));
+                    const float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), sc, st.x));
+                    const float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sc, st.z));
+                    const float d0 = p0 * (__uint_as_float(dp[2 * e]) + st.y) * isd;
+                    const float d1 = p1 * (__uint_as_float(dp[2 * e + 1]) + st.w) * isd;
                     sv[e] = pack_bf16(p0, p1);
-                    dp[e] = pack_bf16(ds.x, ds.y);
+                    dp[e] = pack_bf16(d0, d1);
                 }
                 tmem_st32(base + 0, *reinterpret_cast<const uint32_t(*)[32]>(&sv[0]));
                 tmem_st32(base + 64, *reinterpret_cast<const uint32_t(*)[32]>(&dp[0]));
