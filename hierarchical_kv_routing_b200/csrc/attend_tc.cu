@@ -189,8 +189,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t lane_base, int gc0, int nv
     if (grow) m_ref = mt_new;
     l *= f;
     // P = 2^(s*scale - m_ref) as packed bf16, in place, over the S columns
-    const bool live = m_ref != -INFINITY;
-    const float neg = -m_ref;
+    // A row with no reference yet has every column masked (a valid row sees
+    // a key of its first tile), so s * scale + 0 is -inf and P is 0 without
+    // a per-column branch; rows past the end are never stored.
+    const float neg = m_ref != -INFINITY ? -m_ref : 0.f;
     // pairs of columns in packed two-lane fp32: s * scale - m_ref
     // and the row sum (4 chains of pairs), ex2 per column
     const uint64_t sc2 = f2_pack(sc, sc), neg2 = f2_pack(neg, neg);
@@ -199,16 +201,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t lane_base, int gc0, int nv
     for (int u = 0; u < 4; ++u) l4[u] = f2_pack(0.f, 0.f);
 #pragma unroll
     for (int e = 0; e < 64; ++e) {
-        float p0 = 0.f, p1 = 0.f;
-        if (live) {
-            const uint64_t x2 = f2_fma(
-                f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2);
-            {
-                const float2 x = f2_unpack(x2);
-                p0 = ex2(x.x);
-                p1 = ex2(x.y);
-            }
-        }
+        const float2 x = f2_unpack(f2_fma(
+            f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, neg2));
+        const float p0 = ex2(x.x), p1 = ex2(x.y);
         l4[e & 3] = f2_add(l4[e & 3], f2_pack(p0, p1));
         v[e] = pack_bf16(p0, p1);
     }
