@@ -179,8 +179,10 @@ hga_status hga_route(const hga_dims *dims, const hga_params *prm,
  * result is bit-identical), q is still required for the CUDA-core kernel.
  * Which kernel runs: bf16 with Hq/Hkv a power of two <= 16, g_s a multiple
  * of 8 and a visible set of at most 2048 8-token segments runs on the tensor
- * cores (tcgen05); fp32, and bf16 outside those limits, run on the CUDA cores
- * in fp32 arithmetic.  Both give the same result within rounding (bf16
+ * cores (tcgen05): with q_rot given, Hq/Hkv >= 4 and at most 1024 segments
+ * as one persistent CTA per SM walking the (block, KV head, 256-row) units,
+ * else one CTA per unit; fp32, and bf16 outside those limits, run on the
+ * CUDA cores in fp32 arithmetic.  Both give the same result within rounding (bf16
  * outputs are rounded from fp32 accumulators). */
 hga_status hga_attend(const hga_dims *dims, const hga_params *prm,
                       const void *q, const int32_t *pos,
