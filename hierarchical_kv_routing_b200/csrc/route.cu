@@ -79,6 +79,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const T *q = static_cast<const T *>(A.q);
 
+    // Launched as a programmatic dependent of the previous kernel on the
+    // stream: nothing that kernel may write is read before it completes.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     // ---- phase 1: routing queries sum_i sum_{h'} R_{p_i}(q_{i,h'}), per block
     const int w = threadIdx.x % NS, jt = threadIdx.x / NS;
     for (int blk = 0; blk < nb; ++blk) {
@@ -172,11 +176,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_route(const RouteArgs A) {
         __syncthreads();
     }
 
-    // Phase 1 reads only the queries and positions.  Launched as a
-    // programmatic dependent of stage 1, the kernel overlaps it with the
-    // summaries and waits here for them (and their memory) to complete; the
-    // next kernel (stage 3) may then be launched as this one winds down.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the next kernel (stage 3) may be launched as this one winds down
     asm volatile("griddepcontrol.launch_dependents;");
 
     // ---- phase 2: chunk scores for every block of the run, one row read once
@@ -364,7 +364,7 @@ hga_status run(const Geo &g, const Rope &r, const void *q, const int32_t *pos,
     if ((long long)((g.NB + a.nblk - 1) / a.nblk) * g.Hkv * g.B > (long long)INT32_MAX)
         return HGA_ERR_UNSUPPORTED;
     // a programmatic dependent of the previous kernel on the stream: when
-    // that is stage 1 (which triggers early), the query stream overlaps it
+    // that is stage 1 (which triggers early), the launch and set-up overlap it
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((g.NB + a.nblk - 1) / a.nblk, g.Hkv, g.B);
     cfg.blockDim = dim3(kThreads);
